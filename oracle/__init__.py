@@ -60,8 +60,8 @@ def _load():
         Dbl = ctypes.c_double
         lib.oracle_attn_fwd.argtypes = [P, P, P, P, P, I64, I64, I64, I64, I, Dbl, I]
         lib.oracle_attn_fwd_rows.argtypes = [P, P, P, I64, I64, I, Dbl, P, P, I64, P, P, I]
-        lib.oracle_attn_bwd.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I64, I, Dbl, I]
-        lib.oracle_attn_bwd_rows.argtypes = [P, P, P, P, I64, I64, I, Dbl, P, P, I64, P,
+        lib.oracle_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, I64, I64, I64, I64, I, Dbl, I]
+        lib.oracle_attn_bwd_rows.argtypes = [P, P, P, P, P, I64, I64, I, Dbl, P, P, I64, P,
                                              P, P, I64, P, P, I]
         lib.oracle_nw.argtypes = [P, I64, P, P, I64, Dbl, P, I]
         lib.oracle_max_threads.argtypes = []
@@ -136,32 +136,41 @@ def attn_fwd_rows(q, k, v, heads, rows, causal: bool = True, scale: float | None
 
 
 def attn_bwd(q, k, v, dout, causal: bool = True, scale: float | None = None,
-             threads: int = 0, allow_underflow: bool = False):
+             threads: int = 0, allow_underflow: bool = False, out=None):
     """Backward for upstream gradient dout (dout = out for loss = 1/2 sum out^2).
-    Returns (dq, dk, dv), each [B,H,N,D] float64."""
+    Delta_i = dout_i . out_i is evaluated on ``out`` when given (the stored
+    forward output a backward pass receives), else on the oracle's own
+    float64 output.  Returns (dq, dk, dv), each [B,H,N,D] float64."""
     q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
     B, H, N, D = q.shape
+    given = None if out is None else _f64(out)
     scale = default_scale(D) if scale is None else float(scale)
     dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
-    rc = _load().oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk),
-                                 _ptr(dv), B, H, N, D, int(bool(causal)), scale, int(threads))
+    rc = _load().oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout),
+                                 ctypes.c_void_p(None) if given is None else _ptr(given),
+                                 _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, D, int(bool(causal)),
+                                 scale, int(threads))
     _check(rc, allow_underflow)
     return dq, dk, dv
 
 
 def attn_bwd_rows(q, k, v, dout, qheads, qrows, kheads, krows, causal: bool = True,
                   scale: float | None = None, threads: int = 0,
-                  allow_underflow: bool = False):
+                  allow_underflow: bool = False, out=None):
     """Backward at sampled rows: dq at (qheads, qrows), dk and dv at
-    (kheads, krows).  Returns (dq [nq, D], dk [nk, D], dv [nk, D])."""
+    (kheads, krows); ``out`` as in attn_bwd.  Returns (dq [nq, D], dk [nk, D],
+    dv [nk, D])."""
     q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    given = None if out is None else _f64(out)
     B, H, N, D = q.shape
     qheads, qrows, kheads, krows = _i64(qheads), _i64(qrows), _i64(kheads), _i64(krows)
     scale = default_scale(D) if scale is None else float(scale)
     dq = np.empty((qheads.size, D), dtype=np.float64)
     dk = np.empty((kheads.size, D), dtype=np.float64)
     dv = np.empty((kheads.size, D), dtype=np.float64)
-    rc = _load().oracle_attn_bwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), N, D,
+    rc = _load().oracle_attn_bwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(dout),
+                                      ctypes.c_void_p(None) if given is None else _ptr(given),
+                                      N, D,
                                       int(bool(causal)), scale, _ptr(qheads), _ptr(qrows),
                                       qheads.size, _ptr(dq), _ptr(kheads), _ptr(krows),
                                       kheads.size, _ptr(dk), _ptr(dv), int(threads))

@@ -195,20 +195,28 @@ int oracle_attn_fwd_rows(const double* q, const double* k, const double* v,
  *   dK_j  = scale * sum_{i: j in J(i)} dS_ij q_i
  * Phase 1 (per row i): m_i, z_i, out_i, Delta_i and dQ_i.
  * Phase 2 (per key j): dK_j and dV_j, summing over the rows i that see j.
- * Every sum runs over existing pairs only.
+ * Every sum runs over existing pairs only.  Delta is the streaming form
+ * dout_i . out_i; a caller may pass the stored forward output (what a
+ * backward pass is given) for it, otherwise the oracle's own float64 out_i
+ * is used.  On exact inputs both equal sum_j P_ij dP_ij.
  */
 
-/* Phase-1 work for one row; stats = {m, z, Delta}. */
+/*
+ * Phase-1 work for one row; stats = {m, z, Delta}.  Delta_i is evaluated on
+ * the given output row when `given` is non-NULL (the stored forward output a
+ * backward pass receives), else on this oracle's own float64 out_i.
+ */
 static int bwd_row(const double* qbh, const double* kbh, const double* vbh,
-                   const double* dobh, int64_t i, int64_t N, int64_t D,
-                   int causal, double scale, double* w, double* out_i,
+                   const double* dobh, const double* given_bh, int64_t i, int64_t N,
+                   int64_t D, int causal, double scale, double* w, double* out_i,
                    double* stats, double* dq_i) {
     double m, z;
     int u = row_forward(qbh + i * D, kbh, vbh, i, N, D, causal, scale, w, &m, &z,
                         out_i, NULL);
     const double* doi = dobh + i * D;
+    const double* oi = given_bh ? given_bh + i * D : out_i;
     double delta = 0.0;
-    for (int64_t d = 0; d < D; ++d) delta += doi[d] * out_i[d];
+    for (int64_t d = 0; d < D; ++d) delta += doi[d] * oi[d];
     stats[0] = m;
     stats[1] = z;
     stats[2] = delta;
@@ -259,9 +267,10 @@ static void bwd_key(const double* qbh, const double* kbh, const double* vbh,
     for (int64_t d = 0; d < D; ++d) dk_j[d] *= scale;
 }
 
+/* out_given: NULL, or the stored forward output [B,H,N,D] for Delta. */
 int oracle_attn_bwd(const double* q, const double* k, const double* v,
-                    const double* dout, double* dq, double* dk, double* dv,
-                    int64_t B, int64_t H, int64_t N, int64_t D, int causal,
+                    const double* dout, const double* out_given, double* dq, double* dk,
+                    double* dv, int64_t B, int64_t H, int64_t N, int64_t D, int causal,
                     double scale, int nthreads) {
     if (!q || !k || !v || !dout || !dq || !dk || !dv || B < 0 || H < 0 || N < 0 || D <= 0)
         return OR_EINVAL;
@@ -281,8 +290,8 @@ int oracle_attn_bwd(const double* q, const double* k, const double* v,
             if (!w || !out_i) continue;
             int64_t bh = r / N, i = r % N;
             int u = bwd_row(q + bh * N * D, k + bh * N * D, v + bh * N * D,
-                            dout + bh * N * D, i, N, D, causal, scale, w, out_i,
-                            stats + r * 3, dq + r * D);
+                            dout + bh * N * D, out_given ? out_given + bh * N * D : NULL, i,
+                            N, D, causal, scale, w, out_i, stats + r * 3, dq + r * D);
             if (u) {
 #pragma omp atomic write
                 status = OR_UNDERFLOW;
@@ -309,7 +318,8 @@ int oracle_attn_bwd(const double* q, const double* k, const double* v,
  * only.  dq_s is [nq, D]; dk_s, dv_s are [nk, D].
  */
 int oracle_attn_bwd_rows(const double* q, const double* k, const double* v,
-                         const double* dout, int64_t N, int64_t D, int causal,
+                         const double* dout, const double* out_given, int64_t N, int64_t D,
+                         int causal,
                          double scale, const int64_t* qheads, const int64_t* qrows,
                          int64_t nq, double* dq_s, const int64_t* kheads,
                          const int64_t* krows, int64_t nk, double* dk_s,
@@ -328,8 +338,8 @@ int oracle_attn_bwd_rows(const double* q, const double* k, const double* v,
                 int64_t bh = qheads[t];
                 double st[3];
                 int u = bwd_row(q + bh * N * D, k + bh * N * D, v + bh * N * D,
-                                dout + bh * N * D, qrows[t], N, D, causal, scale, w,
-                                out_i, st, dq_s + t * D);
+                                dout + bh * N * D, out_given ? out_given + bh * N * D : NULL,
+                                qrows[t], N, D, causal, scale, w, out_i, st, dq_s + t * D);
                 if (u) {
 #pragma omp atomic write
                     status = OR_UNDERFLOW;
@@ -352,8 +362,8 @@ int oracle_attn_bwd_rows(const double* q, const double* k, const double* v,
             for (int64_t i = i0; i < N; ++i) {
                 if (!w || !out_i) continue;
                 int u = bwd_row(q + bh * N * D, k + bh * N * D, v + bh * N * D,
-                                dout + bh * N * D, i, N, D, causal, scale, w, out_i,
-                                stats + i * 3, NULL);
+                                dout + bh * N * D, out_given ? out_given + bh * N * D : NULL,
+                                i, N, D, causal, scale, w, out_i, stats + i * 3, NULL);
                 if (u) {
 #pragma omp atomic write
                     status = OR_UNDERFLOW;

@@ -355,3 +355,28 @@ def test_nw_all_weights_underflow_is_nan():
     got = oracle.nw_regrid(np.array([[100.0, 100.0]]), np.array([[0.0, 0.0]]),
                            np.array([1.0]))
     assert np.isnan(got[0])
+
+
+def test_delta_on_a_given_output_moves_gradients_by_the_closed_form():
+    """Delta_i = dout_i . out_i evaluated on a given (stored) output: a change
+    E of that output shifts Delta by delta_i = dout_i . E_i, which moves
+    dq_i by -scale delta_i (P K)_i and dk_j by -scale sum_i P_ij delta_i q_i,
+    and leaves dv unchanged.  P comes from the forward with V = identity."""
+    N, D = 48, 64
+    q, k, v = _rng_qkv(13, 1, 1, N, D)
+    for causal in (True, False):
+        out, _ = oracle.attn_fwd(q, k, v, causal=causal)
+        eye = np.zeros((1, 1, N, D))
+        eye[0, 0, np.arange(N), np.arange(N)] = 1.0
+        P = oracle.attn_fwd(q, k, eye, causal=causal)[0][0, 0, :, :N]
+        E = np.random.default_rng(14).normal(size=out.shape) * 1e-2
+        dq0, dk0, dv0 = oracle.attn_bwd(q, k, v, out, causal=causal)
+        dq1, dk1, dv1 = oracle.attn_bwd(q, k, v, out, causal=causal, out=out + E)
+        dq2, dk2, dv2 = oracle.attn_bwd(q, k, v, out, causal=causal, out=out)
+        assert np.array_equal(dq0, dq2) and np.array_equal(dk0, dk2) and np.array_equal(dv0, dv2)
+        delta = (out[0, 0] * E[0, 0]).sum(axis=1)
+        assert np.array_equal(dv0, dv1)
+        want_dq = -(delta[:, None] * (P @ k[0, 0])) / 8.0
+        want_dk = -(P.T @ (delta[:, None] * q[0, 0])) / 8.0
+        assert np.abs((dq1 - dq0)[0, 0] - want_dq).max() < 1e-12
+        assert np.abs((dk1 - dk0)[0, 0] - want_dk).max() < 1e-12
