@@ -1,0 +1,270 @@
+// swa_api.cu -- the C ABI of libswa.so (include/swa.h): argument checks,
+// workspace carving, per-head dispatch and the device error word.  No
+// allocation happens here: every buffer, workspaces included, is the
+// caller's.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "swa_internal.cuh"
+#include "attn_tc.cuh"
+
+// Device error word: kernels whose bounded waits run out record a code here
+// (first writer wins) instead of trapping; swa_get_device_error() reports
+// and clears it.
+static __device__ unsigned g_swa_error_word;
+
+namespace {
+
+thread_local char t_msg[512];
+thread_local int t_launches;
+
+swa_status fail(swa_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_msg, sizeof(t_msg), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+swa_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(SWA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return p != nullptr && ((uintptr_t)p & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Device address of g_swa_error_word for the current device (host code may
+// not take the symbol's address directly).
+unsigned* device_error_word(swa_status* st) {
+  static std::mutex mu;
+  static unsigned* cache[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 64) {
+    *st = cuda_fail(e == cudaSuccess ? cudaErrorInvalidDevice : e, "cudaGetDevice");
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_swa_error_word);
+    if (e != cudaSuccess) {
+      *st = cuda_fail(e, "cudaGetSymbolAddress(error word)");
+      return nullptr;
+    }
+    cache[dev] = static_cast<unsigned*>(p);
+  }
+  *st = SWA_OK;
+  return cache[dev];
+}
+
+constexpr int64_t kMaxElems = (int64_t)1 << 40;
+
+swa_status check_attn_shape(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtype dt) {
+  if (dt != SWA_F32 && dt != SWA_BF16) return fail(SWA_ERR_INVALID_ARGUMENT, "unknown dtype %d", (int)dt);
+  if (B < 1 || H < 1 || N < 1) return fail(SWA_ERR_INVALID_ARGUMENT, "B, H, N must be >= 1 (got %lld, %lld, %lld)",
+                                           (long long)B, (long long)H, (long long)N);
+  if (D != 64) return fail(SWA_ERR_UNSUPPORTED, "only D = 64 is implemented (got %lld)", (long long)D);
+  if (B * H > 65535) return fail(SWA_ERR_UNSUPPORTED, "B*H must be <= 65535 (got %lld)", (long long)(B * H));
+  if (N > ((int64_t)1 << 30)) return fail(SWA_ERR_UNSUPPORTED, "N must be <= 2^30 (got %lld)", (long long)N);
+  if (B * H * N > kMaxElems / D) return fail(SWA_ERR_UNSUPPORTED, "tensor too large");
+  return SWA_OK;
+}
+
+size_t fwd_ws(int64_t B, int64_t H, swa_dtype dt) {
+  return dt == SWA_BF16 ? round_up((size_t)(B * H) * sizeof(int), 256) : 0;
+}
+
+struct BwdWs {
+  size_t flags, delta, dqacc, total;
+};
+
+BwdWs bwd_ws(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtype dt) {
+  BwdWs w;
+  w.flags = round_up((size_t)(B * H) * sizeof(int), 256);
+  w.delta = round_up((size_t)(B * H * N) * sizeof(float), 256);
+  w.dqacc = dt == SWA_BF16 ? round_up((size_t)(B * H * N * D) * sizeof(float), 256) : 0;
+  w.total = w.flags + w.delta + w.dqacc;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t swa_attn_fwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtype dt) {
+  (void)N;
+  (void)D;
+  if (B < 1 || H < 1) return 0;
+  return fwd_ws(B, H, dt);
+}
+
+swa_status swa_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                        int64_t B, int64_t H, int64_t N, int64_t D, int causal,
+                        swa_dtype dt, void* workspace, size_t workspace_bytes, void* stream) {
+  t_msg[0] = 0;
+  t_launches = 0;
+  swa_status st = check_attn_shape(B, H, N, D, dt);
+  if (st != SWA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return fail(SWA_ERR_INVALID_ARGUMENT, "q, k, v, out, lse must be non-null and 16-byte aligned");
+  const size_t need = fwd_ws(B, H, dt);
+  if (need && (!aligned16(workspace) || workspace_bytes < need))
+    return fail(SWA_ERR_INVALID_ARGUMENT, "workspace must be 16-byte aligned and >= %zu bytes", need);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t BH = B * H;
+  const float scale = 1.0f / sqrtf((float)D);
+  unsigned* err = device_error_word(&st);
+  if (!err) return st;
+  int launches = 0;
+  cudaError_t e;
+  if (dt == SWA_F32) {
+    e = swa::launch_attn_fwd_simt(dt, q, k, v, out, lse, BH, N, causal ? 1 : 0, scale, nullptr,
+                                  0, s, &launches);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_simt");
+  } else {
+    int* flags = static_cast<int*>(workspace);
+    e = cudaMemsetAsync(flags, 0, (size_t)BH * sizeof(int), s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(flags)");
+    e = swa::launch_scan_nonfinite(dt, v, BH, N * D, flags, s, &launches);
+    if (e != cudaSuccess) return cuda_fail(e, "scan_nonfinite(v)");
+    // Heads whose V is all finite: tensor-core kernel.  Heads holding a
+    // non-finite value: the pair-by-pair kernel, so masked pairs stay absent.
+    e = swa::launch_attn_fwd_tc(q, k, v, out, lse, B, H, N, causal ? 1 : 0, scale, flags, err,
+                                s, &launches);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_tc");
+    e = swa::launch_attn_fwd_simt(dt, q, k, v, out, lse, BH, N, causal ? 1 : 0, scale, flags,
+                                  1, s, &launches);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_simt(non-finite heads)");
+  }
+  t_launches = launches;
+  return SWA_OK;
+}
+
+size_t swa_attn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtype dt) {
+  if (B < 1 || H < 1 || N < 1 || D < 1) return 0;
+  return bwd_ws(B, H, N, D, dt).total;
+}
+
+swa_status swa_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                        int64_t B, int64_t H, int64_t N, int64_t D, int causal, swa_dtype dt,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  t_msg[0] = 0;
+  t_launches = 0;
+  swa_status st = check_attn_shape(B, H, N, D, dt);
+  if (st != SWA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return fail(SWA_ERR_INVALID_ARGUMENT,
+                "q, k, v, out, dout, lse, dq, dk, dv must be non-null and 16-byte aligned");
+  const BwdWs ws = bwd_ws(B, H, N, D, dt);
+  if (!aligned16(workspace) || workspace_bytes < ws.total)
+    return fail(SWA_ERR_INVALID_ARGUMENT, "workspace must be 16-byte aligned and >= %zu bytes",
+                ws.total);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t BH = B * H;
+  const float scale = 1.0f / sqrtf((float)D);
+  unsigned* err = device_error_word(&st);
+  if (!err) return st;
+  char* base = static_cast<char*>(workspace);
+  int* flags = reinterpret_cast<int*>(base);
+  float* delta = reinterpret_cast<float*>(base + ws.flags);
+  float* dqacc = reinterpret_cast<float*>(base + ws.flags + ws.delta);
+  const int c = causal ? 1 : 0;
+  int launches = 0;
+  cudaError_t e = swa::launch_attn_bwd_prep(dt, out, dout, delta, BH * N, s, &launches);
+  if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_prep");
+  if (dt == SWA_F32) {
+    e = swa::launch_attn_bwd_simt(dt, q, k, v, dout, lse, delta, dq, dk, dv, BH, N, c, scale,
+                                  nullptr, 0, s, &launches);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_simt");
+  } else {
+    e = cudaMemsetAsync(flags, 0, (size_t)BH * sizeof(int), s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(flags)");
+    e = swa::launch_scan_nonfinite(dt, v, BH, N * D, flags, s, &launches);
+    if (e != cudaSuccess) return cuda_fail(e, "scan_nonfinite(v)");
+    e = swa::launch_scan_nonfinite(dt, dout, BH, N * D, flags, s, &launches);
+    if (e != cudaSuccess) return cuda_fail(e, "scan_nonfinite(dout)");
+    e = swa::launch_attn_bwd_tc(q, k, v, dout, lse, delta, dq, dk, dv, dqacc, B, H, N, c, scale,
+                                flags, err, s, &launches);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_tc");
+    e = swa::launch_attn_bwd_simt(dt, q, k, v, dout, lse, delta, dq, dk, dv, BH, N, c, scale,
+                                  flags, 1, s, &launches);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_simt(non-finite heads)");
+  }
+  t_launches = launches;
+  return SWA_OK;
+}
+
+size_t swa_nw_workspace_size(int64_t M, int64_t S) {
+  if (M < 1 || S < 1) return 0;
+  return round_up(swa::nw_partials_bytes(M, S, 148), 256);
+}
+
+swa_status swa_nw_regrid(const float* targets, int64_t M, const float* sources,
+                         const float* vals, int64_t S, float h, float* out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  t_msg[0] = 0;
+  t_launches = 0;
+  if (M < 1 || S < 1)
+    return fail(SWA_ERR_INVALID_ARGUMENT, "M and S must be >= 1 (got %lld, %lld)", (long long)M,
+                (long long)S);
+  if (M > ((int64_t)1 << 31) || S > ((int64_t)1 << 31))
+    return fail(SWA_ERR_UNSUPPORTED, "M and S must be <= 2^31");
+  if (!(h > 0.f) || !isfinite(h))
+    return fail(SWA_ERR_INVALID_ARGUMENT, "bandwidth h must be finite and > 0");
+  if (!aligned16(targets) || !aligned16(sources) || !aligned16(vals) || !aligned16(out))
+    return fail(SWA_ERR_INVALID_ARGUMENT,
+                "targets, sources, vals, out must be non-null and 16-byte aligned");
+  const size_t need = swa_nw_workspace_size(M, S);
+  if (!aligned16(workspace) || workspace_bytes < need)
+    return fail(SWA_ERR_INVALID_ARGUMENT, "workspace must be 16-byte aligned and >= %zu bytes",
+                need);
+  int launches = 0;
+  cudaError_t e = swa::launch_nw_regrid(targets, M, sources, vals, S, h, out,
+                                        static_cast<float*>(workspace), 148,
+                                        static_cast<cudaStream_t>(stream), &launches);
+  if (e != cudaSuccess) return cuda_fail(e, "nw_regrid");
+  t_launches = launches;
+  return SWA_OK;
+}
+
+swa_status swa_get_device_error(void* stream) {
+  t_msg[0] = 0;
+  swa_status st;
+  unsigned* err = device_error_word(&st);
+  if (!err) return st;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned word = 0;
+  e = cudaMemcpy(&word, err, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read error word");
+  if (word != 0) {
+    const unsigned zero = 0;
+    e = cudaMemcpy(err, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "clear error word");
+    return fail(SWA_ERR_DEVICE_TIMEOUT, "a kernel gave up a bounded wait (device code %u)", word);
+  }
+  return SWA_OK;
+}
+
+const char* swa_status_string(swa_status status) {
+  switch (status) {
+    case SWA_OK: return "SWA_OK";
+    case SWA_ERR_INVALID_ARGUMENT: return "SWA_ERR_INVALID_ARGUMENT";
+    case SWA_ERR_UNSUPPORTED: return "SWA_ERR_UNSUPPORTED";
+    case SWA_ERR_CUDA: return "SWA_ERR_CUDA";
+    case SWA_ERR_DEVICE_TIMEOUT: return "SWA_ERR_DEVICE_TIMEOUT";
+  }
+  return "SWA_ERR_UNKNOWN";
+}
+
+const char* swa_last_error_message(void) { return t_msg; }
+
+int swa_last_launch_count(void) { return t_launches; }
+
+}  // extern "C"

@@ -1,0 +1,69 @@
+// swa_internal.cuh -- declarations shared by the translation units of
+// libswa.so (launchers, device helpers).  Not part of the public ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/swa.h"
+
+namespace swa {
+
+// Error codes a kernel writes into the device error word (first writer wins).
+enum DeviceError : unsigned {
+  kDevOk = 0,
+  kDevTimeoutFull = 1,   // a wait for a "full" (data landed) barrier ran out
+  kDevTimeoutEmpty = 2,  // a wait for an "empty" (slot released) barrier ran out
+  kDevTimeoutMma = 3,    // a wait for an MMA completion ran out
+  kDevTimeoutOther = 4,
+};
+
+__host__ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// Device-side element conversion.
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Per-head selection: a kernel given `flags` handles head h only when
+// (flags[h] != 0) == select; with flags == nullptr it handles every head.
+__device__ __forceinline__ bool head_selected(const int* flags, int64_t head, int select) {
+  return flags == nullptr || ((flags[head] != 0) == (select != 0));
+}
+
+// ---------------------------------------------------------------- launchers
+// Each returns the launch's cudaError_t and adds the number of kernels it
+// enqueued to *launches.
+
+cudaError_t launch_scan_nonfinite(swa_dtype dt, const void* x, int64_t heads,
+                                  int64_t elems_per_head, int* flags, cudaStream_t s,
+                                  int* launches);
+
+cudaError_t launch_attn_fwd_simt(swa_dtype dt, const void* q, const void* k, const void* v,
+                                 void* out, float* lse, int64_t BH, int64_t N, int causal,
+                                 float scale, const int* flags, int select, cudaStream_t s,
+                                 int* launches);
+
+cudaError_t launch_attn_bwd_prep(swa_dtype dt, const void* out, const void* dout,
+                                 float* delta, int64_t rows, cudaStream_t s, int* launches);
+
+cudaError_t launch_attn_bwd_simt(swa_dtype dt, const void* q, const void* k, const void* v,
+                                 const void* dout, const float* lse, const float* delta,
+                                 void* dq, void* dk, void* dv, int64_t BH, int64_t N,
+                                 int causal, float scale, const int* flags, int select,
+                                 cudaStream_t s, int* launches);
+
+size_t nw_partials_bytes(int64_t M, int64_t S, int sm_count);
+cudaError_t launch_nw_regrid(const float* targets, int64_t M, const float* sources,
+                             const float* vals, int64_t S, float h, float* out,
+                             float* partials, int sm_count, cudaStream_t s, int* launches);
+
+}  // namespace swa

@@ -1,0 +1,191 @@
+"""Thin ctypes binding of libswa.so (C ABI in include/swa.h).
+
+Argument marshalling only: every step of the computation runs in the
+library's CUDA kernels.  torch provides device memory (outputs and
+workspaces are torch tensors) and the current CUDA stream.  If the library
+has not been built, or no CUDA device is present, calls raise instead of
+falling back to anything else.
+
+Function names follow the C ABI: ``attn_fwd`` -> ``swa_attn_fwd`` and so on.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libswa.so")
+
+SWA_OK, SWA_ERR_INVALID_ARGUMENT, SWA_ERR_UNSUPPORTED, SWA_ERR_CUDA, SWA_ERR_DEVICE_TIMEOUT = range(5)
+SWA_F32, SWA_BF16 = 0, 1
+
+# Every symbol include/swa.h declares.
+EXPORTS = (
+    "swa_attn_fwd_workspace_size", "swa_attn_fwd", "swa_attn_bwd_workspace_size",
+    "swa_attn_bwd", "swa_nw_workspace_size", "swa_nw_regrid", "swa_get_device_error",
+    "swa_status_string", "swa_last_error_message", "swa_last_launch_count",
+)
+
+
+class SwaError(RuntimeError):
+    def __init__(self, status: int, where: str, message: str):
+        super().__init__(f"{where}: status {status} ({_status_name(status)}): {message}")
+        self.status = status
+
+
+_lib = None
+
+
+def _status_name(st: int) -> str:
+    names = ["SWA_OK", "SWA_ERR_INVALID_ARGUMENT", "SWA_ERR_UNSUPPORTED", "SWA_ERR_CUDA",
+             "SWA_ERR_DEVICE_TIMEOUT"]
+    return names[st] if 0 <= st < len(names) else f"unknown({st})"
+
+
+def load_library():
+    """Load libswa.so with ctypes (no CUDA work).  Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m causal_attention_swa_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I64, I, SZ, F = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t,
+                        ctypes.c_float)
+    lib.swa_attn_fwd_workspace_size.argtypes = [I64, I64, I64, I64, I]
+    lib.swa_attn_fwd_workspace_size.restype = SZ
+    lib.swa_attn_fwd.argtypes = [P, P, P, P, P, I64, I64, I64, I64, I, I, P, SZ, P]
+    lib.swa_attn_fwd.restype = I
+    lib.swa_attn_bwd_workspace_size.argtypes = [I64, I64, I64, I64, I]
+    lib.swa_attn_bwd_workspace_size.restype = SZ
+    lib.swa_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I64, I64, I64, I64, I, I, P, SZ, P]
+    lib.swa_attn_bwd.restype = I
+    lib.swa_nw_workspace_size.argtypes = [I64, I64]
+    lib.swa_nw_workspace_size.restype = SZ
+    lib.swa_nw_regrid.argtypes = [P, I64, P, P, I64, F, P, P, SZ, P]
+    lib.swa_nw_regrid.restype = I
+    lib.swa_get_device_error.argtypes = [P]
+    lib.swa_get_device_error.restype = I
+    lib.swa_status_string.argtypes = [I]
+    lib.swa_status_string.restype = ctypes.c_char_p
+    lib.swa_last_error_message.argtypes = []
+    lib.swa_last_error_message.restype = ctypes.c_char_p
+    lib.swa_last_launch_count.argtypes = []
+    lib.swa_last_launch_count.restype = I
+    _lib = lib
+    return lib
+
+
+def _check(st: int, where: str) -> None:
+    if st != SWA_OK:
+        msg = load_library().swa_last_error_message().decode(errors="replace")
+        raise SwaError(st, where, msg)
+
+
+def _stream_ptr(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SWA_BF16
+    if t.dtype == torch.float32:
+        return SWA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}: bfloat16 or float32")
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if not (isinstance(t, torch.Tensor) and t.is_cuda and t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def last_launch_count() -> int:
+    """Kernels the last successful call on this thread enqueued."""
+    return int(load_library().swa_last_launch_count())
+
+
+def attn_fwd_workspace_size(B, H, N, D, dtype_code) -> int:
+    return int(load_library().swa_attn_fwd_workspace_size(B, H, N, D, dtype_code))
+
+
+def attn_bwd_workspace_size(B, H, N, D, dtype_code) -> int:
+    return int(load_library().swa_attn_bwd_workspace_size(B, H, N, D, dtype_code))
+
+
+def nw_workspace_size(M, S) -> int:
+    return int(load_library().swa_nw_workspace_size(M, S))
+
+
+def _workspace(nbytes: int, device, ws):
+    if nbytes == 0:
+        return None
+    if ws is not None and ws.numel() * ws.element_size() >= nbytes:
+        return ws
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def attn_fwd(q, k, v, causal: bool = True, out=None, lse=None, workspace=None):
+    """swa_attn_fwd: q, k, v [B,H,N,64] bf16 or fp32 CUDA tensors ->
+    (out [B,H,N,64] same dtype, lse [B,H,N] fp32)."""
+    lib = load_library()
+    _require_cuda(q, k, v)
+    B, H, N, D = q.shape
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _require_cuda(out, lse)
+    nbytes = attn_fwd_workspace_size(B, H, N, D, dt)
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib.swa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, D,
+                          int(bool(causal)), dt, _ptr(ws), nbytes, _stream_ptr(q.device))
+    _check(st, "swa_attn_fwd")
+    return out, lse
+
+
+def attn_bwd(q, k, v, out, dout, lse, causal: bool = True, dq=None, dk=None, dv=None,
+             workspace=None):
+    """swa_attn_bwd -> (dq, dk, dv), each [B,H,N,64] of q's dtype."""
+    lib = load_library()
+    _require_cuda(q, k, v, out, dout, lse)
+    B, H, N, D = q.shape
+    dt = _dtype_code(q)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    nbytes = attn_bwd_workspace_size(B, H, N, D, dt)
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib.swa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                          _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, D, int(bool(causal)), dt,
+                          _ptr(ws), nbytes, _stream_ptr(q.device))
+    _check(st, "swa_attn_bwd")
+    return dq, dk, dv
+
+
+def nw_regrid(targets, sources, vals, h: float = 0.5, out=None, workspace=None):
+    """swa_nw_regrid: targets [M,2], sources [S,2], vals [S] fp32 -> out [M] fp32."""
+    lib = load_library()
+    _require_cuda(targets, sources, vals)
+    M, S = targets.shape[0], sources.shape[0]
+    out = torch.empty((M,), dtype=torch.float32, device=targets.device) if out is None else out
+    nbytes = nw_workspace_size(M, S)
+    ws = _workspace(nbytes, targets.device, workspace)
+    st = lib.swa_nw_regrid(_ptr(targets), M, _ptr(sources), _ptr(vals), S, float(h), _ptr(out),
+                           _ptr(ws), nbytes, _stream_ptr(targets.device))
+    _check(st, "swa_nw_regrid")
+    return out
+
+
+def get_device_error(device=None) -> int:
+    """swa_get_device_error on the current stream: returns the status."""
+    dev = torch.device("cuda") if device is None else device
+    return int(load_library().swa_get_device_error(_stream_ptr(dev)))

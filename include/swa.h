@@ -1,0 +1,150 @@
+/*
+ * swa.h -- C ABI of libswa.so: the fused softmax-weighted average on B200
+ * (sm_100a).  Two instances of one operation, "a softmax-weighted average
+ * whose scores come from a join":
+ *
+ *   causal attention   out_i = sum_{j in J(i)} softmax_j(q_i . k_j * scale) v_j
+ *   Nadaraya-Watson    out_p = sum_q w_pq v_q / sum_q w_pq,
+ *                      w_pq = exp(-|t_p - s_q|^2 / h^2)
+ *
+ * Definitions: "Show HN: Automatic deduction of FlashAttention kernel from
+ * ~25 lines of SQL" (page 2), demo script 01_attention.py -- views
+ * ATTENTION_WINDOW / ATTENTION_GROUP_BY (forward), query GRADIENT (backward
+ * of loss = 1/2 sum out^2), query NADARAYA_WATSON (regrid), and
+ * check_masks_are_absent_rows (mask semantics).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor arguments are DEVICE pointers owned by the caller; the
+ *     library never allocates, frees or retains them.  Every pointer must be
+ *     16-byte aligned.
+ *   - Attention tensors are contiguous row-major [B, H, N, D] ("(t, d)"
+ *     matrices per head, ordered by t then d as the FORWARD query orders
+ *     them); lse and delta are [B, H, N] float32.
+ *   - J(i) = {0 .. i} when causal != 0 (the join predicate q.t >= k.t,
+ *     diagonal included), else {0 .. N-1}.  scale = 1/sqrt(D) = 1/8 at D = 64.
+ *   - Masked pairs are absent: a pair (i, j) with j > i is never used in a
+ *     product.  A +inf (or -inf, NaN) in V therefore reaches exactly the
+ *     queries i with j in J(i), per IEEE rules, and never turns into a NaN
+ *     elsewhere.  Q and K must be finite.
+ *   - All work is enqueued asynchronously on `stream` (a cudaStream_t; NULL
+ *     is the legacy default stream).  Argument errors are detected on the
+ *     host and returned before anything is enqueued.  A device-side
+ *     failure (a bounded wait that ran out) is recorded in a device error
+ *     word and reported by swa_get_device_error().
+ *   - Workspaces are caller-owned device buffers of at least the size the
+ *     matching *_workspace_size() returns (0 means none is needed, and
+ *     `workspace` may then be NULL).  Their contents on entry do not matter;
+ *     they must not be shared by calls that can run concurrently.
+ *   - Thread safety: entry points may be called from several host threads
+ *     on different streams; swa_last_error_message() is per host thread.
+ */
+#ifndef SWA_H_
+#define SWA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SWA_OK = 0,
+    SWA_ERR_INVALID_ARGUMENT = 1, /* null/misaligned pointer, bad size, small workspace */
+    SWA_ERR_UNSUPPORTED = 2,      /* a valid request this build does not implement */
+    SWA_ERR_CUDA = 3,             /* a CUDA runtime call failed (message has details) */
+    SWA_ERR_DEVICE_TIMEOUT = 4    /* a kernel's bounded wait ran out (device error word) */
+} swa_status;
+
+typedef enum {
+    SWA_F32 = 0,  /* float32 storage, float32 arithmetic on CUDA cores */
+    SWA_BF16 = 1  /* bfloat16 storage, tensor cores with float32 accumulation */
+} swa_dtype;
+
+/*
+ * Bytes of workspace swa_attn_fwd needs (one int32 flag per head for the
+ * bf16 path, 0 for float32).
+ */
+size_t swa_attn_fwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D,
+                                   swa_dtype dtype);
+
+/*
+ * Attention forward (views ATTENTION_WINDOW / ATTENTION_GROUP_BY; the
+ * FlashAttention plan the demo's docstring names: keys streamed past query
+ * blocks under a running row max and row sum, the N x N scores never
+ * stored).
+ *   q, k, v  [B,H,N,D] of `dtype`         (in)
+ *   out      [B,H,N,D] of `dtype`         (out)  out_i = sum_j P_ij v_j
+ *   lse      [B,H,N] float32              (out)  m_i + ln z_i (natural log)
+ *   B, H >= 1; N >= 1; D == 64.
+ * The bf16 path scans V for non-finite values; heads that hold one are
+ * computed by the exact pair-by-pair kernel so that masked pairs stay
+ * absent, the others by the tensor-core kernel.
+ */
+swa_status swa_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                        float* lse, int64_t B, int64_t H, int64_t N, int64_t D,
+                        int causal, swa_dtype dtype, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/*
+ * Bytes of workspace swa_attn_bwd needs: per-head flags, delta [B,H,N]
+ * float32 and, for bf16, a float32 dQ accumulator [B,H,N,D].
+ */
+size_t swa_attn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D,
+                                   swa_dtype dtype);
+
+/*
+ * Attention backward (query GRADIENT: the gradient of a loss with respect
+ * to every value of q, k and v in one pass; with loss = 1/2 sum out^2 the
+ * upstream gradient dout equals out).
+ *   q, k, v, out, dout  [B,H,N,D] of `dtype`   (in)  out/lse from swa_attn_fwd
+ *   lse                 [B,H,N] float32        (in)
+ *   dq, dk, dv          [B,H,N,D] of `dtype`   (out)
+ * P_ij = exp(s_ij - lse_i); delta_i = sum_d dout_id out_id;
+ * dS_ij = P_ij (dout_i . v_j - delta_i); dq_i = scale sum_j dS_ij k_j;
+ * dk_j = scale sum_i dS_ij q_i; dv_j = sum_i P_ij dout_i (existing pairs only).
+ * V and dout may hold non-finite values (heads with one take the exact
+ * pair-by-pair kernel).
+ */
+swa_status swa_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                        int64_t B, int64_t H, int64_t N, int64_t D, int causal,
+                        swa_dtype dtype, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/* Bytes of workspace swa_nw_regrid needs for M targets and S sources. */
+size_t swa_nw_workspace_size(int64_t M, int64_t S);
+
+/*
+ * Nadaraya-Watson regrid (query NADARAYA_WATSON; "bandwidth h = 0.5" with
+ * divisor 0.25 = h^2):
+ *   targets [M,2] float32 (x, y)   sources [S,2] float32 (x, y)   vals [S] float32
+ *   out     [M] float32            out_p = sum_q w_pq v_q / sum_q w_pq
+ *   w_pq = exp(-((tx-sx)^2 + (ty-sy)^2) / h^2), h > 0.  M, S >= 1.
+ * If every weight of a target underflows, out_p is NaN (0/0).
+ */
+swa_status swa_nw_regrid(const float* targets, int64_t M, const float* sources,
+                         const float* vals, int64_t S, float h, float* out,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears this device's error word.
+ * Returns SWA_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait since
+ * the last call, SWA_ERR_CUDA if the synchronisation failed, else SWA_OK.
+ */
+swa_status swa_get_device_error(void* stream);
+
+/* Static string naming a status code. */
+const char* swa_status_string(swa_status status);
+
+/* Detail of the last failure on this host thread ("" if none). */
+const char* swa_last_error_message(void);
+
+/* Kernel launches the last successful call on this host thread enqueued. */
+int swa_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWA_H_ */

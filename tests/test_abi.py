@@ -1,0 +1,111 @@
+"""CPU-only checks of the C ABI: libswa.so loads, exports every symbol that
+include/swa.h declares, and rejects bad arguments on the host before any
+CUDA work (no compute call needs a GPU here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from causal_attention_swa_b200 import swa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "swa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return set(re.findall(r"\b(swa_[a-z0-9_]+)\s*\(", text))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from causal_attention_swa_b200 import build
+    build.build()
+    return swa.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _declared_symbols()
+    assert declared, "no declarations found in include/swa.h"
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert declared == set(swa.EXPORTS)
+
+
+def test_status_strings(lib):
+    assert lib.swa_status_string(0) == b"SWA_OK"
+    assert lib.swa_status_string(4) == b"SWA_ERR_DEVICE_TIMEOUT"
+
+
+def test_workspace_sizes(lib):
+    # bf16 forward: one int32 flag per head, rounded to 256 bytes
+    assert lib.swa_attn_fwd_workspace_size(2, 16, 16384, 64, swa.SWA_BF16) == 256
+    assert lib.swa_attn_fwd_workspace_size(1, 1, 256, 64, swa.SWA_F32) == 0
+    # bf16 backward: flags + delta + float32 dQ accumulator
+    B, H, N, D = 2, 16, 16384, 64
+    want = 256 + B * H * N * 4 + B * H * N * D * 4
+    assert lib.swa_attn_bwd_workspace_size(B, H, N, D, swa.SWA_BF16) == want
+    assert lib.swa_attn_bwd_workspace_size(1, 1, 256, 64, swa.SWA_F32) == 256 + 1024
+    assert lib.swa_nw_workspace_size(16384, 16384) > 0
+
+
+FAKE = 1 << 20  # a 16-byte aligned non-null address; never dereferenced
+
+
+@pytest.mark.parametrize("args,code", [
+    ((FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 32, 1, swa.SWA_BF16), swa.SWA_ERR_UNSUPPORTED),
+    ((FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1, 16, 64, 1, swa.SWA_BF16), swa.SWA_ERR_INVALID_ARGUMENT),
+    ((FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 64, 1, swa.SWA_BF16), swa.SWA_ERR_INVALID_ARGUMENT),
+    ((None, FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 64, 1, swa.SWA_BF16), swa.SWA_ERR_INVALID_ARGUMENT),
+    ((FAKE + 8, FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 64, 1, swa.SWA_BF16),
+     swa.SWA_ERR_INVALID_ARGUMENT),
+    ((FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 64, 1, 7), swa.SWA_ERR_INVALID_ARGUMENT),
+    ((FAKE, FAKE, FAKE, FAKE, FAKE, 300, 300, 16, 64, 1, swa.SWA_BF16), swa.SWA_ERR_UNSUPPORTED),
+])
+def test_fwd_argument_errors_return_before_launch(lib, args, code):
+    st = lib.swa_attn_fwd(*args, FAKE, 1 << 20, None)
+    assert st == code, lib.swa_last_error_message()
+    assert lib.swa_last_error_message() != b""
+
+
+def test_fwd_small_workspace_is_rejected(lib):
+    st = lib.swa_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 4, 16, 64, 1, swa.SWA_BF16,
+                          FAKE, 4, None)
+    assert st == swa.SWA_ERR_INVALID_ARGUMENT
+    assert b"workspace" in lib.swa_last_error_message()
+
+
+def test_bwd_argument_errors(lib):
+    good = [FAKE] * 9
+    st = lib.swa_attn_bwd(*good, 1, 1, 16, 64, 1, swa.SWA_BF16, FAKE, 16, None)
+    assert st == swa.SWA_ERR_INVALID_ARGUMENT  # workspace too small
+    bad = list(good)
+    bad[6] = None  # dq
+    st = lib.swa_attn_bwd(*bad, 1, 1, 16, 64, 1, swa.SWA_BF16, FAKE, 1 << 30, None)
+    assert st == swa.SWA_ERR_INVALID_ARGUMENT
+
+
+def test_nw_argument_errors(lib):
+    F = ctypes.c_float
+    assert lib.swa_nw_regrid(FAKE, 0, FAKE, FAKE, 4, F(0.5), FAKE, FAKE, 1 << 20, None) == \
+        swa.SWA_ERR_INVALID_ARGUMENT
+    assert lib.swa_nw_regrid(FAKE, 4, FAKE, FAKE, 4, F(0.0), FAKE, FAKE, 1 << 20, None) == \
+        swa.SWA_ERR_INVALID_ARGUMENT
+    assert lib.swa_nw_regrid(FAKE, 4, FAKE, FAKE, 4, F(float("nan")), FAKE, FAKE, 1 << 20,
+                             None) == swa.SWA_ERR_INVALID_ARGUMENT
+    assert lib.swa_nw_regrid(FAKE, 4, FAKE + 4, FAKE, 4, F(0.5), FAKE, FAKE, 1 << 20, None) == \
+        swa.SWA_ERR_INVALID_ARGUMENT
+    assert lib.swa_nw_regrid(FAKE, 4, FAKE, FAKE, 4, F(0.5), FAKE, FAKE, 8, None) == \
+        swa.SWA_ERR_INVALID_ARGUMENT
+
+
+def test_product_path_does_not_import_the_oracle():
+    """The CUDA binding never reaches the oracle (no CPU fallback)."""
+    pkg = os.path.join(ROOT, "causal_attention_swa_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "swa_oracle" not in text and "liboracle" not in text, f

@@ -1,0 +1,218 @@
+"""GPU parity of the attention path (through the C ABI) against the float64
+oracle, element by element.
+
+Workloads: the demo's own inputs ("Show HN: Automatic deduction of
+FlashAttention kernel from ~25 lines of SQL", main(): seed 0, 64 and 256
+tokens, D = 64) on the float32 path; the mask test of
+check_masks_are_absent_rows on both paths; small bf16 shapes that span
+several 128-row tiles with ragged tails; and the three large bf16 workloads
+(4x16x4096 forward, 2x16x16384 forward+backward, 1x8x65536 forward+backward
+with 0.01% of V set to +inf), checked at sampled rows against the oracle and
+everywhere through properties that hold at any size.
+Tolerances: tests/_compare.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from causal_attention_swa_b200 import inputs, swa
+from _compare import check_bf16, check_f32, check_lse, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def dev_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def dev_f32(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+
+def run_fwd_bwd(q, k, v, causal=True, backward=True):
+    out, lse = swa.attn_fwd(q, k, v, causal=causal)
+    grads = swa.attn_bwd(q, k, v, out, out, lse, causal=causal) if backward else None
+    torch.cuda.synchronize()
+    assert swa.get_device_error() == swa.SWA_OK
+    return out, lse, grads
+
+
+# ------------------------------------------------------------ float32 path
+
+@pytest.mark.parametrize("n", [64, 256])
+def test_f32_demo_inputs_forward_and_gradient(n):
+    q, k, v = (a[None, None] for a in inputs.pages_main()[n])
+    out, lse, (dq, dk, dv) = run_fwd_bwd(dev_f32(q), dev_f32(k), dev_f32(v))
+    w_out, w_lse = oracle.attn_fwd(q, k, v)
+    check_f32(out, w_out, "out")
+    check_f32(lse, w_lse, "lse")
+    w_dq, w_dk, w_dv = oracle.attn_bwd(q, k, v, w_out)
+    check_f32(dq, w_dq, "dq")
+    check_f32(dk, w_dk, "dk")
+    check_f32(dv, w_dv, "dv")
+
+
+def test_f32_single_head_inf_in_v():
+    """+inf at V[100, 3] of the 256-token draw: exact inf/NaN pattern of out
+    and of every gradient, finite entries within 1e-5."""
+    q, k, v = inputs.single_head_f64(256, inf_at=(100, 3))
+    out, lse, (dq, dk, dv) = run_fwd_bwd(dev_f32(q), dev_f32(k), dev_f32(v))
+    w_out, w_lse = oracle.attn_fwd(q, k, v)
+    check_f32(out, w_out, "out")
+    o = to_f64(out)[0, 0]
+    assert np.isfinite(o[:100]).all() and np.isposinf(o[100:, 3]).all()
+    check_f32(lse, w_lse, "lse")
+    w = oracle.attn_bwd(q, k, v, w_out)
+    for name, g, ww in zip(("dq", "dk", "dv"), (dq, dk, dv), w):
+        check_f32(g, ww, name)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_pages_mask_test(dtype):
+    """check_masks_are_absent_rows: n = 16, seed 1, V[9, 0] = +inf."""
+    q, k, v = inputs.pages_mask(16, 9)
+    if dtype == "f32":
+        tq, tk, tv = dev_f32(q), dev_f32(k), dev_f32(v)
+    else:
+        tq, tk, tv = (dev_bf16(inputs.bf16_bits(a.astype(np.float32))) for a in (q, k, v))
+    out, _, _ = run_fwd_bwd(tq, tk, tv, backward=False)
+    o = to_f64(out)[0, 0]
+    assert np.isfinite(o[:9]).all()
+    assert np.isposinf(o[9:, 0]).all()
+    assert np.isfinite(o[:, 1:]).all()
+
+
+# --------------------------------------------------------------- bf16 path
+
+def bf16_case(B, H, N, seed, std=1.0):
+    rng = np.random.default_rng(seed)
+    bits = [inputs.bf16_bits(std * rng.standard_normal((B, H, N, 64), dtype=np.float32))
+            for _ in range(3)]
+    return bits, [inputs.bf16_to_f64(b) for b in bits]
+
+
+@pytest.mark.parametrize("N", [1, 7, 64, 127, 128, 129, 255, 256, 257, 383, 640])
+@pytest.mark.parametrize("causal", [True, False])
+def test_bf16_small_shapes_forward_and_gradient(N, causal):
+    bits, (q, k, v) = bf16_case(2, 3, N, seed=N)
+    out, lse, (dq, dk, dv) = run_fwd_bwd(*(dev_bf16(b) for b in bits), causal=causal)
+    w_out, w_lse = oracle.attn_fwd(q, k, v, causal=causal)
+    check_bf16(out, w_out, "out")
+    check_lse(lse, w_lse, "lse")
+    # the gradient of 1/2 sum out^2 at the GPU's stored (bf16) output, which
+    # the backward is given: dout = out, and Delta is evaluated on it
+    w = oracle.attn_bwd(q, k, v, to_f64(out), causal=causal, out=to_f64(out))
+    for name, g, ww in zip(("dq", "dk", "dv"), (dq, dk, dv), w):
+        check_bf16(g, ww, name)
+
+
+def test_bf16_mixed_finite_and_nonfinite_heads():
+    """Heads with a non-finite V take the pair-by-pair kernel, the others the
+    tensor-core kernel; both must match the oracle, pattern included."""
+    bits, (q, k, v) = bf16_case(1, 4, 300, seed=42)
+    vb = bits[2].copy()
+    vb[0, 1, 200, 5] = 0x7F80   # +inf
+    vb[0, 3, 17, 60] = 0xFF80   # -inf
+    vb[0, 3, 250, 60] = 0x7F80  # +inf after -inf: NaN from row 250 on
+    v = inputs.bf16_to_f64(vb)
+    out, lse, (dq, dk, dv) = run_fwd_bwd(dev_bf16(bits[0]), dev_bf16(bits[1]), dev_bf16(vb))
+    w_out, w_lse = oracle.attn_fwd(q, k, v)
+    check_bf16(out, w_out, "out")
+    check_lse(lse, w_lse, "lse")
+    w = oracle.attn_bwd(q, k, v, to_f64(out), out=to_f64(out))
+    for name, g, ww in zip(("dq", "dk", "dv"), (dq, dk, dv), w):
+        check_bf16(g, ww, name)
+
+
+# ------------------------------------------------------ large bf16 workloads
+
+def sample_rows(rng, BH, N, n):
+    heads = rng.integers(0, BH, size=n)
+    rows = rng.integers(0, N, size=n)
+    fixed_rows = np.array([0, 1, 127, 128, 129, N - 1], dtype=np.int64)
+    heads = np.concatenate([heads, rng.integers(0, BH, size=fixed_rows.size)])
+    rows = np.concatenate([rows, fixed_rows])
+    return heads, rows
+
+
+def check_forward_sampled(out, lse, q, k, v, heads, rows, causal=True):
+    N = q.shape[2]
+    w_out, w_lse = oracle.attn_fwd_rows(q, k, v, heads, rows, causal=causal)
+    g_out = to_f64(out).reshape(-1, N, 64)[heads, rows]
+    g_lse = to_f64(lse).reshape(-1, N)[heads, rows]
+    check_bf16(g_out, w_out, "out (sampled rows)")
+    check_lse(g_lse, w_lse, "lse (sampled rows)")
+
+
+def check_forward_properties(out, lse, qb, kb, vb):
+    """Row 0 sees key 0 alone: out_0 = v_0 exactly; lse_i >= s_ii."""
+    o0 = out[:, :, 0].view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(o0, vb[:, :, 0])
+    q = torch.from_numpy(inputs.bf16_to_f32(qb)).cuda()
+    k = torch.from_numpy(inputs.bf16_to_f32(kb)).cuda()
+    sii = (q * k).sum(-1) / 8.0
+    assert bool((lse >= sii - 1e-3 * sii.abs().clamp(min=1)).all())
+
+
+def test_bf16_forward_b4_h16_n4096():
+    wl = inputs.WORKLOADS["attn_fwd_b4h16n4096"]
+    qb, kb, vb, _ = inputs.attn_bf16(**wl)
+    out, lse, _ = run_fwd_bwd(dev_bf16(qb), dev_bf16(kb), dev_bf16(vb), backward=False)
+    assert bool(torch.isfinite(out).all()) and bool(torch.isfinite(lse).all())
+    check_forward_properties(out, lse, qb, kb, vb)
+    q, k, v = (inputs.bf16_to_f64(b) for b in (qb, kb, vb))
+    heads, rows = sample_rows(np.random.default_rng(0), 64, wl["N"], 96)
+    check_forward_sampled(out, lse, q, k, v, heads, rows)
+
+
+def _backward_sampled(qb, kb, vb, out, lse, dq, dk, dv, n_q, n_k, tail, seed):
+    B, H, N, _ = qb.shape
+    q, k, v = (inputs.bf16_to_f64(b) for b in (qb, kb, vb))
+    o = to_f64(out)
+    rng = np.random.default_rng(seed)
+    qh, qr = sample_rows(rng, B * H, N, n_q)
+    kh = rng.integers(0, B * H, size=n_k)
+    kr = N - 1 - rng.integers(0, tail, size=n_k)
+    w_dq, w_dk, w_dv = oracle.attn_bwd_rows(q, k, v, o, qh, qr, kh, kr, out=o)
+    check_bf16(to_f64(dq).reshape(-1, N, 64)[qh, qr], w_dq, "dq (sampled rows)")
+    check_bf16(to_f64(dk).reshape(-1, N, 64)[kh, kr], w_dk, "dk (sampled rows)")
+    check_bf16(to_f64(dv).reshape(-1, N, 64)[kh, kr], w_dv, "dv (sampled rows)")
+
+
+def test_bf16_forward_backward_b2_h16_n16384():
+    wl = inputs.WORKLOADS["attn_fwdbwd_b2h16n16384"]
+    qb, kb, vb, _ = inputs.attn_bf16(**wl)
+    out, lse, (dq, dk, dv) = run_fwd_bwd(dev_bf16(qb), dev_bf16(kb), dev_bf16(vb))
+    for t in (out, lse, dq, dk, dv):
+        assert bool(torch.isfinite(t).all())
+    check_forward_properties(out, lse, qb, kb, vb)
+    q, k, v = (inputs.bf16_to_f64(b) for b in (qb, kb, vb))
+    heads, rows = sample_rows(np.random.default_rng(1), 32, wl["N"], 48)
+    check_forward_sampled(out, lse, q, k, v, heads, rows)
+    _backward_sampled(qb, kb, vb, out, lse, dq, dk, dv, n_q=24, n_k=6, tail=256, seed=2)
+
+
+@pytest.mark.parametrize("with_inf", [False, True])
+def test_bf16_long_context_b1_h8_n65536(with_inf):
+    wl = inputs.WORKLOADS["attn_fwdbwd_b1h8n65536"]
+    n_inf = inputs.LONG_CONTEXT_N_INF if with_inf else 0
+    qb, kb, vb, pos = inputs.attn_bf16(**wl, n_inf=n_inf)
+    assert pos.size == n_inf
+    out, lse, (dq, dk, dv) = run_fwd_bwd(dev_bf16(qb), dev_bf16(kb), dev_bf16(vb))
+    N = wl["N"]
+    # Full-size property: out[h, i, d] = +inf exactly when some V[h, j, d] = +inf
+    # with j <= i; every other entry (and lse) is finite.
+    o = to_f64(out)[0]
+    first = np.full((wl["H"], 64), N, dtype=np.int64)
+    if n_inf:
+        _, h_, j_, d_ = np.unravel_index(pos, (1, wl["H"], N, 64))
+        np.minimum.at(first, (h_, d_), j_)
+    want_inf = np.arange(N)[None, :, None] >= first[:, None, :]
+    assert np.array_equal(np.isposinf(o), want_inf)
+    assert np.isfinite(o[~want_inf]).all()
+    assert bool(torch.isfinite(lse).all())
+    q, k, v = (inputs.bf16_to_f64(b) for b in (qb, kb, vb))
+    heads, rows = sample_rows(np.random.default_rng(3), wl["H"], N, 24)
+    check_forward_sampled(out, lse, q, k, v, heads, rows)
+    _backward_sampled(qb, kb, vb, out, lse, dq, dk, dv, n_q=12, n_k=3, tail=64, seed=4)

@@ -1,0 +1,67 @@
+"""GPU parity of the Nadaraya-Watson regrid (through the C ABI) against the
+float64 oracle: the demo's own check_nadaraya_watson inputs ("Show HN:
+Automatic deduction of FlashAttention kernel from ~25 lines of SQL",
+64 targets x 256 sources in [0,1]^2), the 16384 x 16384 grid in [0,10]^2
+(every target), ragged sizes, and the degenerate cases (one source,
+constant values, all weights underflowing -> NaN).  Tolerance: float32
+path, max abs error <= 1e-5 (tests/_compare.py)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from causal_attention_swa_b200 import inputs, swa
+from _compare import check_f32
+
+pytestmark = pytest.mark.gpu
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+
+def run(t, s, v, h=0.5):
+    out = swa.nw_regrid(dev(t), dev(s), dev(v), h=h)
+    torch.cuda.synchronize()
+    return out
+
+
+def test_nw_demo_inputs():
+    t, s, y = inputs.pages_nw()
+    t32, s32, y32 = (a.astype(np.float32) for a in (t, s, y))
+    got = run(t32, s32, y32)
+    check_f32(got, oracle.nw_regrid(t32, s32, y32, h=0.5), "nw demo")
+
+
+def test_nw_grid_16384():
+    t, s, v = inputs.nw_grid()
+    got = run(t, s, v)
+    want = oracle.nw_regrid(t, s, v, h=0.5)
+    check_f32(got, want, "nw 16384x16384")
+
+
+@pytest.mark.parametrize("M,S", [(1, 1), (1, 5000), (1023, 17), (1025, 2049), (3000, 4097),
+                                 (70000, 300)])
+def test_nw_ragged_sizes(M, S):
+    rng = np.random.default_rng(M * 7 + S)
+    t = rng.uniform(0, 3, size=(M, 2)).astype(np.float32)
+    s = rng.uniform(0, 3, size=(S, 2)).astype(np.float32)
+    v = rng.normal(size=S).astype(np.float32)
+    check_f32(run(t, s, v), oracle.nw_regrid(t, s, v, h=0.5), f"nw {M}x{S}")
+
+
+def test_nw_degenerate_cases():
+    rng = np.random.default_rng(0)
+    t = rng.uniform(0, 2, size=(100, 2)).astype(np.float32)
+    one = np.array([[1.0, 1.0]], np.float32)
+    got = run(t, one, np.array([2.5], np.float32)).cpu().numpy()
+    assert np.abs(got - 2.5).max() <= 2.5 * 2.0 ** -22  # (w v) / w: two roundings
+    s = rng.uniform(0, 2, size=(300, 2)).astype(np.float32)
+    got = run(t, s, np.full(300, 0.7, np.float32)).cpu().numpy()
+    assert np.abs(got - 0.7).max() < 1e-6
+    far = run(np.array([[100.0, 100.0]], np.float32), one, np.array([1.0], np.float32))
+    assert bool(torch.isnan(far).all())
+    # another bandwidth: h = 0.25 -> divisor 0.0625
+    s2 = rng.uniform(0, 2, size=(500, 2)).astype(np.float32)
+    v2 = rng.normal(size=500).astype(np.float32)
+    check_f32(run(t, s2, v2, h=0.25), oracle.nw_regrid(t, s2, v2, h=0.25), "nw h=0.25")
