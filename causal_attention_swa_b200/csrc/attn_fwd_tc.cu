@@ -246,13 +246,15 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (!mbar_wait(&sm.s_full[t], j & 1, abort, err, kDevTimeoutMma)) { ok = false; break; }
       fence_after_sync();
       float x[BN];
+      {
+        uint32_t u[BN / 16][16];
 #pragma unroll
-      for (int i = 0; i < BN / 16; ++i) {
-        uint32_t u[16];
-        tmem_ld16(tS + i * 16, u);
+        for (int i = 0; i < BN / 16; ++i) tmem_ld16(tS + i * 16, u[i]);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) x[i * 16 + e] = __uint_as_float(u[e]) * scale_log2;
+        for (int i = 0; i < BN / 16; ++i)
+#pragma unroll
+          for (int e = 0; e < 16; ++e) x[i * 16 + e] = __uint_as_float(u[i][e]) * scale_log2;
       }
       const bool need_mask = (j * BN + BN > N) || (causal && j == g);
       if (need_mask) {
@@ -262,9 +264,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (key >= N || (causal && key > row)) x[e] = -INFINITY;
         }
       }
-      float mx = x[0];
+      float mxp[8];
 #pragma unroll
-      for (int e = 1; e < BN; ++e) mx = fmaxf(mx, x[e]);
+      for (int a = 0; a < 8; ++a) mxp[a] = x[a];
+#pragma unroll
+      for (int e = 8; e < BN; ++e) mxp[e & 7] = fmaxf(mxp[e & 7], x[e]);
+      const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                             fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
       const float m_new = fmaxf(m_used, mx);
       const bool need = (j == 0) || (m_new > m_used + kRescaleThreshold);
       if (j > 0 && __any_sync(0xffffffffu, need)) {
@@ -281,7 +287,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         l *= alpha;
       }
       if (need) m_used = m_new;
-      float rs = 0.f;
+      float rsp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < BN / 32; ++i) {
         uint32_t pk[16];
@@ -289,7 +295,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int e = 0; e < 16; ++e) {
           const float p0 = ex2(x[i * 32 + 2 * e] - m_used);
           const float p1 = ex2(x[i * 32 + 2 * e + 1] - m_used);
-          rs += p0 + p1;
+          rsp[e & 3] += p0 + p1;
           pk[e] = pack_bf16(p0, p1);
         }
         tmem_st16(tS + i * 16, pk);
@@ -297,7 +303,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       tmem_wait_st();
       fence_before_sync();
       mbar_arrive(&sm.p_full[t]);
-      l += rs;
+      l += (rsp[0] + rsp[1]) + (rsp[2] + rsp[3]);
     }
     if (ok && n_t[t] > 0 && mbar_wait(&sm.o_final[t], 0, abort, err, kDevTimeoutMma)) {
       fence_after_sync();

@@ -110,24 +110,27 @@ Plan plan(int64_t M, int64_t S) {
 
 }  // namespace
 
-size_t nw_partials_bytes(int64_t M, int64_t S, int /*sm_count*/) {
+size_t nw_partials_bytes(int64_t M, int64_t S) {
   const Plan pl = plan(M, S);
   return (size_t)(pl.nchunks * M) * sizeof(float2);
 }
 
-cudaError_t launch_nw_regrid(const float* targets, int64_t M, const float* sources,
-                             const float* vals, int64_t S, float h, float* out,
-                             float* partials, int /*sm_count*/, cudaStream_t s,
-                             int* launches) {
+cudaError_t launch_nw_partial(const float* targets, int64_t M, const float* sources,
+                              const float* vals, int64_t S, float h, float* partials,
+                              cudaStream_t s, int* launches) {
   const Plan pl = plan(M, S);
   const float c = sqrtf(kLog2e) / h;
   dim3 grid((unsigned)pl.mtiles, (unsigned)pl.nchunks);
   const size_t smem = (size_t)pl.chunk * sizeof(float4);
   nw_partial_kernel<<<grid, kThreads, smem, s>>>(targets, M, sources, vals, S, c, pl.chunk,
                                                  reinterpret_cast<float2*>(partials));
-  cudaError_t e = cudaGetLastError();
   *launches += 1;
-  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_nw_finalize(int64_t M, int64_t S, const float* partials, float* out,
+                               cudaStream_t s, int* launches) {
+  const Plan pl = plan(M, S);
   nw_finalize_kernel<<<(unsigned)((M + 255) / 256), 256, 0, s>>>(
       reinterpret_cast<const float2*>(partials), (int)pl.nchunks, M, out);
   *launches += 1;

@@ -20,6 +20,25 @@ namespace {
 thread_local char t_msg[512];
 thread_local int t_launches;
 
+struct Prof {
+  swa_kernel which = SWA_KERNEL_NONE;
+  cudaEvent_t start = nullptr, stop = nullptr;
+};
+thread_local Prof t_prof;
+
+// Records the hook's start/stop events around one launcher call when it
+// names this kernel.
+struct ProfScope {
+  bool on;
+  cudaStream_t s;
+  ProfScope(swa_kernel k, cudaStream_t stream) : on(t_prof.which == k), s(stream) {
+    if (on) cudaEventRecord(t_prof.start, s);
+  }
+  ~ProfScope() {
+    if (on) cudaEventRecord(t_prof.stop, s);
+  }
+};
+
 swa_status fail(swa_status st, const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);
@@ -133,8 +152,11 @@ swa_status swa_attn_fwd(const void* q, const void* k, const void* v, void* out, 
     if (e != cudaSuccess) return cuda_fail(e, "scan_nonfinite(v)");
     // Heads whose V is all finite: tensor-core kernel.  Heads holding a
     // non-finite value: the pair-by-pair kernel, so masked pairs stay absent.
-    e = swa::launch_attn_fwd_tc(q, k, v, out, lse, B, H, N, causal ? 1 : 0, scale, flags, err,
-                                s, &launches);
+    {
+      ProfScope ps(SWA_KERNEL_ATTN_FWD, s);
+      e = swa::launch_attn_fwd_tc(q, k, v, out, lse, B, H, N, causal ? 1 : 0, scale, flags, err,
+                                  s, &launches);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_tc");
     e = swa::launch_attn_fwd_simt(dt, q, k, v, out, lse, BH, N, causal ? 1 : 0, scale, flags,
                                   1, s, &launches);
@@ -189,8 +211,11 @@ swa_status swa_attn_bwd(const void* q, const void* k, const void* v, const void*
     if (e != cudaSuccess) return cuda_fail(e, "scan_nonfinite(v)");
     e = swa::launch_scan_nonfinite(dt, dout, BH, N * D, flags, s, &launches);
     if (e != cudaSuccess) return cuda_fail(e, "scan_nonfinite(dout)");
-    e = swa::launch_attn_bwd_tc(q, k, v, dout, lse, delta, dq, dk, dv, dqacc, B, H, N, c, scale,
-                                flags, err, s, &launches);
+    {
+      ProfScope ps(SWA_KERNEL_ATTN_BWD, s);
+      e = swa::launch_attn_bwd_tc(q, k, v, dout, lse, delta, dq, dk, dv, dqacc, B, H, N, c,
+                                  scale, flags, err, s, &launches);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_tc");
     e = swa::launch_attn_bwd_simt(dt, q, k, v, dout, lse, delta, dq, dk, dv, BH, N, c, scale,
                                   flags, 1, s, &launches);
@@ -202,7 +227,7 @@ swa_status swa_attn_bwd(const void* q, const void* k, const void* v, const void*
 
 size_t swa_nw_workspace_size(int64_t M, int64_t S) {
   if (M < 1 || S < 1) return 0;
-  return round_up(swa::nw_partials_bytes(M, S, 148), 256);
+  return round_up(swa::nw_partials_bytes(M, S), 256);
 }
 
 swa_status swa_nw_regrid(const float* targets, int64_t M, const float* sources,
@@ -225,10 +250,16 @@ swa_status swa_nw_regrid(const float* targets, int64_t M, const float* sources,
     return fail(SWA_ERR_INVALID_ARGUMENT, "workspace must be 16-byte aligned and >= %zu bytes",
                 need);
   int launches = 0;
-  cudaError_t e = swa::launch_nw_regrid(targets, M, sources, vals, S, h, out,
-                                        static_cast<float*>(workspace), 148,
-                                        static_cast<cudaStream_t>(stream), &launches);
-  if (e != cudaSuccess) return cuda_fail(e, "nw_regrid");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  {
+    ProfScope ps(SWA_KERNEL_NW, s);
+    e = swa::launch_nw_partial(targets, M, sources, vals, S, h, static_cast<float*>(workspace),
+                               s, &launches);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "nw_partial");
+  e = swa::launch_nw_finalize(M, S, static_cast<const float*>(workspace), out, s, &launches);
+  if (e != cudaSuccess) return cuda_fail(e, "nw_finalize");
   t_launches = launches;
   return SWA_OK;
 }
@@ -266,5 +297,15 @@ const char* swa_status_string(swa_status status) {
 const char* swa_last_error_message(void) { return t_msg; }
 
 int swa_last_launch_count(void) { return t_launches; }
+
+void swa_profile_kernel(swa_kernel which, void* start_event, void* stop_event) {
+  if (which == SWA_KERNEL_NONE || !start_event || !stop_event) {
+    t_prof = Prof{};
+    return;
+  }
+  t_prof.which = which;
+  t_prof.start = static_cast<cudaEvent_t>(start_event);
+  t_prof.stop = static_cast<cudaEvent_t>(stop_event);
+}
 
 }  // extern "C"

@@ -61,9 +61,11 @@ cudaError_t launch_attn_bwd_simt(swa_dtype dt, const void* q, const void* k, con
                                  int causal, float scale, const int* flags, int select,
                                  cudaStream_t s, int* launches);
 
-size_t nw_partials_bytes(int64_t M, int64_t S, int sm_count);
-cudaError_t launch_nw_regrid(const float* targets, int64_t M, const float* sources,
-                             const float* vals, int64_t S, float h, float* out,
-                             float* partials, int sm_count, cudaStream_t s, int* launches);
+size_t nw_partials_bytes(int64_t M, int64_t S);
+cudaError_t launch_nw_partial(const float* targets, int64_t M, const float* sources,
+                              const float* vals, int64_t S, float h, float* partials,
+                              cudaStream_t s, int* launches);
+cudaError_t launch_nw_finalize(int64_t M, int64_t S, const float* partials, float* out,
+                               cudaStream_t s, int* launches);
 
 }  // namespace swa

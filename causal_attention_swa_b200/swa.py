@@ -26,7 +26,9 @@ EXPORTS = (
     "swa_attn_fwd_workspace_size", "swa_attn_fwd", "swa_attn_bwd_workspace_size",
     "swa_attn_bwd", "swa_nw_workspace_size", "swa_nw_regrid", "swa_get_device_error",
     "swa_status_string", "swa_last_error_message", "swa_last_launch_count",
+    "swa_profile_kernel",
 )
+SWA_KERNEL_NONE, SWA_KERNEL_ATTN_FWD, SWA_KERNEL_ATTN_BWD, SWA_KERNEL_NW = range(4)
 
 
 class SwaError(RuntimeError):
@@ -75,6 +77,8 @@ def load_library():
     lib.swa_last_error_message.restype = ctypes.c_char_p
     lib.swa_last_launch_count.argtypes = []
     lib.swa_last_launch_count.restype = I
+    lib.swa_profile_kernel.argtypes = [I, P, P]
+    lib.swa_profile_kernel.restype = None
     _lib = lib
     return lib
 
@@ -110,6 +114,17 @@ def _require_cuda(*ts):
 def last_launch_count() -> int:
     """Kernels the last successful call on this thread enqueued."""
     return int(load_library().swa_last_launch_count())
+
+
+def profile_kernel(which: int, start=None, stop=None) -> None:
+    """swa_profile_kernel: later calls on this thread record the torch.cuda.Event
+    pair around kernel `which` (SWA_KERNEL_*); which = SWA_KERNEL_NONE stops."""
+    lib = load_library()
+    if which == SWA_KERNEL_NONE or start is None or stop is None:
+        lib.swa_profile_kernel(SWA_KERNEL_NONE, None, None)
+        return
+    lib.swa_profile_kernel(which, ctypes.c_void_p(start.cuda_event),
+                           ctypes.c_void_p(stop.cuda_event))
 
 
 def attn_fwd_workspace_size(B, H, N, D, dtype_code) -> int:

@@ -143,6 +143,22 @@ const char* swa_last_error_message(void);
 /* Kernel launches the last successful call on this host thread enqueued. */
 int swa_last_launch_count(void);
 
+/* Main kernels that swa_profile_kernel can bracket with events. */
+typedef enum {
+    SWA_KERNEL_NONE = 0,
+    SWA_KERNEL_ATTN_FWD = 1, /* swa_attn_fwd: the kernel of the heads with finite V */
+    SWA_KERNEL_ATTN_BWD = 2, /* swa_attn_bwd: the main kernel(s) of the finite heads */
+    SWA_KERNEL_NW = 3        /* swa_nw_regrid: the pair-grid kernel (not the final sum) */
+} swa_kernel;
+
+/*
+ * Timing hook for this host thread: every later call that launches kernel
+ * `which` records `start_event` on its stream just before that launch and
+ * `stop_event` just after it (both are cudaEvent_t created by the caller).
+ * SWA_KERNEL_NONE (or NULL events) turns the hook off.  Never fails.
+ */
+void swa_profile_kernel(swa_kernel which, void* start_event, void* stop_event);
+
 #ifdef __cplusplus
 }
 #endif
