@@ -112,6 +112,22 @@ BwdWs bwd_ws(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtype dt) {
 
 }  // namespace
 
+namespace swa {
+
+swa_status api_fail(swa_status st, const char* msg) { return fail(st, "%s", msg); }
+swa_status api_cuda_fail(cudaError_t e, const char* where) { return cuda_fail(e, where); }
+swa_status api_check_attn_shape(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtype dt) {
+  return check_attn_shape(B, H, N, D, dt);
+}
+unsigned* api_error_word(swa_status* st) { return device_error_word(st); }
+void api_begin_call() {
+  t_msg[0] = 0;
+  t_launches = 0;
+}
+void api_end_call(int launches) { t_launches = launches; }
+
+}  // namespace swa
+
 extern "C" {
 
 size_t swa_attn_fwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtype dt) {

@@ -39,6 +39,16 @@ __device__ __forceinline__ bool head_selected(const int* flags, int64_t head, in
   return flags == nullptr || ((flags[head] != 0) == (select != 0));
 }
 
+// ------------------------------------------------- shared C-ABI bookkeeping
+// (swa_api.cu): error message, argument checks, device error word and the
+// per-thread launch count, for entry points defined in other files.
+swa_status api_fail(swa_status st, const char* msg);
+swa_status api_cuda_fail(cudaError_t e, const char* where);
+swa_status api_check_attn_shape(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtype dt);
+unsigned* api_error_word(swa_status* st);
+void api_begin_call();
+void api_end_call(int launches);
+
 // ---------------------------------------------------------------- launchers
 // Each returns the launch's cudaError_t and adds the number of kernels it
 // enqueued to *launches.

@@ -26,7 +26,7 @@ EXPORTS = (
     "swa_attn_fwd_workspace_size", "swa_attn_fwd", "swa_attn_bwd_workspace_size",
     "swa_attn_bwd", "swa_nw_workspace_size", "swa_nw_regrid", "swa_get_device_error",
     "swa_status_string", "swa_last_error_message", "swa_last_launch_count",
-    "swa_profile_kernel",
+    "swa_profile_kernel", "swa_attn_fwd_noalloc",
 )
 SWA_KERNEL_NONE, SWA_KERNEL_ATTN_FWD, SWA_KERNEL_ATTN_BWD, SWA_KERNEL_NW = range(4)
 

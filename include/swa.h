@@ -112,6 +112,24 @@ swa_status swa_attn_bwd(const void* q, const void* k, const void* v, const void*
                         swa_dtype dtype, void* workspace, size_t workspace_bytes,
                         void* stream);
 
+/*
+ * swa_attn_fwd without a workspace, for callers that cannot allocate device
+ * memory (a plugin whose host application owns every device allocation and
+ * passes it only inputs and outputs; a latency-critical path that must not
+ * pay for cudaMalloc/cudaFree and their implicit synchronisation).  The
+ * pages have no counterpart: this is an interface convenience.
+ * Same arguments, results and errors as swa_attn_fwd minus the workspace.
+ * The forward's scratch (one int32 flag per head) lives in a static device
+ * array of 4096 entries (16 KB, held by every GPU that loads the library
+ * until exit); B*H > 4096 returns SWA_ERR_UNSUPPORTED.  The first call on
+ * each device looks up the array's device address (make it before any
+ * stream capture).  All calls share the array: calls that overlap on the
+ * GPU race.  Allocates nothing.
+ */
+swa_status swa_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
+                                float* lse, int64_t B, int64_t H, int64_t N, int64_t D,
+                                int causal, swa_dtype dtype, void* stream);
+
 /* Bytes of workspace swa_nw_regrid needs for M targets and S sources. */
 size_t swa_nw_workspace_size(int64_t M, int64_t S);
 
