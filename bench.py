@@ -45,7 +45,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # kernel id -> (name, source file whose hash keys the recorded ncu traffic)
 KERNELS = {
     1: ("attn_fwd", "causal_attention_swa_b200/csrc/attn_fwd_tc.cu"),
-    2: ("attn_bwd", "causal_attention_swa_b200/csrc/attn_tc.cu"),
+    2: ("attn_bwd", "causal_attention_swa_b200/csrc/attn_bwd_tc.cu"),
     3: ("nw_regrid", "causal_attention_swa_b200/csrc/nw_regrid.cu"),
 }
 

@@ -1,0 +1,470 @@
+// attn_bwd_tc.cu -- attention backward on the sm_100a tensor cores
+// (tcgen05.mma kind::f16: bf16 operands, f32 accumulators in TMEM).
+//
+// The method: the GRADIENT query of "Show HN: Automatic deduction of
+// FlashAttention kernel from ~25 lines of SQL" (page 2) -- one backward pass
+// for dq, dk and dv of a loss that reads the attention view -- in the
+// FlashAttention form that recomputes P from the saved row logsumexp:
+//   P_ij = exp(s_ij - lse_i)            dP_ij = dout_i . v_j
+//   dS_ij = P_ij (dP_ij - delta_i)      delta_i = dout_i . out_i (prep kernel)
+//   dv_j += P_ij dout_i   dk_j += scale dS_ij q_i   dq_i += scale dS_ij k_j
+// over the pairs that exist (j <= i when causal).
+//
+// Block = one 128-key block j of one head (K_j, V_j stay in shared memory)
+// and 384 threads; it walks the 128-query blocks i that see j:
+//   warps 0-3   "softmax-grad": thread t owns key j0+t (TMEM lane t); from
+//               S^T and dP^T it forms P^T (bf16, back into TMEM for dV) and
+//               dS (float32, split into bf16 hi + lo parts, written to
+//               shared memory); finally stores dv and dk of its key
+//   warp  4     TMA producer: K_j, V_j once; Q_i, dO_i into a 2-stage ring
+//   warp  5     MMA issuer (one thread), TMEM owner
+//   warps 6-7   idle
+//   warps 8-11  dQ drain: dQ_i (TMEM lane = query) -> a shared staging row
+//               per thread -> cp.reduce.async.bulk add.f32 into the float32
+//               dQ accumulator
+// Per query block, seven MMAs (M = 128, K = 64 or 128):
+//   S^T = K_j Q_i^T              (A = K smem K-major, B = Q smem K-major)
+//   dP^T = V_j dO_i^T            (A = V, B = dO, both K-major)
+//   dV += P^T dO_i               (A = P^T from TMEM, B = dO MN-major)
+//   dK += dS_hi^T Q_i + dS_lo^T Q_i   (A = dS tiles read K-major, B = Q MN-major)
+//   dQ_i = dS_hi K_j + dS_lo K_j      (A = the same tiles read MN-major, B = K)
+// dS is carried as hi + lo bf16 pairs (hi = bf16(dS), lo = bf16(dS - hi)),
+// so dk and dq see dS to ~16 bits: a single bf16 rounding of dS, amplified
+// by the cancellation in sum_j dS_ij k_j (sum_j dS_ij = 0), costs dq about
+// 2% of its row RMS at N = 2048.  One [128 keys][128 queries] tile layout
+// (rows = keys, 128-byte swizzle, two 64-query halves) is both the K-major
+// A operand of dK and the MN-major A operand of dQ.
+// TMEM (512 columns): S^T buffers [0,128) and [128,256) (P^T of the block in
+// their first 64 columns, its dQ in the last 64), dP^T [256,384),
+// dV [384,448), dK [448,512).  MMAs of one thread execute in issue order,
+// so a later MMA may overwrite TMEM an earlier one reads.
+// Issue order per block i: S^T_i+1 (other buffer); once the softmax-grad
+// warps are done with block i: dP^T_i+1, dV_i, dK_i, dQ_i -- while they work
+// on block i+1 the tensor core finishes block i.
+// Causal: only query blocks i >= j are visited; in the diagonal block (and
+// past N on a ragged tail) P and dS of a masked pair are set to 0 by select.
+// This kernel takes only heads whose V and dout are all finite, so 0 times
+// a finite value is the same as skipping the pair.
+// Every mbarrier wait is bounded (device error word on expiry).
+#include "attn_tc.cuh"
+#include "tc_ptx.cuh"
+
+namespace swa {
+namespace {
+
+using namespace tc;
+
+constexpr int BK = 128;                 // keys per block
+constexpr int BQ = 128;                 // queries per block
+constexpr int HD = 64;
+constexpr int kTileBytes = 128 * HD * 2;
+constexpr int kThreads = 384;
+constexpr int kTmaWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kDrainWarp0 = 8;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColDP = 256, kColDV = 384, kColDK = 448;
+constexpr int kStageRow = HD + 4;  // floats per staged dQ row: 272 B, so row starts rotate banks
+
+__device__ __forceinline__ uint32_t col_s(int b) { return b ? 128u : 0u; }
+__device__ __forceinline__ uint32_t col_dq(int b) { return b ? 192u : 64u; }
+
+struct __align__(1024) Smem {
+  uint8_t k[kTileBytes];
+  uint8_t v[kTileBytes];
+  uint8_t q[2][kTileBytes];
+  uint8_t dout[2][kTileBytes];
+  uint8_t ds_hi[2][kTileBytes];  // dS tiles [128 keys][queries 0-63 | 64-127]
+  uint8_t ds_lo[2][kTileBytes];
+  float dq[BQ * kStageRow];   // dQ staging, one padded row per drain thread
+  float lse[2][BQ];           // lse_i * log2(e) of the current query block
+  float delta[2][BQ];
+  uint64_t kv_full;
+  uint64_t qd_full[2];
+  uint64_t qd_empty[2];
+  uint64_t s_full[2];
+  uint64_t dp_full;
+  uint64_t sm_done;
+  uint64_t dq_full;
+  uint64_t dq_empty;
+  uint64_t acc_full;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+
+__device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitCycles) return false;
+  }
+  return true;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ lse,
+                   const float* __restrict__ delta, __nv_bfloat16* __restrict__ dk,
+                   __nv_bfloat16* __restrict__ dv, float* __restrict__ dqacc, int N, int BH,
+                   int causal, float scale, float scale_log2, const int* __restrict__ flags,
+                   unsigned* __restrict__ err) {
+  const int L = blockIdx.x;
+  const int head = L % BH;
+  const int jb = L / BH;  // key block; the first ones have the most query blocks
+  if (flags[head] != 0) return;
+
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                      ~static_cast<uintptr_t>(1023));
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int n_blocks = (N + BQ - 1) / BQ;
+  const int ib0 = causal ? jb : 0;
+  const int n_q = n_blocks - ib0;
+  const int j0 = jb * BK;
+
+  if (tid == 0) {
+    mbar_init(&sm.kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.qd_full[s], 1);
+      mbar_init(&sm.qd_empty[s], 1);
+      mbar_init(&sm.s_full[s], 1);
+    }
+    mbar_init(&sm.dp_full, 1);
+    mbar_init(&sm.sm_done, 128);
+    mbar_init(&sm.dq_full, 1);
+    mbar_init(&sm.dq_empty, 128);
+    mbar_init(&sm.acc_full, 1);
+    mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      prefetch_tmap(&tm_do);
+      mbar_arrive_expect_tx(&sm.kv_full, 2 * kTileBytes);
+      tma_load_3d(sm.k, &tm_k, &sm.kv_full, 0, j0, head);
+      tma_load_3d(sm.v, &tm_v, &sm.kv_full, 0, j0, head);
+      for (int it = 0; it < n_q; ++it) {
+        const int s = it & 1;
+        const int round = it >> 1;
+        if (round > 0 &&
+            !mbar_wait(&sm.qd_empty[s], (round - 1) & 1, abort, err, kDevTimeoutEmpty))
+          break;
+        const int i0 = (ib0 + it) * BQ;
+        mbar_arrive_expect_tx(&sm.qd_full[s], 2 * kTileBytes);
+        tma_load_3d(sm.q[s], &tm_q, &sm.qd_full[s], 0, i0, head);
+        tma_load_3d(sm.dout[s], &tm_do, &sm.qd_full[s], 0, i0, head);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // --------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T: both K-major
+      constexpr uint32_t id_mn = idesc_bf16_f32(128, 64, 0, 1);   // dV, dK: B MN-major
+      constexpr uint32_t id_dq = idesc_bf16_f32(128, 64, 1, 1);   // dQ: A and B MN-major
+      const uint32_t k_s = smem_u32(sm.k), v_s = smem_u32(sm.v);
+      auto issue_kk = [&](uint32_t d_col, uint32_t a0, uint32_t b0) {
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk)
+          mma_ss(tmem + d_col, desc_sw128(a0 + kk * 32, 16, 1024),
+                 desc_sw128(b0 + kk * 32, 16, 1024), id_kk, kk > 0 ? 1u : 0u);
+      };
+      // dK += dS^T Q_i from one dS tile: A rows = keys, K = queries (K-major;
+      // queries 64-127 in the second half tile)
+      auto issue_dk = [&](const uint8_t (*ds)[kTileBytes], uint32_t q0, bool first) {
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; ++kk)
+          mma_ss(tmem + kColDK, desc_sw128(smem_u32(ds[kk >> 2]) + (kk & 3) * 32, 16, 1024),
+                 desc_sw128(q0 + kk * 2048, 8192, 1024), id_mn, (!first || kk > 0) ? 1u : 0u);
+      };
+      // dQ_i (+)= dS K_j from one dS tile: A M = queries (MN-major, the two
+      // 64-query halves 16 KB apart), K = keys
+      auto issue_dq = [&](const uint8_t (*ds)[kTileBytes], uint32_t col, bool first) {
+        const uint32_t a0 = smem_u32(ds[0]);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          mma_ss(tmem + col, desc_sw128(a0 + kk * 2048, kTileBytes, 1024),
+                 desc_sw128(k_s + kk * 2048, 8192, 1024), id_dq, (!first || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(&sm.kv_full, 0, abort, err, kDevTimeoutFull) &&
+                mbar_wait(&sm.qd_full[0], 0, abort, err, kDevTimeoutFull);
+      if (ok) {
+        issue_kk(col_s(0), k_s, smem_u32(sm.q[0]));
+        mma_commit(&sm.s_full[0]);
+        issue_kk(kColDP, v_s, smem_u32(sm.dout[0]));
+        mma_commit(&sm.dp_full);
+      }
+      for (int it = 0; ok && it < n_q; ++it) {
+        const int b = it & 1;
+        if (it >= 1 && !mbar_wait(&sm.dq_empty, (it - 1) & 1, abort, err, kDevTimeoutOther)) break;
+        const bool next = it + 1 < n_q;
+        if (next) {
+          if (!mbar_wait(&sm.qd_full[b ^ 1], ((it + 1) >> 1) & 1, abort, err, kDevTimeoutFull))
+            break;
+          issue_kk(col_s(b ^ 1), k_s, smem_u32(sm.q[b ^ 1]));
+          mma_commit(&sm.s_full[b ^ 1]);
+        }
+        if (!mbar_wait(&sm.sm_done, it & 1, abort, err, kDevTimeoutOther)) break;
+        fence_after_sync();
+        if (next) {  // first, so the softmax-grad warps can start block it+1
+          issue_kk(kColDP, v_s, smem_u32(sm.dout[b ^ 1]));
+          mma_commit(&sm.dp_full);
+        }
+        const uint32_t q0 = smem_u32(sm.q[b]);
+        issue_dk(sm.ds_hi, q0, it == 0);
+        issue_dk(sm.ds_lo, q0, false);
+        issue_dq(sm.ds_hi, col_dq(b), true);
+        issue_dq(sm.ds_lo, col_dq(b), false);
+        mma_commit(&sm.dq_full);
+        {  // dV += P^T dO_i
+          const uint32_t b0 = smem_u32(sm.dout[b]);
+#pragma unroll
+          for (int kk = 0; kk < BQ / 16; ++kk)
+            mma_ts(tmem + kColDV, tmem + col_s(b) + kk * 8, desc_sw128(b0 + kk * 2048, 8192, 1024),
+                   id_mn, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&sm.qd_empty[b]);
+      }
+      mma_commit(&sm.acc_full);
+      mma_commit(&sm.drain);
+      wait_drain(&sm.drain, 0);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // -------------------------------------------------------- softmax-grad
+    const int jl = tid;  // key row within the block = TMEM lane
+    const int jg = j0 + jl;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t hi_row[2] = {smem_u32(sm.ds_hi[0]) + jl * 128, smem_u32(sm.ds_hi[1]) + jl * 128};
+    const uint32_t lo_row[2] = {smem_u32(sm.ds_lo[0]) + jl * 128, smem_u32(sm.ds_lo[1]) + jl * 128};
+    bool ok = true;
+    for (int it = 0; it < n_q; ++it) {
+      const int b = it & 1;
+      const int ib = ib0 + it;
+      const int i0 = ib * BQ;
+      {
+        const int r = i0 + tid;
+        sm.lse[b][tid] = r < N ? lse[(size_t)head * N + r] * kLog2e : INFINITY;
+        sm.delta[b][tid] = r < N ? delta[(size_t)head * N + r] : 0.f;
+      }
+      named_bar_sync(1, 128);
+      const bool need_mask = (causal && ib == jb) || (i0 + BQ > N) || (j0 + BK > N);
+      if (!mbar_wait(&sm.s_full[b], (it >> 1) & 1, abort, err, kDevTimeoutMma) ||
+          !mbar_wait(&sm.dp_full, it & 1, abort, err, kDevTimeoutMma)) {
+        ok = false;
+        break;
+      }
+      fence_after_sync();
+      // this key's dS over the 128 queries, as bf16 hi and lo pairs
+      uint32_t wh[BQ / 2], wl[BQ / 2];
+#pragma unroll
+      for (int c = 0; c < BQ / 16; ++c) {
+        uint32_t sv[16], dv16[16];
+        tmem_ld16(tmem + lane_off + col_s(b) + c * 16, sv);
+        tmem_ld16(tmem + lane_off + kColDP + c * 16, dv16);
+        tmem_wait_ld();
+        uint32_t wp[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float p2[2], ds2[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int q = c * 16 + 2 * e + h;  // query within the block
+            float p = ex2(fmaf(__uint_as_float(sv[2 * e + h]), scale_log2, -sm.lse[b][q]));
+            float ds = p * (__uint_as_float(dv16[2 * e + h]) - sm.delta[b][q]);
+            if (need_mask) {
+              const int ig = i0 + q;
+              if (ig >= N || jg >= N || (causal && ig < jg)) {
+                p = 0.f;
+                ds = 0.f;
+              }
+            }
+            p2[h] = p;
+            ds2[h] = ds;
+          }
+          wp[e] = pack_bf16(p2[0], p2[1]);
+          const uint32_t hi = pack_bf16(ds2[0], ds2[1]);
+          wh[c * 8 + e] = hi;
+          wl[c * 8 + e] = pack_bf16(ds2[0] - bf16lo(hi), ds2[1] - bf16hi(hi));
+        }
+        // P^T into columns 8c..8c+7 of this S^T buffer (already read)
+        tmem_st8(tmem + lane_off + col_s(b) + c * 8, wp);
+      }
+      // the dS tiles are free once the previous block's dK and dQ MMAs are done
+      if (it >= 1 && !mbar_wait(&sm.dq_full, (it - 1) & 1, abort, err, kDevTimeoutMma)) {
+        ok = false;
+        break;
+      }
+      // dS row of this key: query q is element q%64 of half q/64; 16-byte
+      // chunk k (8 queries) of a half sits at chunk k ^ (key & 7) (128-byte swizzle)
+#pragma unroll
+      for (int k16 = 0; k16 < BQ / 8; ++k16) {
+        const uint32_t off = ((uint32_t)(k16 & 7) ^ (uint32_t)(jl & 7)) << 4;
+        st_shared_v4(hi_row[k16 >> 3] + off, wh[4 * k16], wh[4 * k16 + 1], wh[4 * k16 + 2],
+                     wh[4 * k16 + 3]);
+        st_shared_v4(lo_row[k16 >> 3] + off, wl[4 * k16], wl[4 * k16 + 1], wl[4 * k16 + 2],
+                     wl[4 * k16 + 3]);
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      fence_before_sync();
+      mbar_arrive(&sm.sm_done);
+    }
+    // ---- dv, dk of this key
+    if (ok && mbar_wait(&sm.acc_full, 0, abort, err, kDevTimeoutMma)) {
+      fence_after_sync();
+      uint32_t a[4][16];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld16(tmem + lane_off + kColDV + c * 16, a[c]);
+      tmem_wait_ld();
+      if (jg < N) {
+        uint4* dst = reinterpret_cast<uint4*>(dv + ((size_t)head * N + jg) * HD);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            dst[2 * c + h] = make_uint4(
+                pack_bf16(__uint_as_float(a[c][8 * h + 0]), __uint_as_float(a[c][8 * h + 1])),
+                pack_bf16(__uint_as_float(a[c][8 * h + 2]), __uint_as_float(a[c][8 * h + 3])),
+                pack_bf16(__uint_as_float(a[c][8 * h + 4]), __uint_as_float(a[c][8 * h + 5])),
+                pack_bf16(__uint_as_float(a[c][8 * h + 6]), __uint_as_float(a[c][8 * h + 7])));
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld16(tmem + lane_off + kColDK + c * 16, a[c]);
+      tmem_wait_ld();
+      if (jg < N) {
+        uint4* dst = reinterpret_cast<uint4*>(dk + ((size_t)head * N + jg) * HD);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            dst[2 * c + h] = make_uint4(
+                pack_bf16(__uint_as_float(a[c][8 * h + 0]) * scale,
+                          __uint_as_float(a[c][8 * h + 1]) * scale),
+                pack_bf16(__uint_as_float(a[c][8 * h + 2]) * scale,
+                          __uint_as_float(a[c][8 * h + 3]) * scale),
+                pack_bf16(__uint_as_float(a[c][8 * h + 4]) * scale,
+                          __uint_as_float(a[c][8 * h + 5]) * scale),
+                pack_bf16(__uint_as_float(a[c][8 * h + 6]) * scale,
+                          __uint_as_float(a[c][8 * h + 7]) * scale));
+      }
+    }
+  } else if (warp >= kDrainWarp0) {
+    // ------------------------------------------------------------ dQ drain
+    // Thread te owns query row i0+te: it copies its dQ row from TMEM into its
+    // own padded staging row and adds that row (256 B) into the float32
+    // accumulator with one bulk reduce; before rewriting the row it waits for
+    // its previous bulk read to finish.
+    const int te = tid - kDrainWarp0 * 32;  // query row within the block = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    float* stage = sm.dq + te * kStageRow;
+    const uint32_t stage_s = smem_u32(stage);
+    for (int it = 0; it < n_q; ++it) {
+      const int b = it & 1;
+      if (!mbar_wait(&sm.dq_full, it & 1, abort, err, kDevTimeoutMma)) break;
+      fence_after_sync();
+      uint32_t a[4][16];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld16(tmem + lane_off + col_dq(b) + c * 16, a[c]);
+      tmem_wait_ld();
+      fence_before_sync();
+      mbar_arrive(&sm.dq_empty);
+      const int row = (ib0 + it) * BQ + te;
+      if (row < N) {
+        bulk_wait_group_read0();
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            st_shared_v4(stage_s + (c * 4 + g) * 16, a[c][4 * g], a[c][4 * g + 1],
+                         a[c][4 * g + 2], a[c][4 * g + 3]);
+        fence_proxy_async_smem();
+        bulk_reduce_add_f32(dqacc + ((size_t)head * N + row) * HD, stage, HD * 4);
+        bulk_commit_group();
+      }
+    }
+    bulk_wait_group0();
+  }
+
+  fence_before_sync();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    fence_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// dq = bf16(scale * dq accumulator) for the heads the tensor-core kernel took.
+__global__ void __launch_bounds__(256)
+attn_dq_convert_kernel(const float4* __restrict__ acc, uint4* __restrict__ dq, int64_t rows_per_head,
+                       int64_t total8, float scale, const int* __restrict__ flags) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t per_head8 = rows_per_head * (HD / 8);
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total8; idx += stride) {
+    if (flags[idx / per_head8] != 0) continue;
+    const float4 a = acc[2 * idx], c = acc[2 * idx + 1];
+    dq[idx] = make_uint4(pack_bf16(a.x * scale, a.y * scale), pack_bf16(a.z * scale, a.w * scale),
+                         pack_bf16(c.x * scale, c.y * scale), pack_bf16(c.z * scale, c.w * scale));
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* dout,
+                               const float* lse, const float* delta, void* dk, void* dv,
+                               float* dqacc, int64_t B, int64_t H, int64_t N, int causal,
+                               float scale, const int* flags, unsigned* err, cudaStream_t s,
+                               int* launches) {
+  const int64_t BH = B * H;
+  CUtensorMap tq, tk, tv, tdo;
+  cudaError_t e;
+  if ((e = make_tmap_bf16_rows(&tq, q, BH, N, BQ)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_rows(&tk, k, BH, N, BK)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_rows(&tv, v, BH, N, BK)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_rows(&tdo, dout, BH, N, BQ)) != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int64_t n_blocks = (N + BK - 1) / BK;
+  attn_bwd_tc_kernel<<<(unsigned)(n_blocks * BH), kThreads, kSmemBytes, s>>>(
+      tq, tk, tv, tdo, lse, delta, static_cast<__nv_bfloat16*>(dk),
+      static_cast<__nv_bfloat16*>(dv), dqacc, (int)N, (int)BH, causal, scale, scale * kLog2e,
+      flags, err);
+  *launches += 1;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_dq_convert(const float* dqacc, void* dq, int64_t BH, int64_t N,
+                                   float scale, const int* flags, cudaStream_t s,
+                                   int* launches) {
+  const int64_t total8 = BH * N * HD / 8;
+  int64_t blocks = (total8 + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  attn_dq_convert_kernel<<<(unsigned)blocks, 256, 0, s>>>(
+      reinterpret_cast<const float4*>(dqacc), static_cast<uint4*>(dq), N, total8, scale, flags);
+  *launches += 1;
+  return cudaGetLastError();
+}
+
+}  // namespace swa

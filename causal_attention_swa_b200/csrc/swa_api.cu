@@ -227,12 +227,18 @@ swa_status swa_attn_bwd(const void* q, const void* k, const void* v, const void*
     if (e != cudaSuccess) return cuda_fail(e, "scan_nonfinite(v)");
     e = swa::launch_scan_nonfinite(dt, dout, BH, N * D, flags, s, &launches);
     if (e != cudaSuccess) return cuda_fail(e, "scan_nonfinite(dout)");
+    // Heads with all-finite V and dout: tensor-core kernel (dk, dv directly,
+    // dq through the float32 accumulator); the others: pair-by-pair kernels.
+    e = cudaMemsetAsync(dqacc, 0, (size_t)BH * N * D * sizeof(float), s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dq accumulator)");
     {
       ProfScope ps(SWA_KERNEL_ATTN_BWD, s);
-      e = swa::launch_attn_bwd_tc(q, k, v, dout, lse, delta, dq, dk, dv, dqacc, B, H, N, c,
-                                  scale, flags, err, s, &launches);
+      e = swa::launch_attn_bwd_tc(q, k, v, dout, lse, delta, dk, dv, dqacc, B, H, N, c, scale,
+                                  flags, err, s, &launches);
     }
     if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_tc");
+    e = swa::launch_attn_dq_convert(dqacc, dq, BH, N, scale, flags, s, &launches);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_dq_convert");
     e = swa::launch_attn_bwd_simt(dt, q, k, v, dout, lse, delta, dq, dk, dv, BH, N, c, scale,
                                   flags, 1, s, &launches);
     if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_simt(non-finite heads)");
