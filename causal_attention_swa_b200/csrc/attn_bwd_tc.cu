@@ -11,17 +11,20 @@
 // over the pairs that exist (j <= i when causal).
 //
 // Block = one 128-key block j of one head (K_j, V_j stay in shared memory)
-// and 384 threads; it walks the 128-query blocks i that see j:
-//   warps 0-3   "softmax-grad": thread t owns key j0+t (TMEM lane t); from
-//               S^T and dP^T it forms P^T (bf16, back into TMEM for dV) and
-//               dS (float32, split into bf16 hi + lo parts, written to
-//               shared memory); finally stores dv and dk of its key
-//   warp  4     TMA producer: K_j, V_j once; Q_i, dO_i into a 2-stage ring
-//   warp  5     MMA issuer (one thread), TMEM owner
-//   warps 6-7   idle
+// and 512 threads; it walks the 128-query blocks i that see j:
+//   warps 0-7   "softmax-grad", two warpgroups: thread t of warpgroup g owns
+//               key j0 + t (TMEM lane t) and queries 64g..64g+63 of the
+//               block; from S^T and dP^T it forms P^T (bf16, back into TMEM
+//               for dV) and dS (float32, split into bf16 hi + lo parts,
+//               written to shared memory); warpgroup 0 finally stores dv and
+//               dk of its key
 //   warps 8-11  dQ drain: dQ_i (TMEM lane = query) -> a shared staging row
 //               per thread -> cp.reduce.async.bulk add.f32 into the float32
 //               dQ accumulator
+//   warp  12    TMA producer: K_j, V_j once; Q_i, dO_i, lse_i, delta_i into a
+//               2-stage ring
+//   warp  13    MMA issuer (one thread), TMEM owner
+//   warps 14-15 idle
 // Per query block, seven MMAs (M = 128, K = 64 or 128):
 //   S^T = K_j Q_i^T              (A = K smem K-major, B = Q smem K-major)
 //   dP^T = V_j dO_i^T            (A = V, B = dO, both K-major)
@@ -34,13 +37,19 @@
 // 2% of its row RMS at N = 2048.  One [128 keys][128 queries] tile layout
 // (rows = keys, 128-byte swizzle, two 64-query halves) is both the K-major
 // A operand of dK and the MN-major A operand of dQ.
-// TMEM (512 columns): S^T buffers [0,128) and [128,256) (P^T of the block in
-// their first 64 columns, its dQ in the last 64), dP^T [256,384),
-// dV [384,448), dK [448,512).  MMAs of one thread execute in issue order,
-// so a later MMA may overwrite TMEM an earlier one reads.
-// Issue order per block i: S^T_i+1 (other buffer); once the softmax-grad
-// warps are done with block i: dP^T_i+1, dV_i, dK_i, dQ_i -- while they work
-// on block i+1 the tensor core finishes block i.
+// TMEM (512 columns): S^T buffers [0,128) and [128,256) (the block's dQ in
+// the first 64 columns once S^T is consumed), dP^T [256,384) with P^T
+// (bf16, two per column) in its columns [32,96), dV [384,448), dK
+// [448,512).  P^T columns 32..63 are dP^T columns of queries 32..63 and
+// P^T columns 64..95 those of queries 64..95: each warpgroup overwrites
+// only columns it has itself read (warpgroup 0 walks its queries
+// downwards, warpgroup 1 upwards), so the two never race.  MMAs of one
+// thread execute in issue order, so a later MMA may overwrite TMEM an
+// earlier one reads.
+// Issue order: S^T_i+1 (other buffer) as soon as its buffer is free; once
+// the softmax-grad warps are done with block i: dV_i, dP^T_i+1, dK_i, dQ_i.
+// The softmax-grad warps hold the first half of a block's dS in registers
+// until block i-1's dK and dQ MMAs have released the dS tiles.
 // Causal: only query blocks i >= j are visited; in the diagonal block (and
 // past N on a ragged tail) P and dS of a masked pair are set to 0 by select.
 // This kernel takes only heads whose V and dout are all finite, so 0 times
@@ -58,16 +67,17 @@ constexpr int BK = 128;                 // keys per block
 constexpr int BQ = 128;                 // queries per block
 constexpr int HD = 64;
 constexpr int kTileBytes = 128 * HD * 2;
-constexpr int kThreads = 384;
-constexpr int kTmaWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kThreads = 512;
+constexpr int kGradThreads = 256;       // two softmax-grad warpgroups
 constexpr int kDrainWarp0 = 8;
+constexpr int kTmaWarp = 12;
+constexpr int kMmaWarp = 13;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColDP = 256, kColDV = 384, kColDK = 448;
+constexpr uint32_t kColDP = 256, kColPT = kColDP + 32, kColDV = 384, kColDK = 448;
 constexpr int kStageRow = HD + 4;  // floats per staged dQ row: 272 B, so row starts rotate banks
+constexpr int kHeadGroup = 4;      // heads scheduled together (their dQ, Q, dO share L2)
 
 __device__ __forceinline__ uint32_t col_s(int b) { return b ? 128u : 0u; }
-__device__ __forceinline__ uint32_t col_dq(int b) { return b ? 192u : 64u; }
 
 struct __align__(1024) Smem {
   uint8_t k[kTileBytes];
@@ -76,9 +86,9 @@ struct __align__(1024) Smem {
   uint8_t dout[2][kTileBytes];
   uint8_t ds_hi[2][kTileBytes];  // dS tiles [128 keys][queries 0-63 | 64-127]
   uint8_t ds_lo[2][kTileBytes];
-  float dq[BQ * kStageRow];   // dQ staging, one padded row per drain thread
-  float lse[2][BQ];           // lse_i * log2(e) of the current query block
-  float delta[2][BQ];
+  float dq[BQ * kStageRow];      // dQ staging, one padded row per drain thread
+  float lse[2][BQ];              // lse_i * log2(e) of each staged query block (+inf past N)
+  float delta[2][BQ];            // delta_i of each staged query block (0 past N)
   uint64_t kv_full;
   uint64_t qd_full[2];
   uint64_t qd_empty[2];
@@ -107,14 +117,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v,
-                   const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ lse,
+                   const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ lse2,
                    const float* __restrict__ delta, __nv_bfloat16* __restrict__ dk,
                    __nv_bfloat16* __restrict__ dv, float* __restrict__ dqacc, int N, int BH,
                    int causal, float scale, float scale_log2, const int* __restrict__ flags,
                    unsigned* __restrict__ err) {
-  const int L = blockIdx.x;
-  const int head = L % BH;
-  const int jb = L / BH;  // key block; the first ones have the most query blocks
+  // Block order: groups of kHeadGroup heads; inside a group the longest key
+  // blocks (j = 0 sees every query block) first, heads interleaved.
+  const int n_blocks = (N + BQ - 1) / BQ;
+  const int Npad = n_blocks * BQ;
+  const int group = blockIdx.x / (kHeadGroup * n_blocks);
+  const int g_heads = min(kHeadGroup, BH - group * kHeadGroup);
+  const int r = blockIdx.x - group * kHeadGroup * n_blocks;
+  const int jb = r / g_heads;
+  const int head = group * kHeadGroup + r % g_heads;
   if (flags[head] != 0) return;
 
   extern __shared__ uint8_t smem_raw[];
@@ -123,7 +139,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int n_blocks = (N + BQ - 1) / BQ;
   const int ib0 = causal ? jb : 0;
   const int n_q = n_blocks - ib0;
   const int j0 = jb * BK;
@@ -136,7 +151,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(&sm.s_full[s], 1);
     }
     mbar_init(&sm.dp_full, 1);
-    mbar_init(&sm.sm_done, 128);
+    mbar_init(&sm.sm_done, kGradThreads);
     mbar_init(&sm.dq_full, 1);
     mbar_init(&sm.dq_empty, 128);
     mbar_init(&sm.acc_full, 1);
@@ -171,9 +186,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             !mbar_wait(&sm.qd_empty[s], (round - 1) & 1, abort, err, kDevTimeoutEmpty))
           break;
         const int i0 = (ib0 + it) * BQ;
-        mbar_arrive_expect_tx(&sm.qd_full[s], 2 * kTileBytes);
+        mbar_arrive_expect_tx(&sm.qd_full[s], 2 * kTileBytes + 2 * BQ * 4);
         tma_load_3d(sm.q[s], &tm_q, &sm.qd_full[s], 0, i0, head);
         tma_load_3d(sm.dout[s], &tm_do, &sm.qd_full[s], 0, i0, head);
+        bulk_load(sm.lse[s], lse2 + (size_t)head * Npad + i0, BQ * 4, &sm.qd_full[s]);
+        bulk_load(sm.delta[s], delta + (size_t)head * Npad + i0, BQ * 4, &sm.qd_full[s]);
       }
     }
     __syncwarp();
@@ -217,8 +234,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       for (int it = 0; ok && it < n_q; ++it) {
         const int b = it & 1;
-        if (it >= 1 && !mbar_wait(&sm.dq_empty, (it - 1) & 1, abort, err, kDevTimeoutOther)) break;
         const bool next = it + 1 < n_q;
+        // the other S^T buffer holds dQ_it-1 until the drain has read it
+        if (it >= 1 && !mbar_wait(&sm.dq_empty, (it - 1) & 1, abort, err, kDevTimeoutOther)) break;
         if (next) {
           if (!mbar_wait(&sm.qd_full[b ^ 1], ((it + 1) >> 1) & 1, abort, err, kDevTimeoutFull))
             break;
@@ -227,23 +245,23 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         if (!mbar_wait(&sm.sm_done, it & 1, abort, err, kDevTimeoutOther)) break;
         fence_after_sync();
-        if (next) {  // first, so the softmax-grad warps can start block it+1
+        {  // dV += P^T dO_i  (P^T in the dP^T region, read before dP^T_it+1 lands)
+          const uint32_t b0 = smem_u32(sm.dout[b]);
+#pragma unroll
+          for (int kk = 0; kk < BQ / 16; ++kk)
+            mma_ts(tmem + kColDV, tmem + kColPT + kk * 8, desc_sw128(b0 + kk * 2048, 8192, 1024),
+                   id_mn, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        if (next) {
           issue_kk(kColDP, v_s, smem_u32(sm.dout[b ^ 1]));
           mma_commit(&sm.dp_full);
         }
         const uint32_t q0 = smem_u32(sm.q[b]);
         issue_dk(sm.ds_hi, q0, it == 0);
         issue_dk(sm.ds_lo, q0, false);
-        issue_dq(sm.ds_hi, col_dq(b), true);
-        issue_dq(sm.ds_lo, col_dq(b), false);
+        issue_dq(sm.ds_hi, col_s(b), true);
+        issue_dq(sm.ds_lo, col_s(b), false);
         mma_commit(&sm.dq_full);
-        {  // dV += P^T dO_i
-          const uint32_t b0 = smem_u32(sm.dout[b]);
-#pragma unroll
-          for (int kk = 0; kk < BQ / 16; ++kk)
-            mma_ts(tmem + kColDV, tmem + col_s(b) + kk * 8, desc_sw128(b0 + kk * 2048, 8192, 1024),
-                   id_mn, (it > 0 || kk > 0) ? 1u : 0u);
-        }
         mma_commit(&sm.qd_empty[b]);
       }
       mma_commit(&sm.acc_full);
@@ -251,46 +269,54 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       wait_drain(&sm.drain, 0);
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // -------------------------------------------------------- softmax-grad
-    const int jl = tid;  // key row within the block = TMEM lane
+    const int g = warp >> 2;          // query half of this warpgroup
+    const int jl = tid & 127;         // key row within the block = TMEM lane
     const int jg = j0 + jl;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t hi_row[2] = {smem_u32(sm.ds_hi[0]) + jl * 128, smem_u32(sm.ds_hi[1]) + jl * 128};
-    const uint32_t lo_row[2] = {smem_u32(sm.ds_lo[0]) + jl * 128, smem_u32(sm.ds_lo[1]) + jl * 128};
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t hi_row = smem_u32(sm.ds_hi[g]) + jl * 128;
+    const uint32_t lo_row = smem_u32(sm.ds_lo[g]) + jl * 128;
     bool ok = true;
     for (int it = 0; it < n_q; ++it) {
       const int b = it & 1;
       const int ib = ib0 + it;
       const int i0 = ib * BQ;
-      {
-        const int r = i0 + tid;
-        sm.lse[b][tid] = r < N ? lse[(size_t)head * N + r] * kLog2e : INFINITY;
-        sm.delta[b][tid] = r < N ? delta[(size_t)head * N + r] : 0.f;
-      }
-      named_bar_sync(1, 128);
       const bool need_mask = (causal && ib == jb) || (i0 + BQ > N) || (j0 + BK > N);
+      // S^T_i done implies Q_i's stage (with lse and delta) has landed
       if (!mbar_wait(&sm.s_full[b], (it >> 1) & 1, abort, err, kDevTimeoutMma) ||
           !mbar_wait(&sm.dp_full, it & 1, abort, err, kDevTimeoutMma)) {
         ok = false;
         break;
       }
       fence_after_sync();
-      // this key's dS over the 128 queries, as bf16 hi and lo pairs
-      uint32_t wh[BQ / 2], wl[BQ / 2];
+      // Four 16-query chunks of this half: warpgroup 0 walks them downwards,
+      // warpgroup 1 upwards, so P^T lands only on dP^T columns already read.
+      // The first two chunks' dS are held in registers until block i-1's dK
+      // and dQ MMAs release the dS tiles.  Query qh of a half is element qh
+      // of that half's tile row; 16-byte chunk k (8 queries) sits at chunk
+      // k ^ (key & 7) (128-byte swizzle).
+      uint32_t wh[16], wl[16];
+      auto store8 = [&](int k8, const uint32_t* h4, const uint32_t* l4) {
+        const uint32_t off = ((uint32_t)k8 ^ (uint32_t)(jl & 7)) << 4;
+        st_shared_v4(hi_row + off, h4[0], h4[1], h4[2], h4[3]);
+        st_shared_v4(lo_row + off, l4[0], l4[1], l4[2], l4[3]);
+      };
 #pragma unroll
-      for (int c = 0; c < BQ / 16; ++c) {
+      for (int step = 0; step < 4; ++step) {
+        const int c = g ? step : 3 - step;  // chunk within the half
+        const int qb0 = g * 64 + c * 16;     // first query of the chunk within the block
         uint32_t sv[16], dv16[16];
-        tmem_ld16(tmem + lane_off + col_s(b) + c * 16, sv);
-        tmem_ld16(tmem + lane_off + kColDP + c * 16, dv16);
+        tmem_ld16(tmem + lane_off + col_s(b) + qb0, sv);
+        tmem_ld16(tmem + lane_off + kColDP + qb0, dv16);
         tmem_wait_ld();
-        uint32_t wp[8];
+        uint32_t wp[8], h8[8], l8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           float p2[2], ds2[2];
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int q = c * 16 + 2 * e + h;  // query within the block
+            const int q = qb0 + 2 * e + h;  // query within the block
             float p = ex2(fmaf(__uint_as_float(sv[2 * e + h]), scale_log2, -sm.lse[b][q]));
             float ds = p * (__uint_as_float(dv16[2 * e + h]) - sm.delta[b][q]);
             if (need_mask) {
@@ -304,35 +330,42 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             ds2[h] = ds;
           }
           wp[e] = pack_bf16(p2[0], p2[1]);
-          const uint32_t hi = pack_bf16(ds2[0], ds2[1]);
-          wh[c * 8 + e] = hi;
-          wl[c * 8 + e] = pack_bf16(ds2[0] - bf16lo(hi), ds2[1] - bf16hi(hi));
+          h8[e] = pack_bf16(ds2[0], ds2[1]);
+          l8[e] = pack_bf16(ds2[0] - bf16lo(h8[e]), ds2[1] - bf16hi(h8[e]));
         }
-        // P^T into columns 8c..8c+7 of this S^T buffer (already read)
-        tmem_st8(tmem + lane_off + col_s(b) + c * 8, wp);
-      }
-      // the dS tiles are free once the previous block's dK and dQ MMAs are done
-      if (it >= 1 && !mbar_wait(&sm.dq_full, (it - 1) & 1, abort, err, kDevTimeoutMma)) {
-        ok = false;
-        break;
-      }
-      // dS row of this key: query q is element q%64 of half q/64; 16-byte
-      // chunk k (8 queries) of a half sits at chunk k ^ (key & 7) (128-byte swizzle)
+        // P^T of queries qb0..qb0+15 -> packed columns qb0 / 2 of the P^T area
+        tmem_st8(tmem + lane_off + kColPT + qb0 / 2, wp);
+        if (step < 2) {
 #pragma unroll
-      for (int k16 = 0; k16 < BQ / 8; ++k16) {
-        const uint32_t off = ((uint32_t)(k16 & 7) ^ (uint32_t)(jl & 7)) << 4;
-        st_shared_v4(hi_row[k16 >> 3] + off, wh[4 * k16], wh[4 * k16 + 1], wh[4 * k16 + 2],
-                     wh[4 * k16 + 3]);
-        st_shared_v4(lo_row[k16 >> 3] + off, wl[4 * k16], wl[4 * k16 + 1], wl[4 * k16 + 2],
-                     wl[4 * k16 + 3]);
+          for (int e = 0; e < 8; ++e) {
+            wh[step * 8 + e] = h8[e];
+            wl[step * 8 + e] = l8[e];
+          }
+          if (step == 1) {
+            if (it >= 1 && !mbar_wait(&sm.dq_full, (it - 1) & 1, abort, err, kDevTimeoutMma)) {
+              ok = false;
+              break;
+            }
+#pragma unroll
+            for (int s2 = 0; s2 < 2; ++s2) {
+              const int cc = g ? s2 : 3 - s2;
+              store8(2 * cc, wh + s2 * 8, wl + s2 * 8);
+              store8(2 * cc + 1, wh + s2 * 8 + 4, wl + s2 * 8 + 4);
+            }
+          }
+        } else {
+          store8(2 * c, h8, l8);
+          store8(2 * c + 1, h8 + 4, l8 + 4);
+        }
       }
+      if (!ok) break;
       tmem_wait_st();
       fence_proxy_async_smem();
       fence_before_sync();
       mbar_arrive(&sm.sm_done);
     }
-    // ---- dv, dk of this key
-    if (ok && mbar_wait(&sm.acc_full, 0, abort, err, kDevTimeoutMma)) {
+    // ---- dv, dk of this key (warpgroup 0)
+    if (g == 0 && ok && mbar_wait(&sm.acc_full, 0, abort, err, kDevTimeoutMma)) {
       fence_after_sync();
       uint32_t a[4][16];
 #pragma unroll
@@ -370,7 +403,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                           __uint_as_float(a[c][8 * h + 7]) * scale));
       }
     }
-  } else if (warp >= kDrainWarp0) {
+  } else if (warp < kTmaWarp) {
     // ------------------------------------------------------------ dQ drain
     // Thread te owns query row i0+te: it copies its dQ row from TMEM into its
     // own padded staging row and adds that row (256 B) into the float32
@@ -386,7 +419,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       fence_after_sync();
       uint32_t a[4][16];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld16(tmem + lane_off + col_dq(b) + c * 16, a[c]);
+      for (int c = 0; c < 4; ++c) tmem_ld16(tmem + lane_off + col_s(b) + c * 16, a[c]);
       tmem_wait_ld();
       fence_before_sync();
       mbar_arrive(&sm.dq_empty);
@@ -396,9 +429,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int g = 0; g < 4; ++g)
-            st_shared_v4(stage_s + (c * 4 + g) * 16, a[c][4 * g], a[c][4 * g + 1],
-                         a[c][4 * g + 2], a[c][4 * g + 3]);
+          for (int q4 = 0; q4 < 4; ++q4)
+            st_shared_v4(stage_s + (c * 4 + q4) * 16, a[c][4 * q4], a[c][4 * q4 + 1],
+                         a[c][4 * q4 + 2], a[c][4 * q4 + 3]);
         fence_proxy_async_smem();
         bulk_reduce_add_f32(dqacc + ((size_t)head * N + row) * HD, stage, HD * 4);
         bulk_commit_group();
@@ -432,7 +465,7 @@ attn_dq_convert_kernel(const float4* __restrict__ acc, uint4* __restrict__ dq, i
 }  // namespace
 
 cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* dout,
-                               const float* lse, const float* delta, void* dk, void* dv,
+                               const float* lse2, const float* delta, void* dk, void* dv,
                                float* dqacc, int64_t B, int64_t H, int64_t N, int causal,
                                float scale, const int* flags, unsigned* err, cudaStream_t s,
                                int* launches) {
@@ -448,7 +481,7 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
   if (e != cudaSuccess) return e;
   const int64_t n_blocks = (N + BK - 1) / BK;
   attn_bwd_tc_kernel<<<(unsigned)(n_blocks * BH), kThreads, kSmemBytes, s>>>(
-      tq, tk, tv, tdo, lse, delta, static_cast<__nv_bfloat16*>(dk),
+      tq, tk, tv, tdo, lse2, delta, static_cast<__nv_bfloat16*>(dk),
       static_cast<__nv_bfloat16*>(dv), dqacc, (int)N, (int)BH, causal, scale, scale * kLog2e,
       flags, err);
   *launches += 1;

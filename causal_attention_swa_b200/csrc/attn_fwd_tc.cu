@@ -97,9 +97,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
                    float* __restrict__ lse, int N, int BH, int n_ctiles, int causal,
                    float scale_log2, const int* __restrict__ flags, unsigned* __restrict__ err) {
-  const int L = blockIdx.x;
-  const int head = L % BH;
-  const int c = n_ctiles - 1 - L / BH;  // heaviest (latest) query tiles first
+  // Longest first: every head's latest (heaviest) query tiles, then the next.
+  const int head = blockIdx.x % BH;
+  const int c = n_ctiles - 1 - blockIdx.x / BH;
   if (flags[head] != 0) return;         // a non-finite head: the pair-by-pair kernel's
 
   extern __shared__ uint8_t smem_raw[];

@@ -13,7 +13,8 @@
 // domain), the output accumulator and the running (max, sum) in registers,
 // and streams 32-key K/V tiles through shared memory; the online softmax
 // rescales once per 16-key chunk.
-// Backward: delta_i = dout_i . out_i (prep kernel); a key-major kernel
+// Backward: delta_i = dout_i . out_i (prep kernel, also lse * log2 e, both
+// padded to whole 128-row blocks for the tensor-core kernel); a key-major kernel
 // accumulates dk_j, dv_j over the rows i that see j; a query-major kernel
 // accumulates dq_i.  Two threads share a row (32 dims each, interleaved in
 // float4 groups so the pair reads distinct banks) and combine their partial
@@ -177,16 +178,23 @@ attn_fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
 
 // ------------------------------------------------------------------ backward
 
-// delta_i = sum_d dout_id * out_id, 8 threads per row.
+// Backward row statistics, 8 threads per row, into two [heads][Npad]
+// float32 arrays (Npad = N rounded up to 128):
+//   delta[h][i] = sum_d dout_id * out_id      (0 for the padding rows)
+//   lse2[h][i]  = lse_i * log2(e)             (+inf for the padding rows)
 template <typename T>
 __global__ void __launch_bounds__(256)
 attn_bwd_prep_kernel(const T* __restrict__ out, const T* __restrict__ dout,
-                     float* __restrict__ delta, int64_t rows) {
+                     const float* __restrict__ lse, float* __restrict__ delta,
+                     float* __restrict__ lse2, int64_t N, int64_t Npad, int64_t rows_pad) {
   const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t r = g >> 3;
+  const int64_t rp = g >> 3;
   const int part = (int)(g & 7);
+  const int64_t head = rp / Npad, i = rp - head * Npad;
+  const bool real = rp < rows_pad && i < N;
   float acc = 0.f;
-  if (r < rows) {
+  if (real) {
+    const int64_t r = head * N + i;
     const T* o = out + r * D + part * 8;
     const T* d = dout + r * D + part * 8;
 #pragma unroll
@@ -195,7 +203,10 @@ attn_bwd_prep_kernel(const T* __restrict__ out, const T* __restrict__ dout,
   acc += __shfl_xor_sync(0xffffffffu, acc, 4);
   acc += __shfl_xor_sync(0xffffffffu, acc, 2);
   acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-  if (r < rows && part == 0) delta[r] = acc;
+  if (rp < rows_pad && part == 0) {
+    delta[rp] = real ? acc : 0.f;
+    lse2[rp] = real ? lse[head * N + i] * kLog2e : INFINITY;
+  }
 }
 
 constexpr int kBwdRows = 64;  // rows per block, two threads per row
@@ -207,9 +218,9 @@ __global__ void __launch_bounds__(2 * kBwdRows)
 attn_bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
                           const T* __restrict__ v, const T* __restrict__ dout,
                           const float* __restrict__ lse, const float* __restrict__ delta,
-                          T* __restrict__ dk, T* __restrict__ dv, int64_t N, int causal,
-                          float scale, float scale_log2, const int* __restrict__ flags,
-                          int select) {
+                          T* __restrict__ dk, T* __restrict__ dv, int64_t N, int64_t dstride,
+                          int causal, float scale, float scale_log2,
+                          const int* __restrict__ flags, int select) {
   const int64_t head = blockIdx.y;
   if (!head_selected(flags, head, select)) return;
   __shared__ __align__(16) float Qs[kBwdTile][D];
@@ -243,7 +254,7 @@ attn_bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
     load_rows_f32(Ds, dout + base * D, t0, nq, kBwdTile, tid, 2 * kBwdRows);
     if (tid < kBwdTile) {
       Ls[tid] = tid < nq ? lse[base + t0 + tid] * kLog2e : 0.f;
-      Es[tid] = tid < nq ? delta[base + t0 + tid] : 0.f;
+      Es[tid] = tid < nq ? delta[head * dstride + t0 + tid] : 0.f;
     }
     __syncthreads();
 #pragma unroll 2
@@ -281,8 +292,9 @@ __global__ void __launch_bounds__(2 * kBwdRows)
 attn_bwd_dq_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
                         const T* __restrict__ v, const T* __restrict__ dout,
                         const float* __restrict__ lse, const float* __restrict__ delta,
-                        T* __restrict__ dq, int64_t N, int causal, float scale,
-                        float scale_log2, const int* __restrict__ flags, int select) {
+                        T* __restrict__ dq, int64_t N, int64_t dstride, int causal,
+                        float scale, float scale_log2, const int* __restrict__ flags,
+                        int select) {
   const int64_t head = blockIdx.y;
   if (!head_selected(flags, head, select)) return;
   __shared__ __align__(16) float Ks[kBwdTile][D];
@@ -301,7 +313,7 @@ attn_bwd_dq_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
     load_half_row(qr, q + (base + i) * D, h, scale_log2);
     load_half_row(dor, dout + (base + i) * D, h, 1.f);
     lrow = lse[base + i] * kLog2e;
-    erow = delta[base + i];
+    erow = delta[head * dstride + i];
   } else {
 #pragma unroll
     for (int e = 0; e < 32; ++e) { qr[e] = 0.f; dor[e] = 0.f; }
@@ -380,18 +392,18 @@ cudaError_t fwd_simt(const void* q, const void* k, const void* v, void* out, flo
 
 template <typename T>
 cudaError_t bwd_simt(const void* q, const void* k, const void* v, const void* dout,
-                     const float* lse, const float* delta, void* dq, void* dk, void* dv,
-                     int64_t BH, int64_t N, int causal, float scale, const int* flags,
+                     const float* lse, const float* delta, int64_t dstride, void* dq, void* dk,
+                     void* dv, int64_t BH, int64_t N, int causal, float scale, const int* flags,
                      int select, cudaStream_t s) {
   dim3 grid((unsigned)((N + kBwdRows - 1) / kBwdRows), (unsigned)BH);
   attn_bwd_dkdv_simt_kernel<T><<<grid, 2 * kBwdRows, 0, s>>>(
       (const T*)q, (const T*)k, (const T*)v, (const T*)dout, lse, delta, (T*)dk, (T*)dv, N,
-      causal, scale, scale * kLog2e, flags, select);
+      dstride, causal, scale, scale * kLog2e, flags, select);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   attn_bwd_dq_simt_kernel<T><<<grid, 2 * kBwdRows, 0, s>>>(
-      (const T*)q, (const T*)k, (const T*)v, (const T*)dout, lse, delta, (T*)dq, N, causal,
-      scale, scale * kLog2e, flags, select);
+      (const T*)q, (const T*)k, (const T*)v, (const T*)dout, lse, delta, (T*)dq, N, dstride,
+      causal, scale, scale * kLog2e, flags, select);
   return cudaGetLastError();
 }
 
@@ -427,30 +439,32 @@ cudaError_t launch_attn_fwd_simt(swa_dtype dt, const void* q, const void* k, con
 }
 
 cudaError_t launch_attn_bwd_prep(swa_dtype dt, const void* out, const void* dout,
-                                 float* delta, int64_t rows, cudaStream_t s, int* launches) {
-  const int64_t threads = rows * 8;
-  const unsigned blocks = (unsigned)((threads + 255) / 256);
+                                 const float* lse, float* delta, float* lse2, int64_t BH,
+                                 int64_t N, int64_t Npad, cudaStream_t s, int* launches) {
+  const int64_t rows_pad = BH * Npad;
+  const unsigned blocks = (unsigned)((rows_pad * 8 + 255) / 256);
   if (dt == SWA_BF16)
     attn_bwd_prep_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
-        (const __nv_bfloat16*)out, (const __nv_bfloat16*)dout, delta, rows);
+        (const __nv_bfloat16*)out, (const __nv_bfloat16*)dout, lse, delta, lse2, N, Npad,
+        rows_pad);
   else
     attn_bwd_prep_kernel<float><<<blocks, 256, 0, s>>>((const float*)out, (const float*)dout,
-                                                       delta, rows);
+                                                       lse, delta, lse2, N, Npad, rows_pad);
   *launches += 1;
   return cudaGetLastError();
 }
 
 cudaError_t launch_attn_bwd_simt(swa_dtype dt, const void* q, const void* k, const void* v,
                                  const void* dout, const float* lse, const float* delta,
-                                 void* dq, void* dk, void* dv, int64_t BH, int64_t N,
-                                 int causal, float scale, const int* flags, int select,
+                                 int64_t dstride, void* dq, void* dk, void* dv, int64_t BH,
+                                 int64_t N, int causal, float scale, const int* flags, int select,
                                  cudaStream_t s, int* launches) {
   *launches += 2;
   if (dt == SWA_BF16)
-    return bwd_simt<__nv_bfloat16>(q, k, v, dout, lse, delta, dq, dk, dv, BH, N, causal, scale,
-                                   flags, select, s);
-  return bwd_simt<float>(q, k, v, dout, lse, delta, dq, dk, dv, BH, N, causal, scale, flags,
-                         select, s);
+    return bwd_simt<__nv_bfloat16>(q, k, v, dout, lse, delta, dstride, dq, dk, dv, BH, N, causal,
+                                   scale, flags, select, s);
+  return bwd_simt<float>(q, k, v, dout, lse, delta, dstride, dq, dk, dv, BH, N, causal, scale,
+                         flags, select, s);
 }
 
 }  // namespace swa

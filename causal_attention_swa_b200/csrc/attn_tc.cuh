@@ -21,9 +21,10 @@ cudaError_t launch_attn_fwd_tc(const void* q, const void* k, const void* v, void
 
 // Backward main kernel of the finite heads: dk, dv written directly; dq
 // contributions added into the float32 accumulator `dqacc` (zeroed by the
-// caller) with bulk reduce-adds.
+// caller) with bulk reduce-adds.  lse2 = lse * log2 e and delta are the
+// prep kernel's [BH][Npad] arrays.
 cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* dout,
-                               const float* lse, const float* delta, void* dk, void* dv,
+                               const float* lse2, const float* delta, void* dk, void* dv,
                                float* dqacc, int64_t B, int64_t H, int64_t N, int causal,
                                float scale, const int* flags, unsigned* err, cudaStream_t s,
                                int* launches);

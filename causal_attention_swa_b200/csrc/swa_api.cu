@@ -97,16 +97,19 @@ size_t fwd_ws(int64_t B, int64_t H, swa_dtype dt) {
   return dt == SWA_BF16 ? round_up((size_t)(B * H) * sizeof(int), 256) : 0;
 }
 
+// Backward workspace: per-head flags | delta [BH][Npad] | lse*log2e [BH][Npad]
+// | float32 dQ accumulator [BH][N][D] (bf16 only); Npad = N rounded up to 128.
 struct BwdWs {
-  size_t flags, delta, dqacc, total;
+  size_t flags, delta, lse2, dqacc, total;
 };
 
 BwdWs bwd_ws(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtype dt) {
   BwdWs w;
   w.flags = round_up((size_t)(B * H) * sizeof(int), 256);
-  w.delta = round_up((size_t)(B * H * N) * sizeof(float), 256);
+  w.delta = round_up((size_t)(B * H * swa::pad128(N)) * sizeof(float), 256);
+  w.lse2 = w.delta;
   w.dqacc = dt == SWA_BF16 ? round_up((size_t)(B * H * N * D) * sizeof(float), 256) : 0;
-  w.total = w.flags + w.delta + w.dqacc;
+  w.total = w.flags + w.delta + w.lse2 + w.dqacc;
   return w;
 }
 
@@ -211,14 +214,17 @@ swa_status swa_attn_bwd(const void* q, const void* k, const void* v, const void*
   char* base = static_cast<char*>(workspace);
   int* flags = reinterpret_cast<int*>(base);
   float* delta = reinterpret_cast<float*>(base + ws.flags);
-  float* dqacc = reinterpret_cast<float*>(base + ws.flags + ws.delta);
+  float* lse2 = reinterpret_cast<float*>(base + ws.flags + ws.delta);
+  float* dqacc = reinterpret_cast<float*>(base + ws.flags + ws.delta + ws.lse2);
+  const int64_t Npad = swa::pad128(N);
   const int c = causal ? 1 : 0;
   int launches = 0;
-  cudaError_t e = swa::launch_attn_bwd_prep(dt, out, dout, delta, BH * N, s, &launches);
+  cudaError_t e = swa::launch_attn_bwd_prep(dt, out, dout, lse, delta, lse2, BH, N, Npad, s,
+                                            &launches);
   if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_prep");
   if (dt == SWA_F32) {
-    e = swa::launch_attn_bwd_simt(dt, q, k, v, dout, lse, delta, dq, dk, dv, BH, N, c, scale,
-                                  nullptr, 0, s, &launches);
+    e = swa::launch_attn_bwd_simt(dt, q, k, v, dout, lse, delta, Npad, dq, dk, dv, BH, N, c,
+                                  scale, nullptr, 0, s, &launches);
     if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_simt");
   } else {
     e = cudaMemsetAsync(flags, 0, (size_t)BH * sizeof(int), s);
@@ -233,14 +239,14 @@ swa_status swa_attn_bwd(const void* q, const void* k, const void* v, const void*
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dq accumulator)");
     {
       ProfScope ps(SWA_KERNEL_ATTN_BWD, s);
-      e = swa::launch_attn_bwd_tc(q, k, v, dout, lse, delta, dk, dv, dqacc, B, H, N, c, scale,
+      e = swa::launch_attn_bwd_tc(q, k, v, dout, lse2, delta, dk, dv, dqacc, B, H, N, c, scale,
                                   flags, err, s, &launches);
     }
     if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_tc");
     e = swa::launch_attn_dq_convert(dqacc, dq, BH, N, scale, flags, s, &launches);
     if (e != cudaSuccess) return cuda_fail(e, "attn_dq_convert");
-    e = swa::launch_attn_bwd_simt(dt, q, k, v, dout, lse, delta, dq, dk, dv, BH, N, c, scale,
-                                  flags, 1, s, &launches);
+    e = swa::launch_attn_bwd_simt(dt, q, k, v, dout, lse, delta, Npad, dq, dk, dv, BH, N, c,
+                                  scale, flags, 1, s, &launches);
     if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_simt(non-finite heads)");
   }
   t_launches = launches;

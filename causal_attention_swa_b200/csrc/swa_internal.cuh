@@ -19,6 +19,7 @@ enum DeviceError : unsigned {
   kDevTimeoutOther = 4,
 };
 
+__host__ __device__ __forceinline__ int64_t pad128(int64_t n) { return (n + 127) / 128 * 128; }
 __host__ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -62,13 +63,16 @@ cudaError_t launch_attn_fwd_simt(swa_dtype dt, const void* q, const void* k, con
                                  float scale, const int* flags, int select, cudaStream_t s,
                                  int* launches);
 
+// delta[h][i] and lse2[h][i] = lse * log2 e, both [BH][Npad] (Npad = N
+// rounded up to 128; padding rows 0 and +inf).
 cudaError_t launch_attn_bwd_prep(swa_dtype dt, const void* out, const void* dout,
-                                 float* delta, int64_t rows, cudaStream_t s, int* launches);
+                                 const float* lse, float* delta, float* lse2, int64_t BH,
+                                 int64_t N, int64_t Npad, cudaStream_t s, int* launches);
 
 cudaError_t launch_attn_bwd_simt(swa_dtype dt, const void* q, const void* k, const void* v,
                                  const void* dout, const float* lse, const float* delta,
-                                 void* dq, void* dk, void* dv, int64_t BH, int64_t N,
-                                 int causal, float scale, const int* flags, int select,
+                                 int64_t dstride, void* dq, void* dk, void* dv, int64_t BH,
+                                 int64_t N, int causal, float scale, const int* flags, int select,
                                  cudaStream_t s, int* launches);
 
 size_t nw_partials_bytes(int64_t M, int64_t S);
