@@ -41,6 +41,7 @@ NW_M = NW_S = 16384
 NW_SEED = 2
 H_BW = 0.5
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+SM_MAX_MHZ = 1965.0
 
 # kernel id -> (name, source file whose hash keys the recorded ncu traffic)
 KERNELS = {
@@ -334,6 +335,20 @@ def run_ours(args, info):
         "peak_source": f"{pk['source']} bf16 dense (burst)",
         "flops_per_launch": bwd_fl, "ms_per_launch": dom_ms,
     }
+    # the other main kernels against their own bounds: the forward against the
+    # bf16 tensor peak, the regrid against MUFU (148 SMs x 16 ex2/clk x max clock)
+    mufu_peak = 148 * 16 * SM_MAX_MHZ * 1e6 / 1e9  # Gpair/s
+    nw_rate = NW_M * NW_S / (kernel_ms[3] * 1e-3) / 1e9 if kernel_ms[3] else None
+    fwd_rate = fwd_fl / (kernel_ms[1] * 1e-3) / 1e12 if kernel_ms[1] else None
+    rooflines = {
+        "attn_fwd": {"bound": "tensor", "achieved": fwd_rate, "peak": pk["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": fwd_rate / pk["bf16_tflops"] if fwd_rate else None,
+                     "traffic": recorded_traffic(1)},
+        "nw_regrid": {"bound": "alu", "achieved": nw_rate, "peak": mufu_peak, "unit": "Gpair/s",
+                      "frac": nw_rate / mufu_peak if nw_rate else None,
+                      "traffic": recorded_traffic(3),
+                      "peak_source": "148 SMs x 16 MUFU ex2/clk x 1965 MHz (one ex2 per pair)"},
+    }
     breakdown = {
         "attn_fwd_ms": kernel_ms[1], "attn_bwd_ms": kernel_ms[2], "nw_ms": kernel_ms[3],
         "attn_fwd_tflops": fwd_fl / (kernel_ms[1] * 1e-3) / 1e12 if kernel_ms[1] else None,
@@ -368,7 +383,7 @@ def run_ours(args, info):
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": timed_launches, "clocks": clocks.summary(),
-            "breakdown": breakdown,
+            "breakdown": breakdown, "rooflines": rooflines,
         }
         print(json.dumps(line), flush=True)
     sdist.shutdown()
