@@ -11,20 +11,19 @@
 // over the pairs that exist (j <= i when causal).
 //
 // Block = one 128-key block j of one head (K_j, V_j stay in shared memory)
-// and 512 threads; it walks the 128-query blocks i that see j:
-//   warps 0-7   "softmax-grad", two warpgroups: thread t of warpgroup g owns
-//               key j0 + t (TMEM lane t) and queries 64g..64g+63 of the
-//               block; from S^T and dP^T it forms P^T (bf16, back into TMEM
-//               for dV) and dS (float32, split into bf16 hi + lo parts,
-//               written to shared memory); warpgroup 0 finally stores dv and
-//               dk of its key
-//   warps 8-11  dQ drain: dQ_i (TMEM lane = query) -> a shared staging row
-//               per thread -> cp.reduce.async.bulk add.f32 into the float32
-//               dQ accumulator
-//   warp  12    TMA producer: K_j, V_j once; Q_i, dO_i, lse_i, delta_i into a
+// and 576 threads; it walks the 128-query blocks i that see j:
+//   warps 0-15  compute, four warpgroups: thread t of warpgroup w owns key
+//               j0 + t (TMEM lane t) and queries 32w..32w+31 of each block.
+//               From S^T and dP^T (one batched TMEM load per block) it forms
+//               P^T (bf16, written back over its own dP^T columns for the
+//               dV MMA) and dS (float32 -> bf16 hi + lo, into shared
+//               memory); then it drains columns 16w..16w+15 of the previous
+//               block's dQ (TMEM lane = query) into the float32 dQ
+//               accumulator with vector red.add; at the end warpgroup w
+//               stores columns 16w..16w+15 of its key's dv and dk
+//   warp  16    TMA producer: K_j, V_j once; Q_i, dO_i, lse_i, delta_i into a
 //               2-stage ring
-//   warp  13    MMA issuer (one thread), TMEM owner
-//   warps 14-15 idle
+//   warp  17    MMA issuer (one thread), TMEM owner
 // Per query block, seven MMAs (M = 128, K = 64 or 128):
 //   S^T = K_j Q_i^T              (A = K smem K-major, B = Q smem K-major)
 //   dP^T = V_j dO_i^T            (A = V, B = dO, both K-major)
@@ -36,20 +35,15 @@
 // by the cancellation in sum_j dS_ij k_j (sum_j dS_ij = 0), costs dq about
 // 2% of its row RMS at N = 2048.  One [128 keys][128 queries] tile layout
 // (rows = keys, 128-byte swizzle, two 64-query halves) is both the K-major
-// A operand of dK and the MN-major A operand of dQ.
+// A operand of dK and the MN-major A operand of dQ; it is double-buffered
+// by query block, so block i's dS is written while block i-1's dK and dQ
+// MMAs still read the other buffer.
 // TMEM (512 columns): S^T buffers [0,128) and [128,256) (the block's dQ in
-// the first 64 columns once S^T is consumed), dP^T [256,384) with P^T
-// (bf16, two per column) in its columns [32,96), dV [384,448), dK
-// [448,512).  P^T columns 32..63 are dP^T columns of queries 32..63 and
-// P^T columns 64..95 those of queries 64..95: each warpgroup overwrites
-// only columns it has itself read (warpgroup 0 walks its queries
-// downwards, warpgroup 1 upwards), so the two never race.  MMAs of one
-// thread execute in issue order, so a later MMA may overwrite TMEM an
-// earlier one reads.
-// Issue order: S^T_i+1 (other buffer) as soon as its buffer is free; once
-// the softmax-grad warps are done with block i: dV_i, dP^T_i+1, dK_i, dQ_i.
-// The softmax-grad warps hold the first half of a block's dS in registers
-// until block i-1's dK and dQ MMAs have released the dS tiles.
+// the first 64 columns once S^T is consumed), dP^T [256,384) (warpgroup w
+// writes the P^T of its 32 queries over its own columns 32w..32w+15 after
+// loading them; the dV MMA takes each 16-query group's A from there),
+// dV [384,448), dK [448,512).  MMAs of one thread execute in issue order,
+// so a later MMA may overwrite TMEM an earlier one reads.
 // Causal: only query blocks i >= j are visited; in the diagonal block (and
 // past N on a ragged tail) P and dS of a masked pair are set to 0 by select.
 // This kernel takes only heads whose V and dout are all finite, so 0 times
@@ -67,28 +61,27 @@ constexpr int BK = 128;                 // keys per block
 constexpr int BQ = 128;                 // queries per block
 constexpr int HD = 64;
 constexpr int kTileBytes = 128 * HD * 2;
-constexpr int kThreads = 512;
-constexpr int kGradThreads = 256;       // two softmax-grad warpgroups
-constexpr int kDrainWarp0 = 8;
-constexpr int kTmaWarp = 12;
-constexpr int kMmaWarp = 13;
+constexpr int kComputeThreads = 512;    // four warpgroups
+constexpr int kTmaWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int kThreads = 576;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColDP = 256, kColPT = kColDP + 32, kColDV = 384, kColDK = 448;
-constexpr int kStageRow = HD + 4;  // floats per staged dQ row: 272 B, so row starts rotate banks
+constexpr uint32_t kColDP = 256, kColDV = 384, kColDK = 448;
 constexpr int kHeadGroup = 4;      // heads scheduled together (their dQ, Q, dO share L2)
 
 __device__ __forceinline__ uint32_t col_s(int b) { return b ? 128u : 0u; }
 
+// Shared memory (227 KB of the 227 KB a block may use): the dynamic base is
+// expected 1024-byte aligned (the kernel checks and reports otherwise).
 struct __align__(1024) Smem {
   uint8_t k[kTileBytes];
   uint8_t v[kTileBytes];
   uint8_t q[2][kTileBytes];
   uint8_t dout[2][kTileBytes];
-  uint8_t ds_hi[2][kTileBytes];  // dS tiles [128 keys][queries 0-63 | 64-127]
-  uint8_t ds_lo[2][kTileBytes];
-  float dq[BQ * kStageRow];      // dQ staging, one padded row per drain thread
-  float lse[2][BQ];              // lse_i * log2(e) of each staged query block (+inf past N)
-  float delta[2][BQ];            // delta_i of each staged query block (0 past N)
+  uint8_t ds_hi[2][2][kTileBytes];  // [buffer][query half]: [128 keys][64 queries]
+  uint8_t ds_lo[2][2][kTileBytes];
+  float lse[2][BQ];                 // lse_i * log2(e) of each staged query block (+inf past N)
+  float delta[2][BQ];               // delta_i of each staged query block (0 past N)
   uint64_t kv_full;
   uint64_t qd_full[2];
   uint64_t qd_empty[2];
@@ -103,7 +96,8 @@ struct __align__(1024) Smem {
   int abort;
 };
 
-constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+constexpr size_t kSmemBytes = sizeof(Smem);
+static_assert(kSmemBytes <= 232448, "shared memory");
 
 __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
   const long long t0 = clock64();
@@ -133,9 +127,12 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int head = group * kHeadGroup + r % g_heads;
   if (flags[head] != 0) return;
 
-  extern __shared__ uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                      ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {  // the swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) atomicCAS(err, 0u, (unsigned)kDevSmemAlign);
+    return;
+  }
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
@@ -151,9 +148,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(&sm.s_full[s], 1);
     }
     mbar_init(&sm.dp_full, 1);
-    mbar_init(&sm.sm_done, kGradThreads);
+    mbar_init(&sm.sm_done, kComputeThreads);
     mbar_init(&sm.dq_full, 1);
-    mbar_init(&sm.dq_empty, 128);
+    mbar_init(&sm.dq_empty, kComputeThreads);
     mbar_init(&sm.acc_full, 1);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
@@ -196,7 +193,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // --------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    {  // the whole warp runs the issue loop; one elected lane issues
       constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T: both K-major
       constexpr uint32_t id_mn = idesc_bf16_f32(128, 64, 0, 1);   // dV, dK: B MN-major
       constexpr uint32_t id_dq = idesc_bf16_f32(128, 64, 1, 1);   // dQ: A and B MN-major
@@ -204,79 +201,99 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       auto issue_kk = [&](uint32_t d_col, uint32_t a0, uint32_t b0) {
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk)
-          mma_ss(tmem + d_col, desc_sw128(a0 + kk * 32, 16, 1024),
+          mma_ss_elect(tmem + d_col, desc_sw128(a0 + kk * 32, 16, 1024),
                  desc_sw128(b0 + kk * 32, 16, 1024), id_kk, kk > 0 ? 1u : 0u);
       };
-      // dK += dS^T Q_i from one dS tile: A rows = keys, K = queries (K-major;
-      // queries 64-127 in the second half tile)
+      // dK += dS^T Q_i from one dS tile pair: A rows = keys, K = queries
+      // (K-major; queries 64-127 in the second half tile)
       auto issue_dk = [&](const uint8_t (*ds)[kTileBytes], uint32_t q0, bool first) {
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk)
-          mma_ss(tmem + kColDK, desc_sw128(smem_u32(ds[kk >> 2]) + (kk & 3) * 32, 16, 1024),
+          mma_ss_elect(tmem + kColDK, desc_sw128(smem_u32(ds[kk >> 2]) + (kk & 3) * 32, 16, 1024),
                  desc_sw128(q0 + kk * 2048, 8192, 1024), id_mn, (!first || kk > 0) ? 1u : 0u);
       };
-      // dQ_i (+)= dS K_j from one dS tile: A M = queries (MN-major, the two
-      // 64-query halves 16 KB apart), K = keys
+      // dQ_i (+)= dS K_j from one dS tile pair: A M = queries (MN-major, the
+      // two 64-query halves 16 KB apart), K = keys
       auto issue_dq = [&](const uint8_t (*ds)[kTileBytes], uint32_t col, bool first) {
         const uint32_t a0 = smem_u32(ds[0]);
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk)
-          mma_ss(tmem + col, desc_sw128(a0 + kk * 2048, kTileBytes, 1024),
+          mma_ss_elect(tmem + col, desc_sw128(a0 + kk * 2048, kTileBytes, 1024),
                  desc_sw128(k_s + kk * 2048, 8192, 1024), id_dq, (!first || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(&sm.kv_full, 0, abort, err, kDevTimeoutFull) &&
                 mbar_wait(&sm.qd_full[0], 0, abort, err, kDevTimeoutFull);
       if (ok) {
         issue_kk(col_s(0), k_s, smem_u32(sm.q[0]));
-        mma_commit(&sm.s_full[0]);
+        mma_commit_elect(&sm.s_full[0]);
         issue_kk(kColDP, v_s, smem_u32(sm.dout[0]));
-        mma_commit(&sm.dp_full);
+        mma_commit_elect(&sm.dp_full);
       }
       for (int it = 0; ok && it < n_q; ++it) {
         const int b = it & 1;
         const bool next = it + 1 < n_q;
-        // the other S^T buffer holds dQ_it-1 until the drain has read it
+        // the other S^T buffer holds dQ_it-1 until the compute warps drained it
         if (it >= 1 && !mbar_wait(&sm.dq_empty, (it - 1) & 1, abort, err, kDevTimeoutOther)) break;
         if (next) {
           if (!mbar_wait(&sm.qd_full[b ^ 1], ((it + 1) >> 1) & 1, abort, err, kDevTimeoutFull))
             break;
           issue_kk(col_s(b ^ 1), k_s, smem_u32(sm.q[b ^ 1]));
-          mma_commit(&sm.s_full[b ^ 1]);
+          mma_commit_elect(&sm.s_full[b ^ 1]);
         }
         if (!mbar_wait(&sm.sm_done, it & 1, abort, err, kDevTimeoutOther)) break;
         fence_after_sync();
-        {  // dV += P^T dO_i  (P^T in the dP^T region, read before dP^T_it+1 lands)
+        {  // dV += P^T dO_i: 16-query group kk's P^T is in dP^T columns 32(kk/2) + 8(kk%2)
           const uint32_t b0 = smem_u32(sm.dout[b]);
 #pragma unroll
           for (int kk = 0; kk < BQ / 16; ++kk)
-            mma_ts(tmem + kColDV, tmem + kColPT + kk * 8, desc_sw128(b0 + kk * 2048, 8192, 1024),
-                   id_mn, (it > 0 || kk > 0) ? 1u : 0u);
+            mma_ts_elect(tmem + kColDV, tmem + kColDP + 32 * (kk >> 1) + 8 * (kk & 1),
+                   desc_sw128(b0 + kk * 2048, 8192, 1024), id_mn, (it > 0 || kk > 0) ? 1u : 0u);
         }
         if (next) {
           issue_kk(kColDP, v_s, smem_u32(sm.dout[b ^ 1]));
-          mma_commit(&sm.dp_full);
+          mma_commit_elect(&sm.dp_full);
         }
         const uint32_t q0 = smem_u32(sm.q[b]);
-        issue_dk(sm.ds_hi, q0, it == 0);
-        issue_dk(sm.ds_lo, q0, false);
-        issue_dq(sm.ds_hi, col_s(b), true);
-        issue_dq(sm.ds_lo, col_s(b), false);
-        mma_commit(&sm.dq_full);
-        mma_commit(&sm.qd_empty[b]);
+        issue_dk(sm.ds_hi[b], q0, it == 0);
+        issue_dk(sm.ds_lo[b], q0, false);
+        issue_dq(sm.ds_hi[b], col_s(b), true);
+        issue_dq(sm.ds_lo[b], col_s(b), false);
+        mma_commit_elect(&sm.dq_full);
+        mma_commit_elect(&sm.qd_empty[b]);
       }
-      mma_commit(&sm.acc_full);
-      mma_commit(&sm.drain);
+      mma_commit_elect(&sm.acc_full);
+      mma_commit_elect(&sm.drain);
       wait_drain(&sm.drain, 0);
     }
     __syncwarp();
-  } else if (warp < 8) {
-    // -------------------------------------------------------- softmax-grad
-    const int g = warp >> 2;          // query half of this warpgroup
-    const int jl = tid & 127;         // key row within the block = TMEM lane
-    const int jg = j0 + jl;
+  } else {
+    // ------------------------------------------------------------- compute
+    const int w = warp >> 2;        // warpgroup: queries 32w..32w+31
+    const int tl = (warp & 3) * 32 + lane;  // TMEM lane: key row here, query row in dQ
+    const int jg = j0 + tl;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t hi_row = smem_u32(sm.ds_hi[g]) + jl * 128;
-    const uint32_t lo_row = smem_u32(sm.ds_lo[g]) + jl * 128;
+    const int qw = 32 * w;                  // first query of this warpgroup in a block
+    const int half = w >> 1;
+    const uint32_t chunk0 = 4u * (uint32_t)(w & 1);  // first 16-byte chunk in the half-tile row
+    // dQ of the block before: rows = queries, this warpgroup's 16 columns
+    auto drain_dq = [&](int itp) -> bool {
+      if (!mbar_wait(&sm.dq_full, itp & 1, abort, err, kDevTimeoutMma)) return false;
+      fence_after_sync();
+      uint32_t a[16];
+      tmem_ld16(tmem + lane_off + col_s(itp & 1) + 16 * w, a);
+      tmem_wait_ld();
+      fence_before_sync();
+      mbar_arrive(&sm.dq_empty);
+      const int row = (ib0 + itp) * BQ + tl;
+      if (row < N) {
+        float* dst = dqacc + ((size_t)head * N + row) * HD + 16 * w;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          red_add_v4(dst + 4 * c, __uint_as_float(a[4 * c]), __uint_as_float(a[4 * c + 1]),
+                     __uint_as_float(a[4 * c + 2]), __uint_as_float(a[4 * c + 3]));
+      }
+      return true;
+    };
     bool ok = true;
     for (int it = 0; it < n_q; ++it) {
       const int b = it & 1;
@@ -290,154 +307,89 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         break;
       }
       fence_after_sync();
-      // Four 16-query chunks of this half: warpgroup 0 walks them downwards,
-      // warpgroup 1 upwards, so P^T lands only on dP^T columns already read.
-      // The first two chunks' dS are held in registers until block i-1's dK
-      // and dQ MMAs release the dS tiles.  Query qh of a half is element qh
-      // of that half's tile row; 16-byte chunk k (8 queries) sits at chunk
-      // k ^ (key & 7) (128-byte swizzle).
-      uint32_t wh[16], wl[16];
-      auto store8 = [&](int k8, const uint32_t* h4, const uint32_t* l4) {
-        const uint32_t off = ((uint32_t)k8 ^ (uint32_t)(jl & 7)) << 4;
-        st_shared_v4(hi_row + off, h4[0], h4[1], h4[2], h4[3]);
-        st_shared_v4(lo_row + off, l4[0], l4[1], l4[2], l4[3]);
-      };
+      uint32_t sv[32], dpv[32];
+      tmem_ld16(tmem + lane_off + col_s(b) + qw, *reinterpret_cast<uint32_t(*)[16]>(sv));
+      tmem_ld16(tmem + lane_off + col_s(b) + qw + 16, *reinterpret_cast<uint32_t(*)[16]>(sv + 16));
+      tmem_ld16(tmem + lane_off + kColDP + qw, *reinterpret_cast<uint32_t(*)[16]>(dpv));
+      tmem_ld16(tmem + lane_off + kColDP + qw + 16,
+                *reinterpret_cast<uint32_t(*)[16]>(dpv + 16));
+      tmem_wait_ld();
+      uint32_t wp[16], wh[16], wl[16];
 #pragma unroll
-      for (int step = 0; step < 4; ++step) {
-        const int c = g ? step : 3 - step;  // chunk within the half
-        const int qb0 = g * 64 + c * 16;     // first query of the chunk within the block
-        uint32_t sv[16], dv16[16];
-        tmem_ld16(tmem + lane_off + col_s(b) + qb0, sv);
-        tmem_ld16(tmem + lane_off + kColDP + qb0, dv16);
-        tmem_wait_ld();
-        uint32_t wp[8], h8[8], l8[8];
+      for (int e = 0; e < 16; ++e) {
+        float p2[2], ds2[2];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float p2[2], ds2[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int q = qb0 + 2 * e + h;  // query within the block
-            float p = ex2(fmaf(__uint_as_float(sv[2 * e + h]), scale_log2, -sm.lse[b][q]));
-            float ds = p * (__uint_as_float(dv16[2 * e + h]) - sm.delta[b][q]);
-            if (need_mask) {
-              const int ig = i0 + q;
-              if (ig >= N || jg >= N || (causal && ig < jg)) {
-                p = 0.f;
-                ds = 0.f;
-              }
+        for (int h = 0; h < 2; ++h) {
+          const int q = qw + 2 * e + h;  // query within the block
+          float p = ex2(fmaf(__uint_as_float(sv[2 * e + h]), scale_log2, -sm.lse[b][q]));
+          float ds = p * (__uint_as_float(dpv[2 * e + h]) - sm.delta[b][q]);
+          if (need_mask) {
+            const int ig = i0 + q;
+            if (ig >= N || jg >= N || (causal && ig < jg)) {
+              p = 0.f;
+              ds = 0.f;
             }
-            p2[h] = p;
-            ds2[h] = ds;
           }
-          wp[e] = pack_bf16(p2[0], p2[1]);
-          h8[e] = pack_bf16(ds2[0], ds2[1]);
-          l8[e] = pack_bf16(ds2[0] - bf16lo(h8[e]), ds2[1] - bf16hi(h8[e]));
+          p2[h] = p;
+          ds2[h] = ds;
         }
-        // P^T of queries qb0..qb0+15 -> packed columns qb0 / 2 of the P^T area
-        tmem_st8(tmem + lane_off + kColPT + qb0 / 2, wp);
-        if (step < 2) {
+        wp[e] = pack_bf16(p2[0], p2[1]);
+        wh[e] = pack_bf16(ds2[0], ds2[1]);
+        wl[e] = pack_bf16(ds2[0] - bf16lo(wh[e]), ds2[1] - bf16hi(wh[e]));
+      }
+      // P^T of this warpgroup's 32 queries over its own (already loaded) dP^T columns
+      tmem_st16(tmem + lane_off + kColDP + qw, wp);
+      // dS row of this key into buffer b: query q is element q % 64 of half
+      // q / 64; 16-byte chunk k (8 queries) of a half-tile row sits at chunk
+      // k ^ (key & 7) (128-byte swizzle)
+      {
+        const uint32_t hi_row = smem_u32(sm.ds_hi[b][half]) + tl * 128;
+        const uint32_t lo_row = smem_u32(sm.ds_lo[b][half]) + tl * 128;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            wh[step * 8 + e] = h8[e];
-            wl[step * 8 + e] = l8[e];
-          }
-          if (step == 1) {
-            if (it >= 1 && !mbar_wait(&sm.dq_full, (it - 1) & 1, abort, err, kDevTimeoutMma)) {
-              ok = false;
-              break;
-            }
-#pragma unroll
-            for (int s2 = 0; s2 < 2; ++s2) {
-              const int cc = g ? s2 : 3 - s2;
-              store8(2 * cc, wh + s2 * 8, wl + s2 * 8);
-              store8(2 * cc + 1, wh + s2 * 8 + 4, wl + s2 * 8 + 4);
-            }
-          }
-        } else {
-          store8(2 * c, h8, l8);
-          store8(2 * c + 1, h8 + 4, l8 + 4);
+        for (int g = 0; g < 4; ++g) {
+          const uint32_t off = ((chunk0 + g) ^ (uint32_t)(tl & 7)) << 4;
+          st_shared_v4(hi_row + off, wh[4 * g], wh[4 * g + 1], wh[4 * g + 2], wh[4 * g + 3]);
+          st_shared_v4(lo_row + off, wl[4 * g], wl[4 * g + 1], wl[4 * g + 2], wl[4 * g + 3]);
         }
       }
-      if (!ok) break;
+      if (it >= 1 && !drain_dq(it - 1)) {
+        ok = false;
+        break;
+      }
       tmem_wait_st();
       fence_proxy_async_smem();
       fence_before_sync();
       mbar_arrive(&sm.sm_done);
     }
-    // ---- dv, dk of this key (warpgroup 0)
-    if (g == 0 && ok && mbar_wait(&sm.acc_full, 0, abort, err, kDevTimeoutMma)) {
+    if (ok && n_q > 0) ok = drain_dq(n_q - 1);
+    // ---- columns 16w..16w+15 of this key's dv and dk
+    if (ok && mbar_wait(&sm.acc_full, 0, abort, err, kDevTimeoutMma)) {
       fence_after_sync();
-      uint32_t a[4][16];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld16(tmem + lane_off + kColDV + c * 16, a[c]);
+      uint32_t av[16], ak[16];
+      tmem_ld16(tmem + lane_off + kColDV + 16 * w, av);
+      tmem_ld16(tmem + lane_off + kColDK + 16 * w, ak);
       tmem_wait_ld();
       if (jg < N) {
-        uint4* dst = reinterpret_cast<uint4*>(dv + ((size_t)head * N + jg) * HD);
+        uint4* dvd = reinterpret_cast<uint4*>(dv + ((size_t)head * N + jg) * HD + 16 * w);
+        uint4* dkd = reinterpret_cast<uint4*>(dk + ((size_t)head * N + jg) * HD + 16 * w);
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-            dst[2 * c + h] = make_uint4(
-                pack_bf16(__uint_as_float(a[c][8 * h + 0]), __uint_as_float(a[c][8 * h + 1])),
-                pack_bf16(__uint_as_float(a[c][8 * h + 2]), __uint_as_float(a[c][8 * h + 3])),
-                pack_bf16(__uint_as_float(a[c][8 * h + 4]), __uint_as_float(a[c][8 * h + 5])),
-                pack_bf16(__uint_as_float(a[c][8 * h + 6]), __uint_as_float(a[c][8 * h + 7])));
-      }
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld16(tmem + lane_off + kColDK + c * 16, a[c]);
-      tmem_wait_ld();
-      if (jg < N) {
-        uint4* dst = reinterpret_cast<uint4*>(dk + ((size_t)head * N + jg) * HD);
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-            dst[2 * c + h] = make_uint4(
-                pack_bf16(__uint_as_float(a[c][8 * h + 0]) * scale,
-                          __uint_as_float(a[c][8 * h + 1]) * scale),
-                pack_bf16(__uint_as_float(a[c][8 * h + 2]) * scale,
-                          __uint_as_float(a[c][8 * h + 3]) * scale),
-                pack_bf16(__uint_as_float(a[c][8 * h + 4]) * scale,
-                          __uint_as_float(a[c][8 * h + 5]) * scale),
-                pack_bf16(__uint_as_float(a[c][8 * h + 6]) * scale,
-                          __uint_as_float(a[c][8 * h + 7]) * scale));
+        for (int h = 0; h < 2; ++h) {
+          dvd[h] = make_uint4(
+              pack_bf16(__uint_as_float(av[8 * h + 0]), __uint_as_float(av[8 * h + 1])),
+              pack_bf16(__uint_as_float(av[8 * h + 2]), __uint_as_float(av[8 * h + 3])),
+              pack_bf16(__uint_as_float(av[8 * h + 4]), __uint_as_float(av[8 * h + 5])),
+              pack_bf16(__uint_as_float(av[8 * h + 6]), __uint_as_float(av[8 * h + 7])));
+          dkd[h] = make_uint4(pack_bf16(__uint_as_float(ak[8 * h + 0]) * scale,
+                                        __uint_as_float(ak[8 * h + 1]) * scale),
+                              pack_bf16(__uint_as_float(ak[8 * h + 2]) * scale,
+                                        __uint_as_float(ak[8 * h + 3]) * scale),
+                              pack_bf16(__uint_as_float(ak[8 * h + 4]) * scale,
+                                        __uint_as_float(ak[8 * h + 5]) * scale),
+                              pack_bf16(__uint_as_float(ak[8 * h + 6]) * scale,
+                                        __uint_as_float(ak[8 * h + 7]) * scale));
+        }
       }
     }
-  } else if (warp < kTmaWarp) {
-    // ------------------------------------------------------------ dQ drain
-    // Thread te owns query row i0+te: it copies its dQ row from TMEM into its
-    // own padded staging row and adds that row (256 B) into the float32
-    // accumulator with one bulk reduce; before rewriting the row it waits for
-    // its previous bulk read to finish.
-    const int te = tid - kDrainWarp0 * 32;  // query row within the block = TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    float* stage = sm.dq + te * kStageRow;
-    const uint32_t stage_s = smem_u32(stage);
-    for (int it = 0; it < n_q; ++it) {
-      const int b = it & 1;
-      if (!mbar_wait(&sm.dq_full, it & 1, abort, err, kDevTimeoutMma)) break;
-      fence_after_sync();
-      uint32_t a[4][16];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld16(tmem + lane_off + col_s(b) + c * 16, a[c]);
-      tmem_wait_ld();
-      fence_before_sync();
-      mbar_arrive(&sm.dq_empty);
-      const int row = (ib0 + it) * BQ + te;
-      if (row < N) {
-        bulk_wait_group_read0();
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            st_shared_v4(stage_s + (c * 4 + q4) * 16, a[c][4 * q4], a[c][4 * q4 + 1],
-                         a[c][4 * q4 + 2], a[c][4 * q4 + 3]);
-        fence_proxy_async_smem();
-        bulk_reduce_add_f32(dqacc + ((size_t)head * N + row) * HD, stage, HD * 4);
-        bulk_commit_group();
-      }
-    }
-    bulk_wait_group0();
   }
 
   fence_before_sync();

@@ -171,7 +171,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // --------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    {  // the whole warp runs the issue loop; one elected lane issues
       constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BN, 0, 0);  // Q, K both K-major
       constexpr uint32_t idesc_o = idesc_bf16_f32(BM, HD, 0, 1);  // V is MN-major (dims contiguous)
       int k_ready = -1;
@@ -188,15 +188,15 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint32_t b0 = smem_u32(sm.k[j % kStages]);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk)
-          mma_ss(tmem + col_s(t), desc_sw128(a0 + kk * 32, 16, 1024),
+          mma_ss_elect(tmem + col_s(t), desc_sw128(a0 + kk * 32, 16, 1024),
                  desc_sw128(b0 + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-        mma_commit(&sm.s_full[t]);
+        mma_commit_elect(&sm.s_full[t]);
       };
       auto issue_pv = [&](int t, int j) {
         const uint32_t b0 = smem_u32(sm.v[j % kStages]);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8,
+          mma_ts_elect(tmem + col_o(t), tmem + col_s(t) + kk * 8,
                  desc_sw128(b0 + kk * 2048, 8192, 1024), idesc_o,
                  (j > 0 || kk > 0) ? 1u : 0u);
       };
@@ -218,13 +218,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             if (!wait_k(j + 1)) { ok = false; break; }
             issue_s(t, j + 1);
           } else {
-            mma_commit(&sm.o_final[t]);
+            mma_commit_elect(&sm.o_final[t]);
           }
         }
-        mma_commit(&sm.kv_empty[s]);
+        mma_commit_elect(&sm.kv_empty[s]);
       }
       // every MMA this thread issued has finished before TMEM is released
-      mma_commit(&sm.drain);
+      mma_commit_elect(&sm.drain);
       wait_unbounded_by_abort(&sm.drain, 0);
     }
     __syncwarp();

@@ -17,6 +17,7 @@ enum DeviceError : unsigned {
   kDevTimeoutEmpty = 2,  // a wait for an "empty" (slot released) barrier ran out
   kDevTimeoutMma = 3,    // a wait for an MMA completion ran out
   kDevTimeoutOther = 4,
+  kDevSmemAlign = 5,     // dynamic shared memory not 1024-byte aligned (kernel did nothing)
 };
 
 __host__ __device__ __forceinline__ int64_t pad128(int64_t n) { return (n + 127) / 128 * 128; }
