@@ -198,28 +198,25 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       constexpr uint32_t id_mn = idesc_bf16_f32(128, 64, 0, 1);   // dV, dK: B MN-major
       constexpr uint32_t id_dq = idesc_bf16_f32(128, 64, 1, 1);   // dQ: A and B MN-major
       const uint32_t k_s = smem_u32(sm.k), v_s = smem_u32(sm.v);
+      // Runs of MMAs from one asm block; descriptor steps in 16-byte units:
+      // K-major operands +32 B (2) per K = 16 step, MN-major +2048 B (128).
       auto issue_kk = [&](uint32_t d_col, uint32_t a0, uint32_t b0) {
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk)
-          mma_ss_elect(tmem + d_col, desc_sw128(a0 + kk * 32, 16, 1024),
-                 desc_sw128(b0 + kk * 32, 16, 1024), id_kk, kk > 0 ? 1u : 0u);
+        mma_ss_run<4, 2, 0, 2>(tmem + d_col, desc_sw128(a0, 16, 1024), desc_sw128(b0, 16, 1024),
+                               id_kk, 0u);
       };
       // dK += dS^T Q_i from one dS tile pair: A rows = keys, K = queries
       // (K-major; queries 64-127 in the second half tile)
+      // (step 4 jumps to the second half tile: +16 KB = 1024 units in all)
       auto issue_dk = [&](const uint8_t (*ds)[kTileBytes], uint32_t q0, bool first) {
-#pragma unroll
-        for (int kk = 0; kk < BQ / 16; ++kk)
-          mma_ss_elect(tmem + kColDK, desc_sw128(smem_u32(ds[kk >> 2]) + (kk & 3) * 32, 16, 1024),
-                 desc_sw128(q0 + kk * 2048, 8192, 1024), id_mn, (!first || kk > 0) ? 1u : 0u);
+        mma_ss_run<8, 2, kTileBytes / 16 - 8, 128>(
+            tmem + kColDK, desc_sw128(smem_u32(ds[0]), 16, 1024), desc_sw128(q0, 8192, 1024),
+            id_mn, first ? 0u : 1u);
       };
       // dQ_i (+)= dS K_j from one dS tile pair: A M = queries (MN-major, the
       // two 64-query halves 16 KB apart), K = keys
       auto issue_dq = [&](const uint8_t (*ds)[kTileBytes], uint32_t col, bool first) {
-        const uint32_t a0 = smem_u32(ds[0]);
-#pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk)
-          mma_ss_elect(tmem + col, desc_sw128(a0 + kk * 2048, kTileBytes, 1024),
-                 desc_sw128(k_s + kk * 2048, 8192, 1024), id_dq, (!first || kk > 0) ? 1u : 0u);
+        mma_ss_run<8, 128, 0, 128>(tmem + col, desc_sw128(smem_u32(ds[0]), kTileBytes, 1024),
+                                   desc_sw128(k_s, 8192, 1024), id_dq, first ? 0u : 1u);
       };
       bool ok = mbar_wait(&sm.kv_full, 0, abort, err, kDevTimeoutFull) &&
                 mbar_wait(&sm.qd_full[0], 0, abort, err, kDevTimeoutFull);
@@ -242,13 +239,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         if (!mbar_wait(&sm.sm_done, it & 1, abort, err, kDevTimeoutOther)) break;
         fence_after_sync();
-        {  // dV += P^T dO_i: 16-query group kk's P^T is in dP^T columns 32(kk/2) + 8(kk%2)
-          const uint32_t b0 = smem_u32(sm.dout[b]);
-#pragma unroll
-          for (int kk = 0; kk < BQ / 16; ++kk)
-            mma_ts_elect(tmem + kColDV, tmem + kColDP + 32 * (kk >> 1) + 8 * (kk & 1),
-                   desc_sw128(b0 + kk * 2048, 8192, 1024), id_mn, (it > 0 || kk > 0) ? 1u : 0u);
-        }
+        // dV += P^T dO_i: 16-query group kk's P^T is in dP^T columns 32(kk/2) + 8(kk%2)
+        mma_ts_run8<128, 8, 32, 40, 64, 72, 96, 104>(
+            tmem + kColDV, tmem + kColDP, desc_sw128(smem_u32(sm.dout[b]), 8192, 1024), id_mn,
+            it > 0 ? 1u : 0u);
         if (next) {
           issue_kk(kColDP, v_s, smem_u32(sm.dout[b ^ 1]));
           mma_commit_elect(&sm.dp_full);
@@ -315,27 +309,34 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 *reinterpret_cast<uint32_t(*)[16]>(dpv + 16));
       tmem_wait_ld();
       uint32_t wp[16], wh[16], wl[16];
+      const float4* l4 = reinterpret_cast<const float4*>(&sm.lse[b][qw]);
+      const float4* d4 = reinterpret_cast<const float4*>(&sm.delta[b][qw]);
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        float p2[2], ds2[2];
+      for (int e4 = 0; e4 < 8; ++e4) {
+        const float4 lv = l4[e4], dl = d4[e4];
+        const float la[4] = {lv.x, lv.y, lv.z, lv.w};
+        const float da[4] = {dl.x, dl.y, dl.z, dl.w};
+        float p[4], ds[4];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int q = qw + 2 * e + h;  // query within the block
-          float p = ex2(fmaf(__uint_as_float(sv[2 * e + h]), scale_log2, -sm.lse[b][q]));
-          float ds = p * (__uint_as_float(dpv[2 * e + h]) - sm.delta[b][q]);
+        for (int u = 0; u < 4; ++u) {
+          const int e = 4 * e4 + u;
+          p[u] = ex2(fmaf(__uint_as_float(sv[e]), scale_log2, -la[u]));
+          ds[u] = p[u] * (__uint_as_float(dpv[e]) - da[u]);
           if (need_mask) {
-            const int ig = i0 + q;
+            const int ig = i0 + qw + e;
             if (ig >= N || jg >= N || (causal && ig < jg)) {
-              p = 0.f;
-              ds = 0.f;
+              p[u] = 0.f;
+              ds[u] = 0.f;
             }
           }
-          p2[h] = p;
-          ds2[h] = ds;
         }
-        wp[e] = pack_bf16(p2[0], p2[1]);
-        wh[e] = pack_bf16(ds2[0], ds2[1]);
-        wl[e] = pack_bf16(ds2[0] - bf16lo(wh[e]), ds2[1] - bf16hi(wh[e]));
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int w2 = 2 * e4 + u;
+          wp[w2] = pack_bf16(p[2 * u], p[2 * u + 1]);
+          wh[w2] = pack_bf16(ds[2 * u], ds[2 * u + 1]);
+          wl[w2] = pack_bf16(ds[2 * u] - bf16lo(wh[w2]), ds[2 * u + 1] - bf16hi(wh[w2]));
+        }
       }
       // P^T of this warpgroup's 32 queries over its own (already loaded) dP^T columns
       tmem_st16(tmem + lane_off + kColDP + qw, wp);

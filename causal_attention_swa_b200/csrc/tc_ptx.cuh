@@ -72,6 +72,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// mbar_wait by lane 0 only (one shared-memory poll per warp instead of 32),
+// result broadcast; the warp barrier orders the other lanes after lane 0's
+// acquire.  All 32 lanes of the warp must call it.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort, unsigned* err,
+                                               unsigned code) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, err, code) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
+}
+
 // ----------------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
@@ -168,6 +181,91 @@ __device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, u
       "setp.ne.b32 p, %4, 0;\n\t"
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// A run of kN MMAs into one accumulator from one asm block (one elect.sync):
+// step k uses A descriptor a + a_step(k) and B descriptor b + b_step(k)
+// (descriptor start-address units, 16 bytes), where the step of A jumps by
+// a_jump after kN/2 steps (the second half tile of a K-major operand).
+// Accumulates from step 0 when `accumulate` is set, always from step 1 on.
+template <int kN, int kAStep, int kAJump, int kBStep>
+__device__ __forceinline__ void mma_ss_run(uint32_t d_tmem, uint64_t a, uint64_t b,
+                                           uint32_t idesc, uint32_t accumulate) {
+  static_assert(kN == 4 || kN == 8, "run length");
+#define SWA_STEP_A(k) ((k) * kAStep + ((k) >= kN / 2 ? kAJump : 0))
+  if constexpr (kN == 4) {
+    asm volatile(
+        "{\n\t.reg .pred e, p, t;\n\t.reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.b32 t, 0, 0;\n\t"
+        "add.s64 a1, %1, %5;\n\tadd.s64 a2, %1, %6;\n\tadd.s64 a3, %1, %7;\n\t"
+        "add.s64 b1, %2, %8;\n\tadd.s64 b2, %2, %9;\n\tadd.s64 b3, %2, %10;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, t;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "n"(SWA_STEP_A(1)), "n"(SWA_STEP_A(2)),
+        "n"(SWA_STEP_A(3)), "n"(1 * kBStep), "n"(2 * kBStep), "n"(3 * kBStep)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred e, p, t;\n\t.reg .b64 a1, a2, a3, a4, a5, a6, a7, b1, b2, b3, b4, b5, b6, b7;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.b32 t, 0, 0;\n\t"
+        "add.s64 a1, %1, %5;\n\tadd.s64 a2, %1, %6;\n\tadd.s64 a3, %1, %7;\n\t"
+        "add.s64 a4, %1, %8;\n\tadd.s64 a5, %1, %9;\n\tadd.s64 a6, %1, %10;\n\t"
+        "add.s64 a7, %1, %11;\n\t"
+        "add.s64 b1, %2, %12;\n\tadd.s64 b2, %2, %13;\n\tadd.s64 b3, %2, %14;\n\t"
+        "add.s64 b4, %2, %15;\n\tadd.s64 b5, %2, %16;\n\tadd.s64 b6, %2, %17;\n\t"
+        "add.s64 b7, %2, %18;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a4, b4, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a5, b5, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a6, b6, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a7, b7, %3, t;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "n"(SWA_STEP_A(1)), "n"(SWA_STEP_A(2)),
+        "n"(SWA_STEP_A(3)), "n"(SWA_STEP_A(4)), "n"(SWA_STEP_A(5)), "n"(SWA_STEP_A(6)),
+        "n"(SWA_STEP_A(7)), "n"(1 * kBStep), "n"(2 * kBStep), "n"(3 * kBStep),
+        "n"(4 * kBStep), "n"(5 * kBStep), "n"(6 * kBStep), "n"(7 * kBStep)
+        : "memory");
+  }
+#undef SWA_STEP_A
+}
+
+// Eight MMAs with A from TMEM: step k reads A at column a_tmem + kACol[k]
+// (constants given as template arguments), B descriptor b + k * kBStep.
+template <int kBStep, int c1, int c2, int c3, int c4, int c5, int c6, int c7>
+__device__ __forceinline__ void mma_ts_run8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, t;\n\t.reg .b32 a1, a2, a3, a4, a5, a6, a7;\n\t"
+      ".reg .b64 b1, b2, b3, b4, b5, b6, b7;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, 0, 0;\n\t"
+      "add.s32 a1, %1, %5;\n\tadd.s32 a2, %1, %6;\n\tadd.s32 a3, %1, %7;\n\t"
+      "add.s32 a4, %1, %8;\n\tadd.s32 a5, %1, %9;\n\tadd.s32 a6, %1, %10;\n\t"
+      "add.s32 a7, %1, %11;\n\t"
+      "add.s64 b1, %2, %12;\n\tadd.s64 b2, %2, %13;\n\tadd.s64 b3, %2, %14;\n\t"
+      "add.s64 b4, %2, %15;\n\tadd.s64 b5, %2, %16;\n\tadd.s64 b6, %2, %17;\n\t"
+      "add.s64 b7, %2, %18;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a4], b4, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a5], b5, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a6], b6, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a7], b7, %3, t;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate), "n"(c1), "n"(c2), "n"(c3), "n"(c4),
+      "n"(c5), "n"(c6), "n"(c7), "n"(1 * kBStep), "n"(2 * kBStep), "n"(3 * kBStep),
+      "n"(4 * kBStep), "n"(5 * kBStep), "n"(6 * kBStep), "n"(7 * kBStep)
       : "memory");
 }
 
