@@ -12,22 +12,36 @@
 // Block = two 128-row query tiles of one head (256 rows) and 384 threads:
 //   warps 0-3  softmax for query tile 0 (thread r owns row r = TMEM lane r)
 //   warps 4-7  softmax for query tile 1
-//   warp  8    TMA producer: Q0, Q1 once, then K_j, V_j into 3 stages
-//   warp  9    MMA issuer (one thread) and TMEM owner
-//   warps 10-11 idle
+//   warp  8    TMA producer: Q0, Q1 once, then K_j, V_j into 4 stages
+//   warp  9    MMA issuer for query tile 0 (one elected lane), TMEM owner
+//   warp  10   MMA issuer for query tile 1
+//   warp  11   idle
+// Each query tile has an issuer of its own, so neither tile's MMAs queue
+// behind the other tile's barriers; each issuer releases a K/V stage on a
+// barrier of its own and the producer waits for the issuers that read it.
 // Registers: launched at 168 per thread (384 x 168); the softmax
 // warpgroups take 224 (a full row of S stays in registers), the
 // producer/MMA warpgroup gives up to 56: 256 x 224 + 128 x 56 = 384 x 168.
-// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,320) O1 [320,384);
-// P_t (bf16, two per column) overwrites the first 64 columns of S_t and is
-// the A operand of O_t += P_t V_j straight from TMEM.
-// Per key tile j the MMA warp issues, for t = 0, 1:  O_t += P_t,j V_j, then
-// S_t,j+1 = Q_t K_j+1^T.  tcgen05 MMAs of one thread execute in issue
-// order, so S_t,j+1 may overwrite P_t,j, and the commit that announces
-// S_t,j+1 also covers O_t's update with P_t,j -- the softmax warps may then
-// rescale O_t in TMEM before publishing P_t,j+1.  The two query tiles
-// ping-pong: while one softmax warpgroup waits for its next S, the other
-// computes.
+// TMEM (512 columns): S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384)
+// O0 [384,448) O1 [448,512).  P_t (bf16, two per column) has columns of its
+// own and is the A operand of O_t += P_t V_j straight from TMEM.
+// The softmax warps copy S_t,j into registers and release its columns
+// (s_free) first, so the MMA warp computes S_t,j+1 while they exponentiate
+// S_t,j: the tensor work hides under the softmax instead of alternating
+// with it.  Per key tile j the MMA warp issues S_t,j+1 = Q_t K_j+1^T once
+// s_free[t] fires and O_t += P_t,j V_j once p_full[t] fires, then commits
+// pv_done[t]; the softmax warps wait on pv_done before they rescale O_t or
+// overwrite P_t, and store P_t only after computing all of it, by which
+// time O_t += P_t,j-1 V_j-1 has long finished.
+// Every wait parks the waiting warp (try_wait with a suspend hint), so idle
+// roles take no issue slots from the softmax warps that share a scheduler.
+// At D = 64 the exponentials bound the kernel: a score costs one MUFU ex2
+// (16 per clock per SM) and 4 * 64 MMA flops (about 8000 per clock per SM),
+// so ex2 time is about twice the MMA time.  Warps w and w + 4 share a
+// scheduler and its MUFU unit: the two warpgroups take
+// turns for their ex2 loops (exp_turn barriers), so that one warpgroup's
+// loads, row max and stores run under the other's exponentials instead of
+// both warpgroups contending for MUFU and then both idling.
 // Online softmax in the log2 domain with a lazy rescale: the reference max
 // of a row moves (and O, l are rescaled) only when the new row max exceeds
 // it by more than 8, so P <= 2^8 (exact after the final division by l).
@@ -51,14 +65,14 @@ using namespace tc;
 constexpr int BM = 128;                 // query rows per tile (MMA M)
 constexpr int BN = 128;                 // keys per K/V tile
 constexpr int HD = 64;                  // head dimension
-constexpr int kStages = 3;              // K/V pipeline depth
+constexpr int kStages = 4;              // K/V pipeline depth
 constexpr int kTileBytes = BM * HD * 2; // 16 KB per bf16 tile
 constexpr int kThreads = 384;
 constexpr int kSoftmaxRegs = 224;
 constexpr int kOtherRegs = 56;
 static_assert(256 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * 168, "register split");
 constexpr int kTmaWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kMmaWarp = 9;             // issuer of tile 0; kMmaWarp + 1 issues tile 1
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
 
@@ -69,11 +83,13 @@ struct __align__(1024) Smem {
   uint64_t q_full;
   uint64_t k_full[kStages];
   uint64_t v_full[kStages];
-  uint64_t kv_empty[kStages];
+  uint64_t kv_empty[2][kStages];  // per issuer
   uint64_t s_full[2];
+  uint64_t s_free[2];
   uint64_t p_full[2];
-  uint64_t o_final[2];
-  uint64_t drain;
+  uint64_t pv_done[2];
+  uint64_t exp_turn[2];  // exp_turn[t]: warpgroup t may start its ex2 loop
+  uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -81,7 +97,8 @@ struct __align__(1024) Smem {
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 
 __device__ __forceinline__ uint32_t col_s(int t) { return t ? 128u : 0u; }
-__device__ __forceinline__ uint32_t col_o(int t) { return t ? 320u : 256u; }
+__device__ __forceinline__ uint32_t col_p(int t) { return t ? 320u : 256u; }
+__device__ __forceinline__ uint32_t col_o(int t) { return t ? 448u : 384u; }
 
 __device__ __forceinline__ bool wait_unbounded_by_abort(uint64_t* bar, uint32_t parity) {
   const long long t0 = clock64();
@@ -124,14 +141,18 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.v_full[s], 1);
-      mbar_init(&sm.kv_empty[s], 1);
+      mbar_init(&sm.kv_empty[0][s], 1);
+      mbar_init(&sm.kv_empty[1][s], 1);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&sm.s_full[t], 1);
+      mbar_init(&sm.s_free[t], 128);
       mbar_init(&sm.p_full[t], 128);
-      mbar_init(&sm.o_final[t], 1);
+      mbar_init(&sm.pv_done[t], 1);
+      mbar_init(&sm.exp_turn[t], 128);
     }
-    mbar_init(&sm.drain, 1);
+    mbar_init(&sm.drain[0], 1);
+    mbar_init(&sm.drain[1], 1);
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -159,9 +180,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % kStages;
         const int round = j / kStages;
-        if (round > 0 && !mbar_wait(&sm.kv_empty[s], (round - 1) & 1, abort, err,
-                                    kDevTimeoutEmpty))
-          break;
+        // the stage held tile j - kStages: wait for each issuer that read it
+        bool ok = true;
+        for (int t = 0; t < 2 && ok && round > 0; ++t)
+          if (j - kStages < n_t[t])
+            ok = mbar_wait_parked(&sm.kv_empty[t][s], (round - 1) & 1, abort, err,
+                                  kDevTimeoutEmpty);
+        if (!ok) break;
         mbar_arrive_expect_tx(&sm.k_full[s], kTileBytes);
         tma_load_3d(sm.k[s], &tm_k, &sm.k_full[s], 0, j * BN, head);
         mbar_arrive_expect_tx(&sm.v_full[s], kTileBytes);
@@ -169,63 +194,56 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
     }
     __syncwarp();
-  } else if (warp == kMmaWarp) {
-    // --------------------------------------------------------- MMA issuer
+  } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
+    // ------------------------------------------------ MMA issuer of tile t
     {  // the whole warp runs the issue loop; one elected lane issues
+      const int t = warp - kMmaWarp;
       constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BN, 0, 0);  // Q, K both K-major
       constexpr uint32_t idesc_o = idesc_bf16_f32(BM, HD, 0, 1);  // V is MN-major (dims contiguous)
-      int k_ready = -1;
-      bool ok = mbar_wait(&sm.q_full, 0, abort, err, kDevTimeoutFull);
-      auto wait_k = [&](int j) -> bool {
-        if (j <= k_ready) return true;
-        if (!mbar_wait(&sm.k_full[j % kStages], (j / kStages) & 1, abort, err, kDevTimeoutFull))
-          return false;
-        k_ready = j;
-        return true;
-      };
-      auto issue_s = [&](int t, int j) {
-        const uint32_t a0 = smem_u32(sm.q[t]);
-        const uint32_t b0 = smem_u32(sm.k[j % kStages]);
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk)
-          mma_ss_elect(tmem + col_s(t), desc_sw128(a0 + kk * 32, 16, 1024),
-                 desc_sw128(b0 + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+      const uint64_t q_desc = desc_sw128(smem_u32(sm.q[t]), 16, 1024);
+      auto issue_s = [&](int j) {
+        // one asm block of 4 MMAs; K steps of 32 B = 2 descriptor units
+        mma_ss_run<4, 2, 0, 2>(tmem + col_s(t), q_desc,
+                               desc_sw128(smem_u32(sm.k[j % kStages]), 16, 1024), idesc_s, 0u);
         mma_commit_elect(&sm.s_full[t]);
       };
-      auto issue_pv = [&](int t, int j) {
-        const uint32_t b0 = smem_u32(sm.v[j % kStages]);
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts_elect(tmem + col_o(t), tmem + col_s(t) + kk * 8,
-                 desc_sw128(b0 + kk * 2048, 8192, 1024), idesc_o,
-                 (j > 0 || kk > 0) ? 1u : 0u);
+      auto issue_pv = [&](int j) {
+        // 8 MMAs: P columns 8k, V rows 16k (+2048 B = 128 units)
+        mma_ts_run8<128, 8, 16, 24, 32, 40, 48, 56>(
+            tmem + col_o(t), tmem + col_p(t), desc_sw128(smem_u32(sm.v[j % kStages]), 8192, 1024),
+            idesc_o, j > 0 ? 1u : 0u);
+        mma_commit_elect(&sm.pv_done[t]);
+        mma_commit_elect(&sm.kv_empty[t][j % kStages]);
       };
-      if (ok) ok = wait_k(0);
+      auto wait_k = [&](int j) {
+        return mbar_wait_parked(&sm.k_full[j % kStages], (j / kStages) & 1, abort, err,
+                                kDevTimeoutFull);
+      };
+      bool ok = n_t[t] > 0 && mbar_wait_parked(&sm.q_full, 0, abort, err, kDevTimeoutFull) &&
+                wait_k(0);
       if (ok) {
         fence_after_sync();
-        for (int t = 0; t < 2; ++t)
-          if (n_t[t] > 0) issue_s(t, 0);
+        issue_s(0);
       }
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int s = j % kStages;
-        if (!mbar_wait(&sm.v_full[s], (j / kStages) & 1, abort, err, kDevTimeoutFull)) break;
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (j >= n_t[t]) continue;
-          if (!mbar_wait(&sm.p_full[t], j & 1, abort, err, kDevTimeoutOther)) { ok = false; break; }
+      for (int j = 0; ok && j < n_t[t]; ++j) {
+        // S_t,j+1 as soon as the softmax warps hold S_t,j in registers
+        if (j + 1 < n_t[t]) {
+          if (!mbar_wait_parked(&sm.s_free[t], j & 1, abort, err, kDevTimeoutOther) ||
+              !wait_k(j + 1))
+            break;
           fence_after_sync();
-          issue_pv(t, j);
-          if (j + 1 < n_t[t]) {
-            if (!wait_k(j + 1)) { ok = false; break; }
-            issue_s(t, j + 1);
-          } else {
-            mma_commit_elect(&sm.o_final[t]);
-          }
+          issue_s(j + 1);
         }
-        mma_commit_elect(&sm.kv_empty[s]);
+        if (!mbar_wait_parked(&sm.v_full[j % kStages], (j / kStages) & 1, abort, err,
+                              kDevTimeoutFull) ||
+            !mbar_wait_parked(&sm.p_full[t], j & 1, abort, err, kDevTimeoutOther))
+          break;
+        fence_after_sync();
+        issue_pv(j);
       }
-      // every MMA this thread issued has finished before TMEM is released
-      mma_commit_elect(&sm.drain);
-      wait_unbounded_by_abort(&sm.drain, 0);
+      // every MMA this warp issued has finished before TMEM is released
+      mma_commit_elect(&sm.drain[t]);
+      wait_unbounded_by_abort(&sm.drain[t], 0);
     }
     __syncwarp();
   } else if (warp < 8) {
@@ -238,12 +256,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int row = g * BM + r;
     const uint32_t lane_off = static_cast<uint32_t>(wt * 32) << 16;
     const uint32_t tS = tmem + lane_off + col_s(t);
+    const uint32_t tP = tmem + lane_off + col_p(t);
     const uint32_t tO = tmem + lane_off + col_o(t);
     float m_used = -INFINITY;  // reference max (log2 domain)
     float l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_t[t]; ++j) {
-      if (!mbar_wait(&sm.s_full[t], j & 1, abort, err, kDevTimeoutMma)) { ok = false; break; }
+      if (!mbar_wait_parked(&sm.s_full[t], j & 1, abort, err, kDevTimeoutMma)) { ok = false; break; }
       fence_after_sync();
       float x[BN];
       {
@@ -254,8 +273,10 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
         for (int i = 0; i < BN / 16; ++i)
 #pragma unroll
-          for (int e = 0; e < 16; ++e) x[i * 16 + e] = __uint_as_float(u[i][e]) * scale_log2;
+          for (int e = 0; e < 16; ++e) x[i * 16 + e] = __uint_as_float(u[i][e]);
       }
+      fence_before_sync();
+      mbar_arrive(&sm.s_free[t]);  // S_t,j is in registers: its columns may take S_t,j+1
       const bool need_mask = (j * BN + BN > N) || (causal && j == g);
       if (need_mask) {
 #pragma unroll
@@ -264,16 +285,33 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (key >= N || (causal && key > row)) x[e] = -INFINITY;
         }
       }
+      // 8 chains of three-input maxima
       float mxp[8];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) mxp[a] = x[a];
+      for (int a = 0; a < 8; ++a) mxp[a] = fmax3(x[a], x[a + 8], x[a + 16]);
 #pragma unroll
-      for (int e = 8; e < BN; ++e) mxp[e & 7] = fmaxf(mxp[e & 7], x[e]);
-      const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                             fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+      for (int e = 24; e + 16 < BN; e += 16)
+#pragma unroll
+        for (int a = 0; a < 8; ++a) mxp[a] = fmax3(mxp[a], x[e + a], x[e + 8 + a]);
+#pragma unroll
+      for (int a = 0; a < 8; ++a) mxp[a] = fmaxf(mxp[a], x[BN - 8 + a]);
+      // raw scores: scaling by scale_log2 > 0 after the max commutes with it
+      const float mx = fmaxf(fmax3(mxp[0], mxp[1], mxp[2]),
+                             fmax3(fmax3(mxp[3], mxp[4], mxp[5]), mxp[6], mxp[7])) *
+                       scale_log2;
       const float m_new = fmaxf(m_used, mx);
       const bool need = (j == 0) || (m_new > m_used + kRescaleThreshold);
+      // O_t += P_t,j-1 V_j-1 must finish before O_t is rescaled or P_t is
+      // overwritten; the wait comes as late as it can (rare rescales first,
+      // else just before P_t,j is stored), so it is normally already over.
+      bool pv_seen = (j == 0);
       if (j > 0 && __any_sync(0xffffffffu, need)) {
+        if (!mbar_wait_parked(&sm.pv_done[t], (j - 1) & 1, abort, err, kDevTimeoutMma)) {
+          ok = false;
+          break;
+        }
+        fence_after_sync();
+        pv_seen = true;
         const float alpha = need ? ex2(m_used - m_new) : 1.f;
 #pragma unroll
         for (int i = 0; i < HD / 16; ++i) {
@@ -287,25 +325,44 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         l *= alpha;
       }
       if (need) m_used = m_new;
-      float rsp[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int i = 0; i < BN / 32; ++i) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2(x[i * 32 + 2 * e] - m_used);
-          const float p1 = ex2(x[i * 32 + 2 * e + 1] - m_used);
-          rsp[e & 3] += p0 + p1;
-          pk[e] = pack_bf16(p0, p1);
+      // MUFU turn: tile 0's ex2 loop for key tile j follows tile 1's for
+      // j - 1, and tile 1's for j follows tile 0's for j (when the other
+      // warpgroup has that key tile at all)
+      if (t == 0 ? (j >= 1 && j - 1 < n_t[1]) : (j < n_t[0])) {
+        if (!mbar_wait_parked(&sm.exp_turn[t], (t == 0 ? j - 1 : j) & 1, abort, err,
+                              kDevTimeoutOther)) {
+          ok = false;
+          break;
         }
-        tmem_st16(tS + i * 16, pk);
       }
+      float2 rsp[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      const float2 sc2 = make_float2(scale_log2, scale_log2);
+      const float2 nm2 = make_float2(-m_used, -m_used);
+      uint32_t pk[BN / 32][16];
+#pragma unroll
+      for (int e = 0; e < BN / 2; ++e) {
+        const float2 a = __ffma2_rn(make_float2(x[2 * e], x[2 * e + 1]), sc2, nm2);
+        const float2 pe = make_float2(ex2(a.x), ex2(a.y));
+        rsp[e & 1] = __fadd2_rn(rsp[e & 1], pe);
+        pk[e >> 4][e & 15] = pack_bf16(pe.x, pe.y);
+      }
+      mbar_arrive(&sm.exp_turn[t ^ 1]);
+      if (!pv_seen) {
+        if (!mbar_wait_parked(&sm.pv_done[t], (j - 1) & 1, abort, err, kDevTimeoutMma)) {
+          ok = false;
+          break;
+        }
+        fence_after_sync();
+      }
+#pragma unroll
+      for (int i = 0; i < BN / 32; ++i) tmem_st16(tP + i * 16, pk[i]);
       tmem_wait_st();
       fence_before_sync();
       mbar_arrive(&sm.p_full[t]);
-      l += (rsp[0] + rsp[1]) + (rsp[2] + rsp[3]);
+      l += (rsp[0].x + rsp[0].y) + (rsp[1].x + rsp[1].y);
     }
-    if (ok && n_t[t] > 0 && mbar_wait(&sm.o_final[t], 0, abort, err, kDevTimeoutMma)) {
+    if (ok && n_t[t] > 0 &&
+        mbar_wait_parked(&sm.pv_done[t], (n_t[t] - 1) & 1, abort, err, kDevTimeoutMma)) {
       fence_after_sync();
       const float inv = 1.f / l;
       uint32_t packed[HD / 2];

@@ -53,6 +53,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a waiting thread is parked (it issues
+// nothing) until the phase completes or about `ns` nanoseconds pass, so a
+// waiting warp leaves its scheduler's issue slots to the warps that compute.
+__device__ __forceinline__ bool mbar_try_wait_parked(uint64_t* bar, uint32_t parity,
+                                                     uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete.  Gives up (returns
 // false) when *abort becomes non-zero or after kWaitCycles; on a timeout it
 // records `code` in the device error word and raises *abort so that every
@@ -63,6 +79,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      atomicCAS(err, 0u, code);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+// mbar_wait that parks between polls (see mbar_try_wait_parked).
+__device__ __forceinline__ bool mbar_wait_parked(uint64_t* bar, uint32_t parity,
+                                                 volatile int* abort, unsigned* err,
+                                                 unsigned code) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait_parked(bar, parity, 20000u)) return true;
     if (*abort) return false;
     if (clock64() - t0 > kWaitCycles) {
       atomicCAS(err, 0u, code);
@@ -426,6 +459,13 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// max of three (sm_100 three-input form; NaN operands are ignored as by fmaxf)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
