@@ -9,19 +9,23 @@
 // (scores = q.k/8 over the pairs with q.t >= k.t, w = exp(s - row max),
 // out = sum w/z v).
 //
-// Block = two 128-row query tiles of one head (256 rows) and 384 threads:
-//   warps 0-3  softmax for query tile 0 (thread r owns row r = TMEM lane r)
-//   warps 4-7  softmax for query tile 1
-//   warp  8    TMA producer: Q0, Q1 once, then K_j, V_j into 4 stages
-//   warp  9    MMA issuer for query tile 0 (one elected lane), TMEM owner
-//   warp  10   MMA issuer for query tile 1
-//   warp  11   idle
+// Block = two 128-row query tiles of one head (256 rows) and 640 threads:
+//   warps 0-7   softmax for query tile 0, warps 8-15 for query tile 1; in
+//               each group, warps 4h + w (w = 0..3) take TMEM lanes
+//               32w..32w+31 (rows) and score columns 64h..64h+63, so a row
+//               is shared by two threads that agree on its max each tile
+//   warp  16    TMA producer: Q0, Q1 once, then K_j, V_j into 4 stages
+//   warp  17    MMA issuer for query tile 0 (one elected lane), TMEM owner
+//   warp  18    MMA issuer for query tile 1
+//   warp  19    idle (gives its registers to the softmax warps of its scheduler)
 // Each query tile has an issuer of its own, so neither tile's MMAs queue
 // behind the other tile's barriers; each issuer releases a K/V stage on a
 // barrier of its own and the producer waits for the issuers that read it.
-// Registers: launched at 168 per thread (384 x 168); the softmax
-// warpgroups take 224 (a full row of S stays in registers), the
-// producer/MMA warpgroup gives up to 56: 256 x 224 + 128 x 56 = 384 x 168.
+// Registers: launched at 96 per thread (640 x 96); the softmax warps take
+// 104 and warps 16-19 give up to 40, one of them on each scheduler (the
+// registers of a warp stay in its scheduler's file).  The launcher checks
+// that the kernel was built with exactly 96: a larger claim than the
+// scheduler holds would stall setmaxnreg.inc.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384)
 // O0 [384,448) O1 [448,512).  P_t (bf16, two per column) has columns of its
 // own and is the A operand of O_t += P_t V_j straight from TMEM.
@@ -37,11 +41,9 @@
 // roles take no issue slots from the softmax warps that share a scheduler.
 // At D = 64 the exponentials bound the kernel: a score costs one MUFU ex2
 // (16 per clock per SM) and 4 * 64 MMA flops (about 8000 per clock per SM),
-// so ex2 time is about twice the MMA time.  Warps w and w + 4 share a
-// scheduler and its MUFU unit: the two warpgroups take
-// turns for their ex2 loops (exp_turn barriers), so that one warpgroup's
-// loads, row max and stores run under the other's exponentials instead of
-// both warpgroups contending for MUFU and then both idling.
+// so ex2 time is about twice the MMA time.  A single warp cannot keep its
+// scheduler's MUFU busy (the FMA -> ex2 -> convert chains are too short),
+// so every scheduler runs four softmax warps.
 // Online softmax in the log2 domain with a lazy rescale: the reference max
 // of a row moves (and O, l are rescaled) only when the new row max exceeds
 // it by more than 8, so P <= 2^8 (exact after the final division by l).
@@ -67,14 +69,23 @@ constexpr int BN = 128;                 // keys per K/V tile
 constexpr int HD = 64;                  // head dimension
 constexpr int kStages = 4;              // K/V pipeline depth
 constexpr int kTileBytes = BM * HD * 2; // 16 KB per bf16 tile
-constexpr int kThreads = 384;
-constexpr int kSoftmaxRegs = 224;
-constexpr int kOtherRegs = 56;
-static_assert(256 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * 168, "register split");
-constexpr int kTmaWarp = 8;
-constexpr int kMmaWarp = 9;             // issuer of tile 0; kMmaWarp + 1 issues tile 1
+constexpr int kSoftmaxWarps = 16;
+constexpr int kThreads = (kSoftmaxWarps + 4) * 32;  // 640: five warps per scheduler
+// 16384 registers per scheduler / (5 warps * 32 threads), rounded down to 8
+constexpr int kLaunchRegs = 96;
+constexpr int kSoftmaxRegs = 104;
+constexpr int kOtherRegs = 40;
+// Warp w runs on scheduler w % 4 and setmaxnreg moves registers only
+// between the warps of one scheduler: each scheduler holds four softmax
+// warps and one of warps 16-19, which gives up what the four take.
+static_assert(4 * kSoftmaxRegs + kOtherRegs <= 5 * kLaunchRegs, "register split per scheduler");
+constexpr int kTmaWarp = kSoftmaxWarps;
+constexpr int kMmaWarp = kSoftmaxWarps + 1;  // issuer of tile 0; kMmaWarp + 1 issues tile 1
+constexpr int kHalf = BN / 2;                // score columns per softmax thread
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
+constexpr float kFastRange = 64.0f;  // P < 2^64 against a stale max still fits
+
 
 struct __align__(1024) Smem {
   uint8_t q[2][kTileBytes];
@@ -88,7 +99,8 @@ struct __align__(1024) Smem {
   uint64_t s_free[2];
   uint64_t p_full[2];
   uint64_t pv_done[2];
-  uint64_t exp_turn[2];  // exp_turn[t]: warpgroup t may start its ex2 loop
+  uint64_t pair[2][4];          // the two threads of a row: tile t, lanes 32w..
+  float part[2][2][2][BM];      // [tile][parity][half][row]: partial row max / sum
   uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
@@ -146,10 +158,10 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&sm.s_full[t], 1);
-      mbar_init(&sm.s_free[t], 128);
-      mbar_init(&sm.p_full[t], 128);
+      mbar_init(&sm.s_free[t], 256);
+      mbar_init(&sm.p_full[t], 256);
       mbar_init(&sm.pv_done[t], 1);
-      mbar_init(&sm.exp_turn[t], 128);
+      for (int w = 0; w < 4; ++w) mbar_init(&sm.pair[t][w], 64);
     }
     mbar_init(&sm.drain[0], 1);
     mbar_init(&sm.drain[1], 1);
@@ -166,7 +178,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
 
-  if (warp >= 8) regs_decrease<kOtherRegs>();
+  if (warp >= kSoftmaxWarps) regs_decrease<kOtherRegs>();
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ producer
@@ -246,32 +258,46 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       wait_unbounded_by_abort(&sm.drain[t], 0);
     }
     __syncwarp();
-  } else if (warp < 8) {
+  } else if (warp < kSoftmaxWarps) {
     // ------------------------------------------------------------ softmax
     regs_increase<kSoftmaxRegs>();
-    const int t = warp >> 2;
-    const int wt = warp & 3;
+    const int t = warp >> 3;        // query tile
+    const int h = (warp >> 2) & 1;  // score columns 64h..64h+63
+    const int wt = warp & 3;        // TMEM lanes 32wt..32wt+31
     const int r = wt * 32 + lane;
     const int g = 2 * c + t;
     const int row = g * BM + r;
     const uint32_t lane_off = static_cast<uint32_t>(wt * 32) << 16;
-    const uint32_t tS = tmem + lane_off + col_s(t);
-    const uint32_t tP = tmem + lane_off + col_p(t);
-    const uint32_t tO = tmem + lane_off + col_o(t);
-    float m_used = -INFINITY;  // reference max (log2 domain)
-    float l = 0.f;
+    const uint32_t tS = tmem + lane_off + col_s(t) + kHalf * h;
+    const uint32_t tP = tmem + lane_off + col_p(t) + (kHalf / 2) * h;
+    const uint32_t tO = tmem + lane_off + col_o(t) + (HD / 2) * h;
+    uint64_t* pair = &sm.pair[t][wt];
+    int pair_phase = 0;
+    // publish v for the row, wait for the partner thread's value
+    auto exchange = [&](float v, float& other) -> bool {
+      const int slot = pair_phase & 1;
+      sm.part[t][slot][h][r] = v;
+      mbar_arrive(pair);
+      if (!mbar_wait_parked(pair, pair_phase & 1, abort, err, kDevTimeoutOther)) return false;
+      other = sm.part[t][slot][h ^ 1][r];
+      ++pair_phase;
+      return true;
+    };
+    float m_used = -INFINITY;  // reference max (log2 domain), the same in both
+                               // threads of the row
+    float l = 0.f;             // this thread's share of the row sum
     bool ok = true;
     for (int j = 0; j < n_t[t]; ++j) {
       if (!mbar_wait_parked(&sm.s_full[t], j & 1, abort, err, kDevTimeoutMma)) { ok = false; break; }
       fence_after_sync();
-      float x[BN];
+      float x[kHalf];
       {
-        uint32_t u[BN / 16][16];
+        uint32_t u[kHalf / 16][16];
 #pragma unroll
-        for (int i = 0; i < BN / 16; ++i) tmem_ld16(tS + i * 16, u[i]);
+        for (int i = 0; i < kHalf / 16; ++i) tmem_ld16(tS + i * 16, u[i]);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < BN / 16; ++i)
+        for (int i = 0; i < kHalf / 16; ++i)
 #pragma unroll
           for (int e = 0; e < 16; ++e) x[i * 16 + e] = __uint_as_float(u[i][e]);
       }
@@ -280,94 +306,108 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       const bool need_mask = (j * BN + BN > N) || (causal && j == g);
       if (need_mask) {
 #pragma unroll
-        for (int e = 0; e < BN; ++e) {
-          const int key = j * BN + e;
+        for (int e = 0; e < kHalf; ++e) {
+          const int key = j * BN + kHalf * h + e;
           if (key >= N || (causal && key > row)) x[e] = -INFINITY;
         }
       }
-      // 8 chains of three-input maxima
+      // 8 chains of three-input maxima over this thread's 64 scores
       float mxp[8];
 #pragma unroll
       for (int a = 0; a < 8; ++a) mxp[a] = fmax3(x[a], x[a + 8], x[a + 16]);
 #pragma unroll
-      for (int e = 24; e + 16 < BN; e += 16)
+      for (int a = 0; a < 8; ++a) mxp[a] = fmax3(mxp[a], x[a + 24], x[a + 32]);
 #pragma unroll
-        for (int a = 0; a < 8; ++a) mxp[a] = fmax3(mxp[a], x[e + a], x[e + 8 + a]);
+      for (int a = 0; a < 8; ++a) mxp[a] = fmax3(mxp[a], x[a + 40], x[a + 48]);
 #pragma unroll
-      for (int a = 0; a < 8; ++a) mxp[a] = fmaxf(mxp[a], x[BN - 8 + a]);
-      // raw scores: scaling by scale_log2 > 0 after the max commutes with it
-      const float mx = fmaxf(fmax3(mxp[0], mxp[1], mxp[2]),
-                             fmax3(fmax3(mxp[3], mxp[4], mxp[5]), mxp[6], mxp[7])) *
-                       scale_log2;
-      const float m_new = fmaxf(m_used, mx);
-      const bool need = (j == 0) || (m_new > m_used + kRescaleThreshold);
-      // O_t += P_t,j-1 V_j-1 must finish before O_t is rescaled or P_t is
-      // overwritten; the wait comes as late as it can (rare rescales first,
-      // else just before P_t,j is stored), so it is normally already over.
-      bool pv_seen = (j == 0);
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        if (!mbar_wait_parked(&sm.pv_done[t], (j - 1) & 1, abort, err, kDevTimeoutMma)) {
-          ok = false;
-          break;
-        }
-        fence_after_sync();
-        pv_seen = true;
-        const float alpha = need ? ex2(m_used - m_new) : 1.f;
-#pragma unroll
-        for (int i = 0; i < HD / 16; ++i) {
-          uint32_t u[16];
-          tmem_ld16(tO + i * 16, u);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
-          tmem_st16(tO + i * 16, u);
-        }
-        l *= alpha;
-      }
-      if (need) m_used = m_new;
-      // MUFU turn: tile 0's ex2 loop for key tile j follows tile 1's for
-      // j - 1, and tile 1's for j follows tile 0's for j (when the other
-      // warpgroup has that key tile at all)
-      if (t == 0 ? (j >= 1 && j - 1 < n_t[1]) : (j < n_t[0])) {
-        if (!mbar_wait_parked(&sm.exp_turn[t], (t == 0 ? j - 1 : j) & 1, abort, err,
-                              kDevTimeoutOther)) {
-          ok = false;
-          break;
-        }
-      }
+      for (int a = 0; a < 8; ++a) mxp[a] = fmaxf(mxp[a], x[a + 56]);
+      const float mine = fmaxf(fmax3(mxp[0], mxp[1], mxp[2]),
+                               fmax3(fmax3(mxp[3], mxp[4], mxp[5]), mxp[6], mxp[7]));
+      // Publish this thread's max now, read the partner's when it is needed:
+      // before the ex2 loop only if a score of this thread could lie far
+      // above m_used (the first tile, a jump of more than kFastRange, a
+      // NaN); else after it, when the partner has long published.  Both
+      // threads derive the same m_new from (m_used, both maxima); a P
+      // computed against m_used is then moved to m_new (rare: the partner
+      // raised the max by more than the lazy threshold) by one rounding.
+      const float mine_l2 = mine * scale_log2;  // scale_log2 > 0 commutes with the max
+      const int slot = pair_phase & 1;
+      const uint32_t par = static_cast<uint32_t>(pair_phase & 1);
+      ++pair_phase;
+      sm.part[t][slot][h][r] = mine_l2;
+      mbar_arrive(pair);
+      float m_new = m_used;
+      auto fetch_and_decide = [&]() -> bool {
+        if (!mbar_wait_parked(pair, par, abort, err, kDevTimeoutOther)) return false;
+        const float theirs = sm.part[t][slot][h ^ 1][r];
+        // the same operand order in both threads of the row
+        const float cand = h == 0 ? fmaxf(mine_l2, theirs) : fmaxf(theirs, mine_l2);
+        const float mc = fmaxf(m_used, cand);
+        if (j == 0 || mc > m_used + kRescaleThreshold) m_new = mc;
+        return true;
+      };
+      const bool early = __any_sync(0xffffffffu, j == 0 || !(mine_l2 <= m_used + kFastRange));
+      if (early && !fetch_and_decide()) { ok = false; break; }
+      const float m_exp = m_new;  // the reference the ex2 loop uses
       float2 rsp[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       const float2 sc2 = make_float2(scale_log2, scale_log2);
-      const float2 nm2 = make_float2(-m_used, -m_used);
-      uint32_t pk[BN / 32][16];
+      const float2 nm2 = make_float2(-m_exp, -m_exp);
+      uint32_t pk[kHalf / 32][16];
 #pragma unroll
-      for (int e = 0; e < BN / 2; ++e) {
+      for (int e = 0; e < kHalf / 2; ++e) {
         const float2 a = __ffma2_rn(make_float2(x[2 * e], x[2 * e + 1]), sc2, nm2);
         const float2 pe = make_float2(ex2(a.x), ex2(a.y));
         rsp[e & 1] = __fadd2_rn(rsp[e & 1], pe);
         pk[e >> 4][e & 15] = pack_bf16(pe.x, pe.y);
       }
-      mbar_arrive(&sm.exp_turn[t ^ 1]);
-      if (!pv_seen) {
+      if (!early && !fetch_and_decide()) { ok = false; break; }
+      if (__any_sync(0xffffffffu, m_exp != m_new)) {  // rare: the partner moved the max
+        const float beta = ex2(m_exp - m_new);
+#pragma unroll
+        for (int i = 0; i < kHalf / 32; ++i)
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[i][e] = pack_bf16(bf16lo(pk[i][e]) * beta, bf16hi(pk[i][e]) * beta);
+        rsp[0].x *= beta; rsp[0].y *= beta; rsp[1].x *= beta; rsp[1].y *= beta;
+      }
+      // O_t += P_t,j-1 V_j-1 must finish before O_t is rescaled or P_t is
+      // overwritten: by now it normally has.
+      if (j > 0) {
         if (!mbar_wait_parked(&sm.pv_done[t], (j - 1) & 1, abort, err, kDevTimeoutMma)) {
           ok = false;
           break;
         }
         fence_after_sync();
-      }
+        if (__any_sync(0xffffffffu, m_new != m_used)) {
+          const float alpha = ex2(m_used - m_new);
 #pragma unroll
-      for (int i = 0; i < BN / 32; ++i) tmem_st16(tP + i * 16, pk[i]);
+          for (int i = 0; i < HD / 32; ++i) {
+            uint32_t u[16];
+            tmem_ld16(tO + i * 16, u);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
+            tmem_st16(tO + i * 16, u);
+          }
+          l *= alpha;
+        }
+      }
+      m_used = m_new;
+#pragma unroll
+      for (int i = 0; i < kHalf / 32; ++i) tmem_st16(tP + i * 16, pk[i]);
       tmem_wait_st();
       fence_before_sync();
       mbar_arrive(&sm.p_full[t]);
       l += (rsp[0].x + rsp[0].y) + (rsp[1].x + rsp[1].y);
     }
-    if (ok && n_t[t] > 0 &&
+    float l_other = 0.f;
+    if (ok && n_t[t] > 0 && exchange(l, l_other) &&
         mbar_wait_parked(&sm.pv_done[t], (n_t[t] - 1) & 1, abort, err, kDevTimeoutMma)) {
       fence_after_sync();
-      const float inv = 1.f / l;
-      uint32_t packed[HD / 2];
+      const float inv = 1.f / (h == 0 ? l + l_other : l_other + l);
+      uint32_t packed[HD / 4];
 #pragma unroll
-      for (int i = 0; i < HD / 16; ++i) {
+      for (int i = 0; i < HD / 32; ++i) {
         uint32_t u[16];
         tmem_ld16(tO + i * 16, u);
         tmem_wait_ld();
@@ -377,12 +417,12 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                         __uint_as_float(u[2 * e + 1]) * inv);
       }
       if (row < N) {
-        uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)head * N + row) * HD);
+        uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)head * N + row) * HD + (HD / 2) * h);
 #pragma unroll
-        for (int i = 0; i < HD / 8; ++i)
+        for (int i = 0; i < HD / 16; ++i)
           dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2],
                               packed[4 * i + 3]);
-        lse[(size_t)head * N + row] = (m_used + __log2f(l)) * kLn2;
+        if (h == 0) lse[(size_t)head * N + row] = (m_used + __log2f(l + l_other)) * kLn2;
       }
     }
   }
@@ -441,6 +481,10 @@ cudaError_t launch_attn_fwd_tc(const void* q, const void* k, const void* v, void
   e = cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)kSmemBytes);
   if (e != cudaSuccess) return e;
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, attn_fwd_tc_kernel);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;  // register split unsafe
   const int n_ctiles = (int)((N + 2 * BM - 1) / (2 * BM));
   const int64_t grid = (int64_t)n_ctiles * BH;
   attn_fwd_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(
