@@ -10,44 +10,44 @@
 //   dv_j += P_ij dout_i   dk_j += scale dS_ij q_i   dq_i += scale dS_ij k_j
 // over the pairs that exist (j <= i when causal).
 //
-// Block = one 128-key block j of one head (K_j, V_j stay in shared memory)
-// and 576 threads; it walks the 128-query blocks i that see j:
-//   warps 0-15  compute, four warpgroups: thread t of warpgroup w owns key
-//               j0 + t (TMEM lane t) and queries 32w..32w+31 of each block.
-//               From S^T and dP^T (one batched TMEM load per block) it forms
-//               P^T (bf16, written back over its own dP^T columns for the
-//               dV MMA) and dS (float32 -> bf16 hi + lo, into shared
-//               memory); then it drains columns 16w..16w+15 of the previous
-//               block's dQ (TMEM lane = query) into the float32 dQ
-//               accumulator with vector red.add; at the end warpgroup w
-//               stores columns 16w..16w+15 of its key's dv and dk
-//   warp  16    TMA producer: K_j, V_j once; Q_i, dO_i, lse_i, delta_i into a
-//               2-stage ring
-//   warp  17    MMA issuer (one thread), TMEM owner
-// Per query block, seven MMAs (M = 128, K = 64 or 128):
-//   S^T = K_j Q_i^T              (A = K smem K-major, B = Q smem K-major)
-//   dP^T = V_j dO_i^T            (A = V, B = dO, both K-major)
-//   dV += P^T dO_i               (A = P^T from TMEM, B = dO MN-major)
-//   dK += dS_hi^T Q_i + dS_lo^T Q_i   (A = dS tiles read K-major, B = Q MN-major)
-//   dQ_i = dS_hi K_j + dS_lo K_j      (A = the same tiles read MN-major, B = K)
-// dS is carried as hi + lo bf16 pairs (hi = bf16(dS), lo = bf16(dS - hi)),
-// so dk and dq see dS to ~16 bits: a single bf16 rounding of dS, amplified
-// by the cancellation in sum_j dS_ij k_j (sum_j dS_ij = 0), costs dq about
-// 2% of its row RMS at N = 2048.  One [128 keys][128 queries] tile layout
-// (rows = keys, 128-byte swizzle, two 64-query halves) is both the K-major
-// A operand of dK and the MN-major A operand of dQ; it is double-buffered
-// by query block, so block i's dS is written while block i-1's dK and dQ
-// MMAs still read the other buffer.
-// TMEM (512 columns): S^T buffers [0,128) and [128,256) (the block's dQ in
-// the first 64 columns once S^T is consumed), dP^T [256,384) (warpgroup w
-// writes the P^T of its 32 queries over its own columns 32w..32w+15 after
-// loading them; the dV MMA takes each 16-query group's A from there),
-// dV [384,448), dK [448,512).  MMAs of one thread execute in issue order,
-// so a later MMA may overwrite TMEM an earlier one reads.
-// Causal: only query blocks i >= j are visited; in the diagonal block (and
-// past N on a ragged tail) P and dS of a masked pair are set to 0 by select.
-// This kernel takes only heads whose V and dout are all finite, so 0 times
-// a finite value is the same as skipping the pair.
+// Two kernels, neither with atomics:
+//   attn_bwd_dkdv_kernel  block = one 128-key block j; it walks the query
+//                         blocks i that see j and keeps dV_j, dK_j in TMEM
+//   attn_bwd_dq_kernel    block = one 128-query block i; it walks the key
+//                         blocks j that i sees and keeps dQ_i in TMEM
+// Each recomputes S and dP for its pairs (two of the products are done
+// twice), in exchange for no float32 dQ accumulator in memory, no reduce
+// traffic and no conversion pass.
+//
+// Both kernels: 576 threads = warps 0-15 compute (four warpgroups), warp 16
+// TMA producer, warp 17 MMA issuer (one elected lane) and TMEM owner.  The
+// compute warps copy S and dP of a block into registers and release dP's
+// TMEM columns at once (dp_free), so the MMA warp computes the next block's
+// dP (and S, double-buffered) while they form P and dS: the tensor pipe
+// works under the exponentials instead of waiting for them.
+//
+// dkdv: thread t of warpgroup w owns key j0 + t (TMEM lane t) and queries
+// 32w..32w+31 of a block.  Per query block four products (M = 128):
+//   S^T = K_j Q_i^T      (A = K smem K-major, B = Q smem K-major)
+//   dP^T = V_j dO_i^T    (A = V, B = dO, both K-major)
+//   dV += P^T dO_i       (A = P^T from TMEM, B = dO MN-major)
+//   dK += dS^T Q_i       (A = dS^T tile from smem, K-major; B = Q MN-major)
+// P^T (bf16) goes back over the warpgroup's own S^T columns 32w..32w+15
+// once loaded; dS^T (bf16) into a double-buffered [128 keys][128 queries]
+// tile (two 64-query halves, 128-byte swizzle).
+// dq: thread t of warpgroup w owns query i0 + t (TMEM lane t) and keys
+// 32w..32w+31 of a block.  Per key block:
+//   S = Q_i K_j^T, dP = dO_i V_j^T   (all K-major)
+//   dQ += dS_hi K_j + dS_lo K_j      (A = dS tiles K-major, B = K MN-major)
+// dS is carried as hi + lo bf16 (hi = bf16(dS), lo = bf16(dS - hi)) for dq:
+// sum_j dS_ij = 0, and a single bf16 rounding of dS, amplified by that
+// cancellation in sum_j dS_ij k_j, costs dq about 2% of its row RMS at
+// N = 2048.  dk has no such cancellation (its sum runs over queries), so
+// dS^T enters dK at bf16.
+// Causal: a key block meets only the query blocks i >= j; inside a diagonal
+// block (and past N on a ragged tail) P and dS of a masked pair are set to
+// 0 by select.  These kernels take only heads whose V and dout are all
+// finite, so 0 times a finite value is the same as skipping the pair.
 // Every mbarrier wait is bounded (device error word on expiry).
 #include "attn_tc.cuh"
 #include "tc_ptx.cuh"
@@ -65,39 +65,12 @@ constexpr int kComputeThreads = 512;    // four warpgroups
 constexpr int kTmaWarp = 16;
 constexpr int kMmaWarp = 17;
 constexpr int kThreads = 576;
+constexpr int kStages = 3;              // streamed operand ring depth
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColDP = 256, kColDV = 384, kColDK = 448;
-constexpr int kHeadGroup = 4;      // heads scheduled together (their dQ, Q, dO share L2)
+constexpr uint32_t kColDP = 256;
+constexpr int kHeadGroup = 4;           // heads scheduled together (their operands share L2)
 
 __device__ __forceinline__ uint32_t col_s(int b) { return b ? 128u : 0u; }
-
-// Shared memory (227 KB of the 227 KB a block may use): the dynamic base is
-// expected 1024-byte aligned (the kernel checks and reports otherwise).
-struct __align__(1024) Smem {
-  uint8_t k[kTileBytes];
-  uint8_t v[kTileBytes];
-  uint8_t q[2][kTileBytes];
-  uint8_t dout[2][kTileBytes];
-  uint8_t ds_hi[2][2][kTileBytes];  // [buffer][query half]: [128 keys][64 queries]
-  uint8_t ds_lo[2][2][kTileBytes];
-  float lse[2][BQ];                 // lse_i * log2(e) of each staged query block (+inf past N)
-  float delta[2][BQ];               // delta_i of each staged query block (0 past N)
-  uint64_t kv_full;
-  uint64_t qd_full[2];
-  uint64_t qd_empty[2];
-  uint64_t s_full[2];
-  uint64_t dp_full;
-  uint64_t sm_done;
-  uint64_t dq_full;
-  uint64_t dq_empty;
-  uint64_t acc_full;
-  uint64_t drain;
-  uint32_t tmem_base;
-  int abort;
-};
-
-constexpr size_t kSmemBytes = sizeof(Smem);
-static_assert(kSmemBytes <= 232448, "shared memory");
 
 __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
   const long long t0 = clock64();
@@ -107,24 +80,74 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
-                   const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v,
-                   const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ lse2,
-                   const float* __restrict__ delta, __nv_bfloat16* __restrict__ dk,
-                   __nv_bfloat16* __restrict__ dv, float* __restrict__ dqacc, int N, int BH,
-                   int causal, float scale, float scale_log2, const int* __restrict__ flags,
-                   unsigned* __restrict__ err) {
-  // Block order: groups of kHeadGroup heads; inside a group the longest key
-  // blocks (j = 0 sees every query block) first, heads interleaved.
-  const int n_blocks = (N + BQ - 1) / BQ;
-  const int Npad = n_blocks * BQ;
+// Block -> (head, block index) in groups of kHeadGroup heads; inside a
+// group the heaviest blocks first, heads interleaved.  heavy_low: block
+// index 0 is the heaviest (dkdv: key block 0 meets every query block);
+// else the last one is (dq: the last query block sees every key block).
+__device__ __forceinline__ void block_order(int n_blocks, int BH, bool heavy_low, int* head,
+                                            int* blk) {
   const int group = blockIdx.x / (kHeadGroup * n_blocks);
   const int g_heads = min(kHeadGroup, BH - group * kHeadGroup);
   const int r = blockIdx.x - group * kHeadGroup * n_blocks;
-  const int jb = r / g_heads;
-  const int head = group * kHeadGroup + r % g_heads;
+  const int rank = r / g_heads;
+  *head = group * kHeadGroup + r % g_heads;
+  *blk = heavy_low ? rank : n_blocks - 1 - rank;
+}
+
+// Stores 32 bf16 values of one row (w[0..15], columns col0..col0+31) into a
+// [128 rows][128 columns] bf16 tile kept as two 64-column halves [128][64]
+// with the 128-byte swizzle: 16-byte chunk c of a half-tile row sits at
+// chunk c ^ (row & 7).
+__device__ __forceinline__ void store_tile_row32(const uint8_t (*tile)[kTileBytes], int row,
+                                                 int col0, const uint32_t (&w)[16]) {
+  const uint32_t base = smem_u32(tile[col0 >> 6]) + row * 128;
+  const uint32_t chunk0 = static_cast<uint32_t>((col0 & 63) >> 3);
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const uint32_t off = ((chunk0 + g) ^ static_cast<uint32_t>(row & 7)) << 4;
+    st_shared_v4(base + off, w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
+  }
+}
+
+// =================================================================== dK, dV
+
+struct __align__(1024) SmemKV {
+  uint8_t k[kTileBytes];
+  uint8_t v[kTileBytes];
+  uint8_t q[kStages][kTileBytes];
+  uint8_t dout[kStages][kTileBytes];
+  uint8_t ds[2][2][kTileBytes];  // [buffer][query half]: dS^T [128 keys][64 queries]
+  float nlse[kStages][BQ];       // -lse_i * log2(e) of each staged query block (-inf past N)
+  float delta[kStages][BQ];      // delta_i (0 past N)
+  uint64_t kv_full;
+  uint64_t qd_full[kStages];
+  uint64_t qd_empty[kStages];
+  uint64_t s_full[2];
+  uint64_t dp_full;
+  uint64_t dp_free;
+  uint64_t sm_done;
+  uint64_t ds_free[2];
+  uint64_t acc_full;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr size_t kSmemKV = sizeof(SmemKV);
+static_assert(kSmemKV <= 232448, "shared memory");
+constexpr uint32_t kColDV = 384, kColDK = 448;
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
+                     const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ nlse2,
+                     const float* __restrict__ delta, __nv_bfloat16* __restrict__ dk,
+                     __nv_bfloat16* __restrict__ dv, int N, int BH, int causal, float scale,
+                     float scale_log2, const int* __restrict__ flags, unsigned* __restrict__ err) {
+  const int n_blocks = (N + BQ - 1) / BQ;
+  const int Npad = n_blocks * BQ;
+  int head, jb;
+  block_order(n_blocks, BH, true, &head, &jb);
   if (flags[head] != 0) return;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -132,7 +155,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (threadIdx.x == 0) atomicCAS(err, 0u, (unsigned)kDevSmemAlign);
     return;
   }
-  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  SmemKV& sm = *reinterpret_cast<SmemKV*>(smem_raw);
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
@@ -142,15 +165,17 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   if (tid == 0) {
     mbar_init(&sm.kv_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.qd_full[s], 1);
       mbar_init(&sm.qd_empty[s], 1);
-      mbar_init(&sm.s_full[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.ds_free[b], 1);
     }
     mbar_init(&sm.dp_full, 1);
+    mbar_init(&sm.dp_free, kComputeThreads);
     mbar_init(&sm.sm_done, kComputeThreads);
-    mbar_init(&sm.dq_full, 1);
-    mbar_init(&sm.dq_empty, kComputeThreads);
     mbar_init(&sm.acc_full, 1);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
@@ -177,16 +202,16 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       tma_load_3d(sm.k, &tm_k, &sm.kv_full, 0, j0, head);
       tma_load_3d(sm.v, &tm_v, &sm.kv_full, 0, j0, head);
       for (int it = 0; it < n_q; ++it) {
-        const int s = it & 1;
-        const int round = it >> 1;
-        if (round > 0 &&
-            !mbar_wait(&sm.qd_empty[s], (round - 1) & 1, abort, err, kDevTimeoutEmpty))
+        const int s = it % kStages;
+        const int round = it / kStages;
+        if (round > 0 && !mbar_wait_parked(&sm.qd_empty[s], (round - 1) & 1, abort, err,
+                                           kDevTimeoutEmpty))
           break;
         const int i0 = (ib0 + it) * BQ;
         mbar_arrive_expect_tx(&sm.qd_full[s], 2 * kTileBytes + 2 * BQ * 4);
         tma_load_3d(sm.q[s], &tm_q, &sm.qd_full[s], 0, i0, head);
         tma_load_3d(sm.dout[s], &tm_do, &sm.qd_full[s], 0, i0, head);
-        bulk_load(sm.lse[s], lse2 + (size_t)head * Npad + i0, BQ * 4, &sm.qd_full[s]);
+        bulk_load(sm.nlse[s], nlse2 + (size_t)head * Npad + i0, BQ * 4, &sm.qd_full[s]);
         bulk_load(sm.delta[s], delta + (size_t)head * Npad + i0, BQ * 4, &sm.qd_full[s]);
       }
     }
@@ -196,31 +221,21 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     {  // the whole warp runs the issue loop; one elected lane issues
       constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T: both K-major
       constexpr uint32_t id_mn = idesc_bf16_f32(128, 64, 0, 1);   // dV, dK: B MN-major
-      constexpr uint32_t id_dq = idesc_bf16_f32(128, 64, 1, 1);   // dQ: A and B MN-major
       const uint32_t k_s = smem_u32(sm.k), v_s = smem_u32(sm.v);
-      // Runs of MMAs from one asm block; descriptor steps in 16-byte units:
-      // K-major operands +32 B (2) per K = 16 step, MN-major +2048 B (128).
+      // descriptor steps in 16-byte units: K-major +32 B (2) per K = 16
+      // step, MN-major +2048 B (128)
       auto issue_kk = [&](uint32_t d_col, uint32_t a0, uint32_t b0) {
         mma_ss_run<4, 2, 0, 2>(tmem + d_col, desc_sw128(a0, 16, 1024), desc_sw128(b0, 16, 1024),
                                id_kk, 0u);
       };
-      // dK += dS^T Q_i from one dS tile pair: A rows = keys, K = queries
-      // (K-major; queries 64-127 in the second half tile)
-      // (step 4 jumps to the second half tile: +16 KB = 1024 units in all)
-      auto issue_dk = [&](const uint8_t (*ds)[kTileBytes], uint32_t q0, bool first) {
-        mma_ss_run<8, 2, kTileBytes / 16 - 8, 128>(
-            tmem + kColDK, desc_sw128(smem_u32(ds[0]), 16, 1024), desc_sw128(q0, 8192, 1024),
-            id_mn, first ? 0u : 1u);
+      auto wait_qd = [&](int it) {
+        return mbar_wait_parked(&sm.qd_full[it % kStages], (it / kStages) & 1, abort, err,
+                                kDevTimeoutFull);
       };
-      // dQ_i (+)= dS K_j from one dS tile pair: A M = queries (MN-major, the
-      // two 64-query halves 16 KB apart), K = keys
-      auto issue_dq = [&](const uint8_t (*ds)[kTileBytes], uint32_t col, bool first) {
-        mma_ss_run<8, 128, 0, 128>(tmem + col, desc_sw128(smem_u32(ds[0]), kTileBytes, 1024),
-                                   desc_sw128(k_s, 8192, 1024), id_dq, first ? 0u : 1u);
-      };
-      bool ok = mbar_wait(&sm.kv_full, 0, abort, err, kDevTimeoutFull) &&
-                mbar_wait(&sm.qd_full[0], 0, abort, err, kDevTimeoutFull);
+      bool ok = mbar_wait_parked(&sm.kv_full, 0, abort, err, kDevTimeoutFull) && n_q > 0 &&
+                wait_qd(0);
       if (ok) {
+        fence_after_sync();
         issue_kk(col_s(0), k_s, smem_u32(sm.q[0]));
         mma_commit_elect(&sm.s_full[0]);
         issue_kk(kColDP, v_s, smem_u32(sm.dout[0]));
@@ -228,32 +243,33 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       for (int it = 0; ok && it < n_q; ++it) {
         const int b = it & 1;
-        const bool next = it + 1 < n_q;
-        // the other S^T buffer holds dQ_it-1 until the compute warps drained it
-        if (it >= 1 && !mbar_wait(&sm.dq_empty, (it - 1) & 1, abort, err, kDevTimeoutOther)) break;
-        if (next) {
-          if (!mbar_wait(&sm.qd_full[b ^ 1], ((it + 1) >> 1) & 1, abort, err, kDevTimeoutFull))
-            break;
-          issue_kk(col_s(b ^ 1), k_s, smem_u32(sm.q[b ^ 1]));
+        const int st = it % kStages;
+        if (it + 1 < n_q) {
+          const int sn = (it + 1) % kStages;
+          // S^T_it+1 over P^T_it-1: the dV MMA that reads it was issued before
+          if (!wait_qd(it + 1)) break;
+          fence_after_sync();
+          issue_kk(col_s(b ^ 1), k_s, smem_u32(sm.q[sn]));
           mma_commit_elect(&sm.s_full[b ^ 1]);
-        }
-        if (!mbar_wait(&sm.sm_done, it & 1, abort, err, kDevTimeoutOther)) break;
-        fence_after_sync();
-        // dV += P^T dO_i: 16-query group kk's P^T is in dP^T columns 32(kk/2) + 8(kk%2)
-        mma_ts_run8<128, 8, 32, 40, 64, 72, 96, 104>(
-            tmem + kColDV, tmem + kColDP, desc_sw128(smem_u32(sm.dout[b]), 8192, 1024), id_mn,
-            it > 0 ? 1u : 0u);
-        if (next) {
-          issue_kk(kColDP, v_s, smem_u32(sm.dout[b ^ 1]));
+          // dP^T_it+1 once the compute warps hold dP^T_it in registers
+          if (!mbar_wait_parked(&sm.dp_free, it & 1, abort, err, kDevTimeoutOther)) break;
+          fence_after_sync();
+          issue_kk(kColDP, v_s, smem_u32(sm.dout[sn]));
           mma_commit_elect(&sm.dp_full);
         }
-        const uint32_t q0 = smem_u32(sm.q[b]);
-        issue_dk(sm.ds_hi[b], q0, it == 0);
-        issue_dk(sm.ds_lo[b], q0, false);
-        issue_dq(sm.ds_hi[b], col_s(b), true);
-        issue_dq(sm.ds_lo[b], col_s(b), false);
-        mma_commit_elect(&sm.dq_full);
-        mma_commit_elect(&sm.qd_empty[b]);
+        if (!mbar_wait_parked(&sm.sm_done, it & 1, abort, err, kDevTimeoutOther)) break;
+        fence_after_sync();
+        // dV += P^T dO_i: 16-query group kk's P^T is in S^T columns 32(kk/2) + 8(kk%2)
+        mma_ts_run8<128, 8, 32, 40, 64, 72, 96, 104>(
+            tmem + kColDV, tmem + col_s(b), desc_sw128(smem_u32(sm.dout[st]), 8192, 1024),
+            id_mn, it > 0 ? 1u : 0u);
+        // dK += dS^T Q_i: A rows = keys, K = queries (K-major; queries 64-127
+        // in the second half tile: step 4 jumps +16 KB = 1024 units in all)
+        mma_ss_run<8, 2, kTileBytes / 16 - 8, 128>(
+            tmem + kColDK, desc_sw128(smem_u32(sm.ds[b][0]), 16, 1024),
+            desc_sw128(smem_u32(sm.q[st]), 8192, 1024), id_mn, it > 0 ? 1u : 0u);
+        mma_commit_elect(&sm.ds_free[b]);
+        mma_commit_elect(&sm.qd_empty[st]);
       }
       mma_commit_elect(&sm.acc_full);
       mma_commit_elect(&sm.drain);
@@ -262,109 +278,81 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     __syncwarp();
   } else {
     // ------------------------------------------------------------- compute
-    const int w = warp >> 2;        // warpgroup: queries 32w..32w+31
-    const int tl = (warp & 3) * 32 + lane;  // TMEM lane: key row here, query row in dQ
+    const int w = warp >> 2;                 // warpgroup: queries 32w..32w+31
+    const int tl = (warp & 3) * 32 + lane;   // TMEM lane = key row
     const int jg = j0 + tl;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const int qw = 32 * w;                  // first query of this warpgroup in a block
-    const int half = w >> 1;
-    const uint32_t chunk0 = 4u * (uint32_t)(w & 1);  // first 16-byte chunk in the half-tile row
-    // dQ of the block before: rows = queries, this warpgroup's 16 columns
-    auto drain_dq = [&](int itp) -> bool {
-      if (!mbar_wait(&sm.dq_full, itp & 1, abort, err, kDevTimeoutMma)) return false;
-      fence_after_sync();
-      uint32_t a[16];
-      tmem_ld16(tmem + lane_off + col_s(itp & 1) + 16 * w, a);
-      tmem_wait_ld();
-      fence_before_sync();
-      mbar_arrive(&sm.dq_empty);
-      const int row = (ib0 + itp) * BQ + tl;
-      if (row < N) {
-        float* dst = dqacc + ((size_t)head * N + row) * HD + 16 * w;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          red_add_v4(dst + 4 * c, __uint_as_float(a[4 * c]), __uint_as_float(a[4 * c + 1]),
-                     __uint_as_float(a[4 * c + 2]), __uint_as_float(a[4 * c + 3]));
-      }
-      return true;
-    };
+    const int qw = 32 * w;
     bool ok = true;
     for (int it = 0; it < n_q; ++it) {
       const int b = it & 1;
+      const int st = it % kStages;
       const int ib = ib0 + it;
       const int i0 = ib * BQ;
       const bool need_mask = (causal && ib == jb) || (i0 + BQ > N) || (j0 + BK > N);
       // S^T_i done implies Q_i's stage (with lse and delta) has landed
-      if (!mbar_wait(&sm.s_full[b], (it >> 1) & 1, abort, err, kDevTimeoutMma) ||
-          !mbar_wait(&sm.dp_full, it & 1, abort, err, kDevTimeoutMma)) {
+      if (!mbar_wait_parked(&sm.s_full[b], (it >> 1) & 1, abort, err, kDevTimeoutMma) ||
+          !mbar_wait_parked(&sm.dp_full, it & 1, abort, err, kDevTimeoutMma)) {
         ok = false;
         break;
       }
       fence_after_sync();
       uint32_t sv[32], dpv[32];
       tmem_ld16(tmem + lane_off + col_s(b) + qw, *reinterpret_cast<uint32_t(*)[16]>(sv));
-      tmem_ld16(tmem + lane_off + col_s(b) + qw + 16, *reinterpret_cast<uint32_t(*)[16]>(sv + 16));
+      tmem_ld16(tmem + lane_off + col_s(b) + qw + 16,
+                *reinterpret_cast<uint32_t(*)[16]>(sv + 16));
       tmem_ld16(tmem + lane_off + kColDP + qw, *reinterpret_cast<uint32_t(*)[16]>(dpv));
       tmem_ld16(tmem + lane_off + kColDP + qw + 16,
                 *reinterpret_cast<uint32_t(*)[16]>(dpv + 16));
       tmem_wait_ld();
-      uint32_t wp[16], wh[16], wl[16];
-      const float4* l4 = reinterpret_cast<const float4*>(&sm.lse[b][qw]);
-      const float4* d4 = reinterpret_cast<const float4*>(&sm.delta[b][qw]);
+      fence_before_sync();
+      mbar_arrive(&sm.dp_free);  // dP^T's columns may take the next block's
+      // two queries at a time in packed f32x2 arithmetic:
+      //   p = 2^(s c - lse log2 e),  dS = p (dP - delta)
+      uint32_t wp[16], wd[16];
+      const float4* l4 = reinterpret_cast<const float4*>(&sm.nlse[st][qw]);
+      const float4* d4 = reinterpret_cast<const float4*>(&sm.delta[st][qw]);
+      const float2 c2 = make_float2(scale_log2, scale_log2);
+      const float2 m1 = make_float2(-1.f, -1.f);
 #pragma unroll
       for (int e4 = 0; e4 < 8; ++e4) {
         const float4 lv = l4[e4], dl = d4[e4];
-        const float la[4] = {lv.x, lv.y, lv.z, lv.w};
-        const float da[4] = {dl.x, dl.y, dl.z, dl.w};
-        float p[4], ds[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int e = 4 * e4 + u;
-          p[u] = ex2(fmaf(__uint_as_float(sv[e]), scale_log2, -la[u]));
-          ds[u] = p[u] * (__uint_as_float(dpv[e]) - da[u]);
-          if (need_mask) {
-            const int ig = i0 + qw + e;
-            if (ig >= N || jg >= N || (causal && ig < jg)) {
-              p[u] = 0.f;
-              ds[u] = 0.f;
-            }
-          }
-        }
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-          const int w2 = 2 * e4 + u;
-          wp[w2] = pack_bf16(p[2 * u], p[2 * u + 1]);
-          wh[w2] = pack_bf16(ds[2 * u], ds[2 * u + 1]);
-          wl[w2] = pack_bf16(ds[2 * u] - bf16lo(wh[w2]), ds[2 * u + 1] - bf16hi(wh[w2]));
+          const int e = 4 * e4 + 2 * u;
+          const float2 nl = u ? make_float2(lv.z, lv.w) : make_float2(lv.x, lv.y);
+          const float2 de = u ? make_float2(dl.z, dl.w) : make_float2(dl.x, dl.y);
+          const float2 a = __ffma2_rn(
+              make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), c2, nl);
+          float2 p = make_float2(ex2(a.x), ex2(a.y));
+          const float2 dd = __ffma2_rn(
+              de, m1, make_float2(__uint_as_float(dpv[e]), __uint_as_float(dpv[e + 1])));
+          float2 ds = __fmul2_rn(p, dd);
+          if (need_mask) {
+            const int ig = i0 + qw + e;
+            if (ig >= N || jg >= N || (causal && ig < jg)) p.x = ds.x = 0.f;
+            if (ig + 1 >= N || jg >= N || (causal && ig + 1 < jg)) p.y = ds.y = 0.f;
+          }
+          wp[2 * e4 + u] = pack_bf16(p.x, p.y);
+          wd[2 * e4 + u] = pack_bf16(ds.x, ds.y);
         }
       }
-      // P^T of this warpgroup's 32 queries over its own (already loaded) dP^T columns
-      tmem_st16(tmem + lane_off + kColDP + qw, wp);
-      // dS row of this key into buffer b: query q is element q % 64 of half
-      // q / 64; 16-byte chunk k (8 queries) of a half-tile row sits at chunk
-      // k ^ (key & 7) (128-byte swizzle)
-      {
-        const uint32_t hi_row = smem_u32(sm.ds_hi[b][half]) + tl * 128;
-        const uint32_t lo_row = smem_u32(sm.ds_lo[b][half]) + tl * 128;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const uint32_t off = ((chunk0 + g) ^ (uint32_t)(tl & 7)) << 4;
-          st_shared_v4(hi_row + off, wh[4 * g], wh[4 * g + 1], wh[4 * g + 2], wh[4 * g + 3]);
-          st_shared_v4(lo_row + off, wl[4 * g], wl[4 * g + 1], wl[4 * g + 2], wl[4 * g + 3]);
-        }
-      }
-      if (it >= 1 && !drain_dq(it - 1)) {
+      // P^T of this warpgroup's 32 queries over its own (already loaded) S^T columns
+      tmem_st16(tmem + lane_off + col_s(b) + qw, wp);
+      // dS^T row of this key into buffer b, once dK of block it-2 has read it
+      if (it >= 2 &&
+          !mbar_wait_parked(&sm.ds_free[b], ((it >> 1) - 1) & 1, abort, err, kDevTimeoutMma)) {
         ok = false;
         break;
       }
+      store_tile_row32(sm.ds[b], tl, qw, wd);
       tmem_wait_st();
       fence_proxy_async_smem();
       fence_before_sync();
       mbar_arrive(&sm.sm_done);
     }
-    if (ok && n_q > 0) ok = drain_dq(n_q - 1);
     // ---- columns 16w..16w+15 of this key's dv and dk
-    if (ok && mbar_wait(&sm.acc_full, 0, abort, err, kDevTimeoutMma)) {
+    if (ok && mbar_wait_parked(&sm.acc_full, 0, abort, err, kDevTimeoutMma)) {
       fence_after_sync();
       uint32_t av[16], ak[16];
       tmem_ld16(tmem + lane_off + kColDV + 16 * w, av);
@@ -375,19 +363,16 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         uint4* dkd = reinterpret_cast<uint4*>(dk + ((size_t)head * N + jg) * HD + 16 * w);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          dvd[h] = make_uint4(
-              pack_bf16(__uint_as_float(av[8 * h + 0]), __uint_as_float(av[8 * h + 1])),
-              pack_bf16(__uint_as_float(av[8 * h + 2]), __uint_as_float(av[8 * h + 3])),
-              pack_bf16(__uint_as_float(av[8 * h + 4]), __uint_as_float(av[8 * h + 5])),
-              pack_bf16(__uint_as_float(av[8 * h + 6]), __uint_as_float(av[8 * h + 7])));
-          dkd[h] = make_uint4(pack_bf16(__uint_as_float(ak[8 * h + 0]) * scale,
-                                        __uint_as_float(ak[8 * h + 1]) * scale),
-                              pack_bf16(__uint_as_float(ak[8 * h + 2]) * scale,
-                                        __uint_as_float(ak[8 * h + 3]) * scale),
-                              pack_bf16(__uint_as_float(ak[8 * h + 4]) * scale,
-                                        __uint_as_float(ak[8 * h + 5]) * scale),
-                              pack_bf16(__uint_as_float(ak[8 * h + 6]) * scale,
-                                        __uint_as_float(ak[8 * h + 7]) * scale));
+          uint32_t pv[4], pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            pv[e] = pack_bf16(__uint_as_float(av[8 * h + 2 * e]),
+                              __uint_as_float(av[8 * h + 2 * e + 1]));
+            pk[e] = pack_bf16(__uint_as_float(ak[8 * h + 2 * e]) * scale,
+                              __uint_as_float(ak[8 * h + 2 * e + 1]) * scale);
+          }
+          dvd[h] = make_uint4(pv[0], pv[1], pv[2], pv[3]);
+          dkd[h] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
       }
     }
@@ -401,25 +386,273 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   }
 }
 
-// dq = bf16(scale * dq accumulator) for the heads the tensor-core kernel took.
-__global__ void __launch_bounds__(256)
-attn_dq_convert_kernel(const float4* __restrict__ acc, uint4* __restrict__ dq, int64_t rows_per_head,
-                       int64_t total8, float scale, const int* __restrict__ flags) {
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  const int64_t per_head8 = rows_per_head * (HD / 8);
-  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total8; idx += stride) {
-    if (flags[idx / per_head8] != 0) continue;
-    const float4 a = acc[2 * idx], c = acc[2 * idx + 1];
-    dq[idx] = make_uint4(pack_bf16(a.x * scale, a.y * scale), pack_bf16(a.z * scale, a.w * scale),
-                         pack_bf16(c.x * scale, c.y * scale), pack_bf16(c.z * scale, c.w * scale));
+// ======================================================================= dQ
+
+struct __align__(1024) SmemQ {
+  uint8_t q[kTileBytes];
+  uint8_t dout[kTileBytes];
+  uint8_t k[kStages][kTileBytes];
+  uint8_t v[kStages][kTileBytes];
+  uint8_t ds_hi[2][kTileBytes];  // [key half]: dS [128 queries][64 keys]
+  uint8_t ds_lo[2][kTileBytes];
+  uint64_t q_full;
+  uint64_t kv_full[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t s_full[2];
+  uint64_t s_free[2];
+  uint64_t dp_full;
+  uint64_t dp_free;
+  uint64_t sm_done;
+  uint64_t ds_free;
+  uint64_t acc_full;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr size_t kSmemQ = sizeof(SmemQ);
+static_assert(kSmemQ <= 232448, "shared memory");
+constexpr uint32_t kColDQ = 384;
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ nlse2,
+                   const float* __restrict__ delta, __nv_bfloat16* __restrict__ dq, int N, int BH,
+                   int causal, float scale, float scale_log2, const int* __restrict__ flags,
+                   unsigned* __restrict__ err) {
+  const int n_blocks = (N + BQ - 1) / BQ;
+  const int Npad = n_blocks * BQ;
+  int head, ib;
+  block_order(n_blocks, BH, false, &head, &ib);
+  if (flags[head] != 0) return;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicCAS(err, 0u, (unsigned)kDevSmemAlign);
+    return;
+  }
+  SmemQ& sm = *reinterpret_cast<SmemQ*>(smem_raw);
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int n_k = causal ? ib + 1 : n_blocks;
+  const int i0 = ib * BQ;
+
+  if (tid == 0) {
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.kv_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.s_free[b], kComputeThreads);
+    }
+    mbar_init(&sm.dp_full, 1);
+    mbar_init(&sm.dp_free, kComputeThreads);
+    mbar_init(&sm.sm_done, kComputeThreads);
+    mbar_init(&sm.ds_free, 1);
+    mbar_init(&sm.acc_full, 1);
+    mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      prefetch_tmap(&tm_do);
+      mbar_arrive_expect_tx(&sm.q_full, 2 * kTileBytes);
+      tma_load_3d(sm.q, &tm_q, &sm.q_full, 0, i0, head);
+      tma_load_3d(sm.dout, &tm_do, &sm.q_full, 0, i0, head);
+      for (int jt = 0; jt < n_k; ++jt) {
+        const int s = jt % kStages;
+        const int round = jt / kStages;
+        if (round > 0 && !mbar_wait_parked(&sm.kv_empty[s], (round - 1) & 1, abort, err,
+                                           kDevTimeoutEmpty))
+          break;
+        mbar_arrive_expect_tx(&sm.kv_full[s], 2 * kTileBytes);
+        tma_load_3d(sm.k[s], &tm_k, &sm.kv_full[s], 0, jt * BK, head);
+        tma_load_3d(sm.v[s], &tm_v, &sm.kv_full[s], 0, jt * BK, head);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // --------------------------------------------------------- MMA issuer
+    {
+      constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, 0, 0);  // S, dP: both K-major
+      constexpr uint32_t id_mn = idesc_bf16_f32(128, 64, 0, 1);   // dQ: B (K_j) MN-major
+      const uint32_t q_s = smem_u32(sm.q), do_s = smem_u32(sm.dout);
+      auto issue_kk = [&](uint32_t d_col, uint32_t a0, uint32_t b0) {
+        mma_ss_run<4, 2, 0, 2>(tmem + d_col, desc_sw128(a0, 16, 1024), desc_sw128(b0, 16, 1024),
+                               id_kk, 0u);
+      };
+      // dQ (+)= dS K_j from one dS tile pair: A rows = queries, K = keys
+      // (K-major, keys 64-127 in the second half tile), B = K_j rows
+      // (+2048 B per 16 keys)
+      auto issue_dq = [&](const uint8_t (*ds)[kTileBytes], uint32_t k0, bool first) {
+        mma_ss_run<8, 2, kTileBytes / 16 - 8, 128>(
+            tmem + kColDQ, desc_sw128(smem_u32(ds[0]), 16, 1024), desc_sw128(k0, 8192, 1024),
+            id_mn, first ? 0u : 1u);
+      };
+      auto wait_kv = [&](int jt) {
+        return mbar_wait_parked(&sm.kv_full[jt % kStages], (jt / kStages) & 1, abort, err,
+                                kDevTimeoutFull);
+      };
+      bool ok = mbar_wait_parked(&sm.q_full, 0, abort, err, kDevTimeoutFull) && n_k > 0 &&
+                wait_kv(0);
+      if (ok) {
+        fence_after_sync();
+        issue_kk(col_s(0), q_s, smem_u32(sm.k[0]));
+        mma_commit_elect(&sm.s_full[0]);
+        issue_kk(kColDP, do_s, smem_u32(sm.v[0]));
+        mma_commit_elect(&sm.dp_full);
+      }
+      for (int jt = 0; ok && jt < n_k; ++jt) {
+        const int b = jt & 1;
+        const int st = jt % kStages;
+        if (jt + 1 < n_k) {
+          const int sn = (jt + 1) % kStages;
+          // S_jt+1 into the buffer of S_jt-1 once the compute warps hold it
+          if (!wait_kv(jt + 1)) break;
+          if (jt >= 1 && !mbar_wait_parked(&sm.s_free[b ^ 1], ((jt - 1) >> 1) & 1, abort, err,
+                                           kDevTimeoutOther))
+            break;
+          fence_after_sync();
+          issue_kk(col_s(b ^ 1), q_s, smem_u32(sm.k[sn]));
+          mma_commit_elect(&sm.s_full[b ^ 1]);
+          if (!mbar_wait_parked(&sm.dp_free, jt & 1, abort, err, kDevTimeoutOther)) break;
+          fence_after_sync();
+          issue_kk(kColDP, do_s, smem_u32(sm.v[sn]));
+          mma_commit_elect(&sm.dp_full);
+        }
+        if (!mbar_wait_parked(&sm.sm_done, jt & 1, abort, err, kDevTimeoutOther)) break;
+        fence_after_sync();
+        const uint32_t k0 = smem_u32(sm.k[st]);
+        issue_dq(sm.ds_hi, k0, jt == 0);
+        issue_dq(sm.ds_lo, k0, false);
+        mma_commit_elect(&sm.ds_free);
+        mma_commit_elect(&sm.kv_empty[st]);
+      }
+      mma_commit_elect(&sm.acc_full);
+      mma_commit_elect(&sm.drain);
+      wait_drain(&sm.drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------- compute
+    const int w = warp >> 2;                 // warpgroup: keys 32w..32w+31 of a block
+    const int tl = (warp & 3) * 32 + lane;   // TMEM lane = query row
+    const int ig = i0 + tl;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int kw = 32 * w;
+    const float nl = nlse2[(size_t)head * Npad + ig];  // -inf past N
+    const float dl = delta[(size_t)head * Npad + ig];  // 0 past N
+    const float2 c2 = make_float2(scale_log2, scale_log2);
+    const float2 nl2 = make_float2(nl, nl);
+    const float2 dl2 = make_float2(dl, dl);
+    const float2 m1 = make_float2(-1.f, -1.f);
+    bool ok = true;
+    for (int jt = 0; jt < n_k; ++jt) {
+      const int b = jt & 1;
+      const int j0 = jt * BK;
+      const bool need_mask = (causal && jt == ib) || (j0 + BK > N) || (i0 + BQ > N);
+      if (!mbar_wait_parked(&sm.s_full[b], (jt >> 1) & 1, abort, err, kDevTimeoutMma) ||
+          !mbar_wait_parked(&sm.dp_full, jt & 1, abort, err, kDevTimeoutMma)) {
+        ok = false;
+        break;
+      }
+      fence_after_sync();
+      uint32_t sv[32], dpv[32];
+      tmem_ld16(tmem + lane_off + col_s(b) + kw, *reinterpret_cast<uint32_t(*)[16]>(sv));
+      tmem_ld16(tmem + lane_off + col_s(b) + kw + 16,
+                *reinterpret_cast<uint32_t(*)[16]>(sv + 16));
+      tmem_ld16(tmem + lane_off + kColDP + kw, *reinterpret_cast<uint32_t(*)[16]>(dpv));
+      tmem_ld16(tmem + lane_off + kColDP + kw + 16,
+                *reinterpret_cast<uint32_t(*)[16]>(dpv + 16));
+      tmem_wait_ld();
+      fence_before_sync();
+      mbar_arrive(&sm.s_free[b]);  // S_jt's buffer may take S_jt+2
+      mbar_arrive(&sm.dp_free);    // dP's columns may take dP_jt+1
+      // two keys at a time in packed f32x2 arithmetic; lo = dS - hi is exact
+      uint32_t wh[16], wl[16];
+#pragma unroll
+      for (int e2 = 0; e2 < 16; ++e2) {
+        const int e = 2 * e2;
+        const float2 a = __ffma2_rn(
+            make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), c2, nl2);
+        const float2 p = make_float2(ex2(a.x), ex2(a.y));
+        const float2 dd = __ffma2_rn(
+            dl2, m1, make_float2(__uint_as_float(dpv[e]), __uint_as_float(dpv[e + 1])));
+        float2 ds = __fmul2_rn(p, dd);
+        if (need_mask) {
+          const int jg = j0 + kw + e;
+          if (jg >= N || ig >= N || (causal && jg > ig)) ds.x = 0.f;
+          if (jg + 1 >= N || ig >= N || (causal && jg + 1 > ig)) ds.y = 0.f;
+        }
+        wh[e2] = pack_bf16(ds.x, ds.y);
+        const float2 lo = __ffma2_rn(make_float2(bf16lo(wh[e2]), bf16hi(wh[e2])), m1, ds);
+        wl[e2] = pack_bf16(lo.x, lo.y);
+      }
+      // dS row of this query, once dQ of block jt-1 has read the tiles
+      if (jt >= 1 &&
+          !mbar_wait_parked(&sm.ds_free, (jt - 1) & 1, abort, err, kDevTimeoutMma)) {
+        ok = false;
+        break;
+      }
+      store_tile_row32(sm.ds_hi, tl, kw, wh);
+      store_tile_row32(sm.ds_lo, tl, kw, wl);
+      fence_proxy_async_smem();
+      fence_before_sync();
+      mbar_arrive(&sm.sm_done);
+    }
+    // ---- columns 16w..16w+15 of this query's dq
+    if (ok && mbar_wait_parked(&sm.acc_full, 0, abort, err, kDevTimeoutMma)) {
+      fence_after_sync();
+      uint32_t a[16];
+      tmem_ld16(tmem + lane_off + kColDQ + 16 * w, a);
+      tmem_wait_ld();
+      if (ig < N) {
+        uint4* dst = reinterpret_cast<uint4*>(dq + ((size_t)head * N + ig) * HD + 16 * w);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pq[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            pq[e] = pack_bf16(__uint_as_float(a[8 * h + 2 * e]) * scale,
+                              __uint_as_float(a[8 * h + 2 * e + 1]) * scale);
+          dst[h] = make_uint4(pq[0], pq[1], pq[2], pq[3]);
+        }
+      }
+    }
+  }
+
+  fence_before_sync();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    fence_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
 }  // namespace
 
 cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* dout,
-                               const float* lse2, const float* delta, void* dk, void* dv,
-                               float* dqacc, int64_t B, int64_t H, int64_t N, int causal,
+                               const float* nlse2, const float* delta, void* dq, void* dk,
+                               void* dv, int64_t B, int64_t H, int64_t N, int causal,
                                float scale, const int* flags, unsigned* err, cudaStream_t s,
                                int* launches) {
   const int64_t BH = B * H;
@@ -429,26 +662,22 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
   if ((e = make_tmap_bf16_rows(&tk, k, BH, N, BK)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_rows(&tv, v, BH, N, BK)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_rows(&tdo, dout, BH, N, BQ)) != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kSmemBytes);
+  e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kSmemKV);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attn_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kSmemQ);
   if (e != cudaSuccess) return e;
   const int64_t n_blocks = (N + BK - 1) / BK;
-  attn_bwd_tc_kernel<<<(unsigned)(n_blocks * BH), kThreads, kSmemBytes, s>>>(
-      tq, tk, tv, tdo, lse2, delta, static_cast<__nv_bfloat16*>(dk),
-      static_cast<__nv_bfloat16*>(dv), dqacc, (int)N, (int)BH, causal, scale, scale * kLog2e,
-      flags, err);
+  attn_bwd_dkdv_kernel<<<(unsigned)(n_blocks * BH), kThreads, kSmemKV, s>>>(
+      tq, tk, tv, tdo, nlse2, delta, static_cast<__nv_bfloat16*>(dk),
+      static_cast<__nv_bfloat16*>(dv), (int)N, (int)BH, causal, scale, scale * kLog2e, flags,
+      err);
   *launches += 1;
-  return cudaGetLastError();
-}
-
-cudaError_t launch_attn_dq_convert(const float* dqacc, void* dq, int64_t BH, int64_t N,
-                                   float scale, const int* flags, cudaStream_t s,
-                                   int* launches) {
-  const int64_t total8 = BH * N * HD / 8;
-  int64_t blocks = (total8 + 255) / 256;
-  if (blocks > 148 * 16) blocks = 148 * 16;
-  attn_dq_convert_kernel<<<(unsigned)blocks, 256, 0, s>>>(
-      reinterpret_cast<const float4*>(dqacc), static_cast<uint4*>(dq), N, total8, scale, flags);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  attn_bwd_dq_kernel<<<(unsigned)(n_blocks * BH), kThreads, kSmemQ, s>>>(
+      tq, tk, tv, tdo, nlse2, delta, static_cast<__nv_bfloat16*>(dq), (int)N, (int)BH, causal,
+      scale, scale * kLog2e, flags, err);
   *launches += 1;
   return cudaGetLastError();
 }

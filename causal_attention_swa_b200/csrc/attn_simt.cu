@@ -181,12 +181,12 @@ attn_fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
 // Backward row statistics, 8 threads per row, into two [heads][Npad]
 // float32 arrays (Npad = N rounded up to 128):
 //   delta[h][i] = sum_d dout_id * out_id      (0 for the padding rows)
-//   lse2[h][i]  = lse_i * log2(e)             (+inf for the padding rows)
+//   nlse2[h][i] = -lse_i * log2(e)            (-inf for the padding rows)
 template <typename T>
 __global__ void __launch_bounds__(256)
 attn_bwd_prep_kernel(const T* __restrict__ out, const T* __restrict__ dout,
                      const float* __restrict__ lse, float* __restrict__ delta,
-                     float* __restrict__ lse2, int64_t N, int64_t Npad, int64_t rows_pad) {
+                     float* __restrict__ nlse2, int64_t N, int64_t Npad, int64_t rows_pad) {
   const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t rp = g >> 3;
   const int part = (int)(g & 7);
@@ -205,7 +205,7 @@ attn_bwd_prep_kernel(const T* __restrict__ out, const T* __restrict__ dout,
   acc += __shfl_xor_sync(0xffffffffu, acc, 1);
   if (rp < rows_pad && part == 0) {
     delta[rp] = real ? acc : 0.f;
-    lse2[rp] = real ? lse[head * N + i] * kLog2e : INFINITY;
+    nlse2[rp] = real ? -lse[head * N + i] * kLog2e : -INFINITY;
   }
 }
 
@@ -439,17 +439,17 @@ cudaError_t launch_attn_fwd_simt(swa_dtype dt, const void* q, const void* k, con
 }
 
 cudaError_t launch_attn_bwd_prep(swa_dtype dt, const void* out, const void* dout,
-                                 const float* lse, float* delta, float* lse2, int64_t BH,
+                                 const float* lse, float* delta, float* nlse2, int64_t BH,
                                  int64_t N, int64_t Npad, cudaStream_t s, int* launches) {
   const int64_t rows_pad = BH * Npad;
   const unsigned blocks = (unsigned)((rows_pad * 8 + 255) / 256);
   if (dt == SWA_BF16)
     attn_bwd_prep_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
-        (const __nv_bfloat16*)out, (const __nv_bfloat16*)dout, lse, delta, lse2, N, Npad,
+        (const __nv_bfloat16*)out, (const __nv_bfloat16*)dout, lse, delta, nlse2, N, Npad,
         rows_pad);
   else
     attn_bwd_prep_kernel<float><<<blocks, 256, 0, s>>>((const float*)out, (const float*)dout,
-                                                       lse, delta, lse2, N, Npad, rows_pad);
+                                                       lse, delta, nlse2, N, Npad, rows_pad);
   *launches += 1;
   return cudaGetLastError();
 }

@@ -19,19 +19,14 @@ cudaError_t launch_attn_fwd_tc(const void* q, const void* k, const void* v, void
                                float scale, const int* flags, unsigned* err, cudaStream_t s,
                                int* launches);
 
-// Backward main kernel of the finite heads: dk, dv written directly; dq
-// contributions added into the float32 accumulator `dqacc` (zeroed by the
-// caller) with bulk reduce-adds.  lse2 = lse * log2 e and delta are the
-// prep kernel's [BH][Npad] arrays.
+// Backward of the finite heads: a key-major kernel writes dk and dv, a
+// query-major kernel writes dq (both directly in bf16, no accumulator in
+// memory).  nlse2 = -lse * log2 e and delta are the prep kernel's [BH][Npad]
+// arrays.
 cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* dout,
-                               const float* lse2, const float* delta, void* dk, void* dv,
-                               float* dqacc, int64_t B, int64_t H, int64_t N, int causal,
+                               const float* nlse2, const float* delta, void* dq, void* dk,
+                               void* dv, int64_t B, int64_t H, int64_t N, int causal,
                                float scale, const int* flags, unsigned* err, cudaStream_t s,
                                int* launches);
-
-// dq = bf16(scale * dqacc) for the finite heads.
-cudaError_t launch_attn_dq_convert(const float* dqacc, void* dq, int64_t BH, int64_t N,
-                                   float scale, const int* flags, cudaStream_t s,
-                                   int* launches);
 
 }  // namespace swa

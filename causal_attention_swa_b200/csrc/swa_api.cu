@@ -97,19 +97,18 @@ size_t fwd_ws(int64_t B, int64_t H, swa_dtype dt) {
   return dt == SWA_BF16 ? round_up((size_t)(B * H) * sizeof(int), 256) : 0;
 }
 
-// Backward workspace: per-head flags | delta [BH][Npad] | lse*log2e [BH][Npad]
-// | float32 dQ accumulator [BH][N][D] (bf16 only); Npad = N rounded up to 128.
+// Backward workspace: per-head flags | delta [BH][Npad] | -lse*log2e [BH][Npad];
+// Npad = N rounded up to 128.
 struct BwdWs {
-  size_t flags, delta, lse2, dqacc, total;
+  size_t flags, delta, nlse2, total;
 };
 
 BwdWs bwd_ws(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtype dt) {
   BwdWs w;
   w.flags = round_up((size_t)(B * H) * sizeof(int), 256);
   w.delta = round_up((size_t)(B * H * swa::pad128(N)) * sizeof(float), 256);
-  w.lse2 = w.delta;
-  w.dqacc = dt == SWA_BF16 ? round_up((size_t)(B * H * N * D) * sizeof(float), 256) : 0;
-  w.total = w.flags + w.delta + w.lse2 + w.dqacc;
+  w.nlse2 = w.delta;
+  w.total = w.flags + w.delta + w.nlse2;
   return w;
 }
 
@@ -214,12 +213,11 @@ swa_status swa_attn_bwd(const void* q, const void* k, const void* v, const void*
   char* base = static_cast<char*>(workspace);
   int* flags = reinterpret_cast<int*>(base);
   float* delta = reinterpret_cast<float*>(base + ws.flags);
-  float* lse2 = reinterpret_cast<float*>(base + ws.flags + ws.delta);
-  float* dqacc = reinterpret_cast<float*>(base + ws.flags + ws.delta + ws.lse2);
+  float* nlse2 = reinterpret_cast<float*>(base + ws.flags + ws.delta);
   const int64_t Npad = swa::pad128(N);
   const int c = causal ? 1 : 0;
   int launches = 0;
-  cudaError_t e = swa::launch_attn_bwd_prep(dt, out, dout, lse, delta, lse2, BH, N, Npad, s,
+  cudaError_t e = swa::launch_attn_bwd_prep(dt, out, dout, lse, delta, nlse2, BH, N, Npad, s,
                                             &launches);
   if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_prep");
   if (dt == SWA_F32) {
@@ -233,18 +231,14 @@ swa_status swa_attn_bwd(const void* q, const void* k, const void* v, const void*
     if (e != cudaSuccess) return cuda_fail(e, "scan_nonfinite(v)");
     e = swa::launch_scan_nonfinite(dt, dout, BH, N * D, flags, s, &launches);
     if (e != cudaSuccess) return cuda_fail(e, "scan_nonfinite(dout)");
-    // Heads with all-finite V and dout: tensor-core kernel (dk, dv directly,
-    // dq through the float32 accumulator); the others: pair-by-pair kernels.
-    e = cudaMemsetAsync(dqacc, 0, (size_t)BH * N * D * sizeof(float), s);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dq accumulator)");
+    // Heads with all-finite V and dout: tensor-core kernels (dk and dv
+    // key-major, dq query-major); the others: pair-by-pair kernels.
     {
       ProfScope ps(SWA_KERNEL_ATTN_BWD, s);
-      e = swa::launch_attn_bwd_tc(q, k, v, dout, lse2, delta, dk, dv, dqacc, B, H, N, c, scale,
+      e = swa::launch_attn_bwd_tc(q, k, v, dout, nlse2, delta, dq, dk, dv, B, H, N, c, scale,
                                   flags, err, s, &launches);
     }
     if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_tc");
-    e = swa::launch_attn_dq_convert(dqacc, dq, BH, N, scale, flags, s, &launches);
-    if (e != cudaSuccess) return cuda_fail(e, "attn_dq_convert");
     e = swa::launch_attn_bwd_simt(dt, q, k, v, dout, lse, delta, Npad, dq, dk, dv, BH, N, c,
                                   scale, flags, 1, s, &launches);
     if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_simt(non-finite heads)");

@@ -64,10 +64,10 @@ cudaError_t launch_attn_fwd_simt(swa_dtype dt, const void* q, const void* k, con
                                  float scale, const int* flags, int select, cudaStream_t s,
                                  int* launches);
 
-// delta[h][i] and lse2[h][i] = lse * log2 e, both [BH][Npad] (Npad = N
-// rounded up to 128; padding rows 0 and +inf).
+// delta[h][i] and nlse2[h][i] = -lse * log2 e, both [BH][Npad] (Npad = N
+// rounded up to 128; padding rows 0 and -inf).
 cudaError_t launch_attn_bwd_prep(swa_dtype dt, const void* out, const void* dout,
-                                 const float* lse, float* delta, float* lse2, int64_t BH,
+                                 const float* lse, float* delta, float* nlse2, int64_t BH,
                                  int64_t N, int64_t Npad, cudaStream_t s, int* launches);
 
 cudaError_t launch_attn_bwd_simt(swa_dtype dt, const void* q, const void* k, const void* v,

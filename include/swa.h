@@ -87,8 +87,8 @@ swa_status swa_attn_fwd(const void* q, const void* k, const void* v, void* out,
                         size_t workspace_bytes, void* stream);
 
 /*
- * Bytes of workspace swa_attn_bwd needs: per-head flags, delta [B,H,N]
- * float32 and, for bf16, a float32 dQ accumulator [B,H,N,D].
+ * Bytes of workspace swa_attn_bwd needs: per-head flags, and delta and
+ * lse * log2(e) as float32 [B,H,Npad] each (Npad = N rounded up to 128).
  */
 size_t swa_attn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D,
                                    swa_dtype dtype);

@@ -42,10 +42,9 @@ def test_workspace_sizes(lib):
     # bf16 forward: one int32 flag per head, rounded to 256 bytes
     assert lib.swa_attn_fwd_workspace_size(2, 16, 16384, 64, swa.SWA_BF16) == 256
     assert lib.swa_attn_fwd_workspace_size(1, 1, 256, 64, swa.SWA_F32) == 0
-    # bf16 backward: flags + delta and lse*log2(e) padded to 128-row blocks +
-    # float32 dQ accumulator
+    # backward: flags + delta and lse*log2(e) padded to 128-row blocks
     B, H, N, D = 2, 16, 16384, 64
-    want = 256 + 2 * B * H * N * 4 + B * H * N * D * 4
+    want = 256 + 2 * B * H * N * 4
     assert lib.swa_attn_bwd_workspace_size(B, H, N, D, swa.SWA_BF16) == want
     assert lib.swa_attn_bwd_workspace_size(1, 1, 256, 64, swa.SWA_F32) == 256 + 2 * 1024
     assert lib.swa_attn_bwd_workspace_size(1, 1, 300, 64, swa.SWA_F32) == 256 + 2 * 1536
