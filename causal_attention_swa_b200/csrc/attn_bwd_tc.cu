@@ -98,12 +98,14 @@ __device__ __forceinline__ void block_order(int n_blocks, int BH, bool heavy_low
 // [128 rows][128 columns] bf16 tile kept as two 64-column halves [128][64]
 // with the 128-byte swizzle: 16-byte chunk c of a half-tile row sits at
 // chunk c ^ (row & 7).
+// G0 and G1 select the 8-column chunks stored (0..3: columns col0 + 8g..).
+template <int G0 = 0, int G1 = 4>
 __device__ __forceinline__ void store_tile_row32(const uint8_t (*tile)[kTileBytes], int row,
                                                  int col0, const uint32_t (&w)[16]) {
   const uint32_t base = smem_u32(tile[col0 >> 6]) + row * 128;
   const uint32_t chunk0 = static_cast<uint32_t>((col0 & 63) >> 3);
 #pragma unroll
-  for (int g = 0; g < 4; ++g) {
+  for (int g = G0; g < G1; ++g) {
     const uint32_t off = ((chunk0 + g) ^ static_cast<uint32_t>(row & 7)) << 4;
     st_shared_v4(base + off, w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
   }
@@ -122,8 +124,7 @@ struct __align__(1024) SmemKV {
   uint64_t kv_full;
   uint64_t qd_full[kStages];
   uint64_t qd_empty[kStages];
-  uint64_t s_full[2];
-  uint64_t dp_full;
+  uint64_t dp_full;  // dP^T (and the S^T issued before it) of the next block
   uint64_t dp_free;
   uint64_t sm_done;
   uint64_t ds_free[2];
@@ -169,10 +170,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(&sm.qd_full[s], 1);
       mbar_init(&sm.qd_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm.s_full[b], 1);
-      mbar_init(&sm.ds_free[b], 1);
-    }
+    for (int b = 0; b < 2; ++b) mbar_init(&sm.ds_free[b], 1);
     mbar_init(&sm.dp_full, 1);
     mbar_init(&sm.dp_free, kComputeThreads);
     mbar_init(&sm.sm_done, kComputeThreads);
@@ -237,7 +235,6 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (ok) {
         fence_after_sync();
         issue_kk(col_s(0), k_s, smem_u32(sm.q[0]));
-        mma_commit_elect(&sm.s_full[0]);
         issue_kk(kColDP, v_s, smem_u32(sm.dout[0]));
         mma_commit_elect(&sm.dp_full);
       }
@@ -250,7 +247,6 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (!wait_qd(it + 1)) break;
           fence_after_sync();
           issue_kk(col_s(b ^ 1), k_s, smem_u32(sm.q[sn]));
-          mma_commit_elect(&sm.s_full[b ^ 1]);
           // dP^T_it+1 once the compute warps hold dP^T_it in registers
           if (!mbar_wait_parked(&sm.dp_free, it & 1, abort, err, kDevTimeoutOther)) break;
           fence_after_sync();
@@ -290,23 +286,21 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int ib = ib0 + it;
       const int i0 = ib * BQ;
       const bool need_mask = (causal && ib == jb) || (i0 + BQ > N) || (j0 + BK > N);
-      // S^T_i done implies Q_i's stage (with lse and delta) has landed
-      if (!mbar_wait_parked(&sm.s_full[b], (it >> 1) & 1, abort, err, kDevTimeoutMma) ||
-          !mbar_wait_parked(&sm.dp_full, it & 1, abort, err, kDevTimeoutMma)) {
+      // dP^T_i done implies S^T_i (issued before it) is done and Q_i's
+      // stage (with lse and delta) has landed
+      if (!mbar_wait_parked(&sm.dp_full, it & 1, abort, err, kDevTimeoutMma)) {
         ok = false;
         break;
       }
       fence_after_sync();
-      uint32_t sv[32], dpv[32];
-      tmem_ld16(tmem + lane_off + col_s(b) + qw, *reinterpret_cast<uint32_t(*)[16]>(sv));
-      tmem_ld16(tmem + lane_off + col_s(b) + qw + 16,
-                *reinterpret_cast<uint32_t(*)[16]>(sv + 16));
-      tmem_ld16(tmem + lane_off + kColDP + qw, *reinterpret_cast<uint32_t(*)[16]>(dpv));
-      tmem_ld16(tmem + lane_off + kColDP + qw + 16,
-                *reinterpret_cast<uint32_t(*)[16]>(dpv + 16));
+      // queries qw..qw+15 first; qw+16..qw+31 load while the first half is
+      // worked, and the first half's stores drain under the second half
+      uint32_t s0[16], d0[16], s1[16], d1[16];
+      tmem_ld16(tmem + lane_off + col_s(b) + qw, s0);
+      tmem_ld16(tmem + lane_off + kColDP + qw, d0);
       tmem_wait_ld();
-      fence_before_sync();
-      mbar_arrive(&sm.dp_free);  // dP^T's columns may take the next block's
+      tmem_ld16(tmem + lane_off + col_s(b) + qw + 16, s1);
+      tmem_ld16(tmem + lane_off + kColDP + qw + 16, d1);
       // two queries at a time in packed f32x2 arithmetic:
       //   p = 2^(s c - lse log2 e),  dS = p (dP - delta)
       uint32_t wp[16], wd[16];
@@ -314,38 +308,49 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       const float4* d4 = reinterpret_cast<const float4*>(&sm.delta[st][qw]);
       const float2 c2 = make_float2(scale_log2, scale_log2);
       const float2 m1 = make_float2(-1.f, -1.f);
+      auto math = [&](const uint32_t (&sv)[16], const uint32_t (&dpv)[16], int h) {
 #pragma unroll
-      for (int e4 = 0; e4 < 8; ++e4) {
-        const float4 lv = l4[e4], dl = d4[e4];
+        for (int e4 = 0; e4 < 4; ++e4) {
+          const float4 lv = l4[4 * h + e4], dl = d4[4 * h + e4];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int e = 4 * e4 + 2 * u;
-          const float2 nl = u ? make_float2(lv.z, lv.w) : make_float2(lv.x, lv.y);
-          const float2 de = u ? make_float2(dl.z, dl.w) : make_float2(dl.x, dl.y);
-          const float2 a = __ffma2_rn(
-              make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), c2, nl);
-          float2 p = make_float2(ex2(a.x), ex2(a.y));
-          const float2 dd = __ffma2_rn(
-              de, m1, make_float2(__uint_as_float(dpv[e]), __uint_as_float(dpv[e + 1])));
-          float2 ds = __fmul2_rn(p, dd);
-          if (need_mask) {
-            const int ig = i0 + qw + e;
-            if (ig >= N || jg >= N || (causal && ig < jg)) p.x = ds.x = 0.f;
-            if (ig + 1 >= N || jg >= N || (causal && ig + 1 < jg)) p.y = ds.y = 0.f;
+          for (int u = 0; u < 2; ++u) {
+            const int e = 4 * e4 + 2 * u;
+            const float2 nl = u ? make_float2(lv.z, lv.w) : make_float2(lv.x, lv.y);
+            const float2 de = u ? make_float2(dl.z, dl.w) : make_float2(dl.x, dl.y);
+            const float2 a = __ffma2_rn(
+                make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), c2, nl);
+            float2 p = make_float2(ex2(a.x), ex2(a.y));
+            const float2 dd = __ffma2_rn(
+                de, m1, make_float2(__uint_as_float(dpv[e]), __uint_as_float(dpv[e + 1])));
+            float2 ds = __fmul2_rn(p, dd);
+            if (need_mask) {
+              const int ig = i0 + qw + 16 * h + e;
+              if (ig >= N || jg >= N || (causal && ig < jg)) p.x = ds.x = 0.f;
+              if (ig + 1 >= N || jg >= N || (causal && ig + 1 < jg)) p.y = ds.y = 0.f;
+            }
+            wp[8 * h + 2 * e4 + u] = pack_bf16(p.x, p.y);
+            wd[8 * h + 2 * e4 + u] = pack_bf16(ds.x, ds.y);
           }
-          wp[2 * e4 + u] = pack_bf16(p.x, p.y);
-          wd[2 * e4 + u] = pack_bf16(ds.x, ds.y);
         }
-      }
-      // P^T of this warpgroup's 32 queries over its own (already loaded) S^T columns
-      tmem_st16(tmem + lane_off + col_s(b) + qw, wp);
+      };
+      math(s0, d0, 0);
+      // P^T of these 16 queries over the warpgroup's own, already loaded,
+      // S^T columns (16-query group 2w at columns 32w..32w+7)
+      tmem_st8(tmem + lane_off + col_s(b) + qw, *reinterpret_cast<const uint32_t(*)[8]>(wp));
+      tmem_wait_ld_tied(s1, d1);
+      fence_before_sync();
+      mbar_arrive(&sm.dp_free);  // dP^T's columns may take the next block's
       // dS^T row of this key into buffer b, once dK of block it-2 has read it
       if (it >= 2 &&
           !mbar_wait_parked(&sm.ds_free[b], ((it >> 1) - 1) & 1, abort, err, kDevTimeoutMma)) {
         ok = false;
         break;
       }
-      store_tile_row32(sm.ds[b], tl, qw, wd);
+      store_tile_row32<0, 2>(sm.ds[b], tl, qw, wd);
+      math(s1, d1, 1);
+      tmem_st8(tmem + lane_off + col_s(b) + qw + 8,
+               *reinterpret_cast<const uint32_t(*)[8]>(wp + 8));
+      store_tile_row32<2, 4>(sm.ds[b], tl, qw, wd);
       tmem_wait_st();
       fence_proxy_async_smem();
       fence_before_sync();
@@ -398,9 +403,8 @@ struct __align__(1024) SmemQ {
   uint64_t q_full;
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
-  uint64_t s_full[2];
   uint64_t s_free[2];
-  uint64_t dp_full;
+  uint64_t dp_full;  // dP (and the S issued before it) of the next block
   uint64_t dp_free;
   uint64_t sm_done;
   uint64_t ds_free;
@@ -445,10 +449,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm.s_full[b], 1);
-      mbar_init(&sm.s_free[b], kComputeThreads);
-    }
+    for (int b = 0; b < 2; ++b) mbar_init(&sm.s_free[b], kComputeThreads);
     mbar_init(&sm.dp_full, 1);
     mbar_init(&sm.dp_free, kComputeThreads);
     mbar_init(&sm.sm_done, kComputeThreads);
@@ -517,7 +518,6 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (ok) {
         fence_after_sync();
         issue_kk(col_s(0), q_s, smem_u32(sm.k[0]));
-        mma_commit_elect(&sm.s_full[0]);
         issue_kk(kColDP, do_s, smem_u32(sm.v[0]));
         mma_commit_elect(&sm.dp_full);
       }
@@ -533,7 +533,6 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
             break;
           fence_after_sync();
           issue_kk(col_s(b ^ 1), q_s, smem_u32(sm.k[sn]));
-          mma_commit_elect(&sm.s_full[b ^ 1]);
           if (!mbar_wait_parked(&sm.dp_free, jt & 1, abort, err, kDevTimeoutOther)) break;
           fence_after_sync();
           issue_kk(kColDP, do_s, smem_u32(sm.v[sn]));
@@ -570,51 +569,59 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int b = jt & 1;
       const int j0 = jt * BK;
       const bool need_mask = (causal && jt == ib) || (j0 + BK > N) || (i0 + BQ > N);
-      if (!mbar_wait_parked(&sm.s_full[b], (jt >> 1) & 1, abort, err, kDevTimeoutMma) ||
-          !mbar_wait_parked(&sm.dp_full, jt & 1, abort, err, kDevTimeoutMma)) {
+      // dP_jt done implies S_jt (issued before it) is done
+      if (!mbar_wait_parked(&sm.dp_full, jt & 1, abort, err, kDevTimeoutMma)) {
         ok = false;
         break;
       }
       fence_after_sync();
-      uint32_t sv[32], dpv[32];
-      tmem_ld16(tmem + lane_off + col_s(b) + kw, *reinterpret_cast<uint32_t(*)[16]>(sv));
-      tmem_ld16(tmem + lane_off + col_s(b) + kw + 16,
-                *reinterpret_cast<uint32_t(*)[16]>(sv + 16));
-      tmem_ld16(tmem + lane_off + kColDP + kw, *reinterpret_cast<uint32_t(*)[16]>(dpv));
-      tmem_ld16(tmem + lane_off + kColDP + kw + 16,
-                *reinterpret_cast<uint32_t(*)[16]>(dpv + 16));
+      // keys kw..kw+15 first; kw+16..kw+31 load while the first half is
+      // worked, and the first half's dS stores drain under the second half
+      uint32_t s0[16], d0[16], s1[16], d1[16];
+      tmem_ld16(tmem + lane_off + col_s(b) + kw, s0);
+      tmem_ld16(tmem + lane_off + kColDP + kw, d0);
       tmem_wait_ld();
+      tmem_ld16(tmem + lane_off + col_s(b) + kw + 16, s1);
+      tmem_ld16(tmem + lane_off + kColDP + kw + 16, d1);
+      // two keys at a time in packed f32x2 arithmetic; lo = dS - hi is exact
+      uint32_t wh[16], wl[16];
+      auto math = [&](const uint32_t (&sv)[16], const uint32_t (&dpv)[16], int h) {
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) {
+          const int e = 2 * e2;
+          const float2 a = __ffma2_rn(
+              make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), c2, nl2);
+          const float2 p = make_float2(ex2(a.x), ex2(a.y));
+          const float2 dd = __ffma2_rn(
+              dl2, m1, make_float2(__uint_as_float(dpv[e]), __uint_as_float(dpv[e + 1])));
+          float2 ds = __fmul2_rn(p, dd);
+          if (need_mask) {
+            const int jg = j0 + kw + 16 * h + e;
+            if (jg >= N || ig >= N || (causal && jg > ig)) ds.x = 0.f;
+            if (jg + 1 >= N || ig >= N || (causal && jg + 1 > ig)) ds.y = 0.f;
+          }
+          const int wi = 8 * h + e2;
+          wh[wi] = pack_bf16(ds.x, ds.y);
+          const float2 lo = __ffma2_rn(make_float2(bf16lo(wh[wi]), bf16hi(wh[wi])), m1, ds);
+          wl[wi] = pack_bf16(lo.x, lo.y);
+        }
+      };
+      math(s0, d0, 0);
+      tmem_wait_ld_tied(s1, d1);
       fence_before_sync();
       mbar_arrive(&sm.s_free[b]);  // S_jt's buffer may take S_jt+2
       mbar_arrive(&sm.dp_free);    // dP's columns may take dP_jt+1
-      // two keys at a time in packed f32x2 arithmetic; lo = dS - hi is exact
-      uint32_t wh[16], wl[16];
-#pragma unroll
-      for (int e2 = 0; e2 < 16; ++e2) {
-        const int e = 2 * e2;
-        const float2 a = __ffma2_rn(
-            make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), c2, nl2);
-        const float2 p = make_float2(ex2(a.x), ex2(a.y));
-        const float2 dd = __ffma2_rn(
-            dl2, m1, make_float2(__uint_as_float(dpv[e]), __uint_as_float(dpv[e + 1])));
-        float2 ds = __fmul2_rn(p, dd);
-        if (need_mask) {
-          const int jg = j0 + kw + e;
-          if (jg >= N || ig >= N || (causal && jg > ig)) ds.x = 0.f;
-          if (jg + 1 >= N || ig >= N || (causal && jg + 1 > ig)) ds.y = 0.f;
-        }
-        wh[e2] = pack_bf16(ds.x, ds.y);
-        const float2 lo = __ffma2_rn(make_float2(bf16lo(wh[e2]), bf16hi(wh[e2])), m1, ds);
-        wl[e2] = pack_bf16(lo.x, lo.y);
-      }
       // dS row of this query, once dQ of block jt-1 has read the tiles
       if (jt >= 1 &&
           !mbar_wait_parked(&sm.ds_free, (jt - 1) & 1, abort, err, kDevTimeoutMma)) {
         ok = false;
         break;
       }
-      store_tile_row32(sm.ds_hi, tl, kw, wh);
-      store_tile_row32(sm.ds_lo, tl, kw, wl);
+      store_tile_row32<0, 2>(sm.ds_hi, tl, kw, wh);
+      store_tile_row32<0, 2>(sm.ds_lo, tl, kw, wl);
+      math(s1, d1, 1);
+      store_tile_row32<2, 4>(sm.ds_hi, tl, kw, wh);
+      store_tile_row32<2, 4>(sm.ds_lo, tl, kw, wl);
       fence_proxy_async_smem();
       fence_before_sync();
       mbar_arrive(&sm.sm_done);
