@@ -337,8 +337,10 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       sm.part[t][slot][h][r] = mine_l2;
       mbar_arrive(pair);
       float m_new = m_used;
+      bool pair_seen = false;  // set by an earlier successful probe
       auto fetch_and_decide = [&]() -> bool {
-        if (!mbar_wait_parked(pair, par, abort, err, kDevTimeoutOther)) return false;
+        if (!pair_seen && !mbar_wait_parked(pair, par, abort, err, kDevTimeoutOther))
+          return false;
         const float theirs = sm.part[t][slot][h ^ 1][r];
         // the same operand order in both threads of the row
         const float cand = h == 0 ? fmaxf(mine_l2, theirs) : fmaxf(theirs, mine_l2);
@@ -349,17 +351,26 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       const bool early = __any_sync(0xffffffffu, j == 0 || !(mine_l2 <= m_used + kFastRange));
       if (early && !fetch_and_decide()) { ok = false; break; }
       const float m_exp = m_new;  // the reference the ex2 loop uses
+      // O_t += P_t,j-1 V_j-1 (issued at the end of the last tile) is probed
+      // now and waited for, if still needed, only after the ex2 loop
+      const bool pv_ready = j == 0 || mbar_test_wait(&sm.pv_done[t], (j - 1) & 1);
       float2 rsp[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       const float2 sc2 = make_float2(scale_log2, scale_log2);
       const float2 nm2 = make_float2(-m_exp, -m_exp);
       uint32_t pk[kHalf / 32][16];
+      auto exps = [&](int i) {
 #pragma unroll
-      for (int e = 0; e < kHalf / 2; ++e) {
-        const float2 a = __ffma2_rn(make_float2(x[2 * e], x[2 * e + 1]), sc2, nm2);
-        const float2 pe = make_float2(ex2(a.x), ex2(a.y));
-        rsp[e & 1] = __fadd2_rn(rsp[e & 1], pe);
-        pk[e >> 4][e & 15] = pack_bf16(pe.x, pe.y);
-      }
+        for (int e = 16 * i; e < 16 * i + 16; ++e) {
+          const float2 a = __ffma2_rn(make_float2(x[2 * e], x[2 * e + 1]), sc2, nm2);
+          const float2 pe = make_float2(ex2(a.x), ex2(a.y));
+          rsp[e & 1] = __fadd2_rn(rsp[e & 1], pe);
+          pk[i][e & 15] = pack_bf16(pe.x, pe.y);
+        }
+      };
+      exps(0);
+      // the partner published with this thread: probe between the halves
+      if (!early) pair_seen = mbar_test_wait(pair, par);
+      exps(1);
       if (!early && !fetch_and_decide()) { ok = false; break; }
       if (__any_sync(0xffffffffu, m_exp != m_new)) {  // rare: the partner moved the max
         const float beta = ex2(m_exp - m_new);
@@ -373,7 +384,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       // O_t += P_t,j-1 V_j-1 must finish before O_t is rescaled or P_t is
       // overwritten: by now it normally has.
       if (j > 0) {
-        if (!mbar_wait_parked(&sm.pv_done[t], (j - 1) & 1, abort, err, kDevTimeoutMma)) {
+        if (!pv_ready &&
+            !mbar_wait_parked(&sm.pv_done[t], (j - 1) & 1, abort, err, kDevTimeoutMma)) {
           ok = false;
           break;
         }
