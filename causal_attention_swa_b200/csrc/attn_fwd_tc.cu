@@ -287,8 +287,12 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                // threads of the row
     float l = 0.f;             // this thread's share of the row sum
     bool ok = true;
+    bool s_ready = false;  // S_t,j already seen complete by the probe of tile j-1
     for (int j = 0; j < n_t[t]; ++j) {
-      if (!mbar_wait_parked(&sm.s_full[t], j & 1, abort, err, kDevTimeoutMma)) { ok = false; break; }
+      if (!s_ready && !mbar_wait_parked(&sm.s_full[t], j & 1, abort, err, kDevTimeoutMma)) {
+        ok = false;
+        break;
+      }
       fence_after_sync();
       float x[kHalf];
       {
@@ -407,6 +411,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       m_used = m_new;
 #pragma unroll
       for (int i = 0; i < kHalf / 32; ++i) tmem_st16(tP + i * 16, pk[i]);
+      // S_t,j+1 was issued early in this tile: probe it while the stores land
+      s_ready = j + 1 < n_t[t] && mbar_test_wait(&sm.s_full[t], (j + 1) & 1);
       tmem_wait_st();
       fence_before_sync();
       mbar_arrive(&sm.p_full[t]);
