@@ -49,6 +49,8 @@
 // 0 by select.  These kernels take only heads whose V and dout are all
 // finite, so 0 times a finite value is the same as skipping the pair.
 // Every mbarrier wait is bounded (device error word on expiry).
+#include <type_traits>
+
 #include "attn_tc.cuh"
 #include "tc_ptx.cuh"
 
@@ -308,7 +310,11 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       const float4* d4 = reinterpret_cast<const float4*>(&sm.delta[st][qw]);
       const float2 c2 = make_float2(scale_log2, scale_log2);
       const float2 m1 = make_float2(-1.f, -1.f);
-      auto math = [&](const uint32_t (&sv)[16], const uint32_t (&dpv)[16], int h) {
+      // the mask flag is a compile-time constant of each instance, so the
+      // unmasked blocks' code carries no per-pair tests
+      auto math = [&](auto mask_tag, const uint32_t (&sv)[16], const uint32_t (&dpv)[16],
+                      int h) {
+        constexpr bool kMask = decltype(mask_tag)::value;
 #pragma unroll
         for (int e4 = 0; e4 < 4; ++e4) {
           const float4 lv = l4[4 * h + e4], dl = d4[4 * h + e4];
@@ -323,7 +329,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
             const float2 dd = __ffma2_rn(
                 de, m1, make_float2(__uint_as_float(dpv[e]), __uint_as_float(dpv[e + 1])));
             float2 ds = __fmul2_rn(p, dd);
-            if (need_mask) {
+            if constexpr (kMask) {
               const int ig = i0 + qw + 16 * h + e;
               if (ig >= N || jg >= N || (causal && ig < jg)) p.x = ds.x = 0.f;
               if (ig + 1 >= N || jg >= N || (causal && ig + 1 < jg)) p.y = ds.y = 0.f;
@@ -333,7 +339,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
         }
       };
-      math(s0, d0, 0);
+      if (need_mask) math(std::true_type{}, s0, d0, 0);
+      else math(std::false_type{}, s0, d0, 0);
       // P^T of these 16 queries over the warpgroup's own, already loaded,
       // S^T columns (16-query group 2w at columns 32w..32w+7)
       tmem_st8(tmem + lane_off + col_s(b) + qw, *reinterpret_cast<const uint32_t(*)[8]>(wp));
@@ -347,7 +354,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
         break;
       }
       store_tile_row32<0, 2>(sm.ds[b], tl, qw, wd);
-      math(s1, d1, 1);
+      if (need_mask) math(std::true_type{}, s1, d1, 1);
+      else math(std::false_type{}, s1, d1, 1);
       tmem_st8(tmem + lane_off + col_s(b) + qw + 8,
                *reinterpret_cast<const uint32_t(*)[8]>(wp + 8));
       store_tile_row32<2, 4>(sm.ds[b], tl, qw, wd);
@@ -585,7 +593,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
       tmem_ld16(tmem + lane_off + kColDP + kw + 16, d1);
       // two keys at a time in packed f32x2 arithmetic; lo = dS - hi is exact
       uint32_t wh[16], wl[16];
-      auto math = [&](const uint32_t (&sv)[16], const uint32_t (&dpv)[16], int h) {
+      auto math = [&](auto mask_tag, const uint32_t (&sv)[16], const uint32_t (&dpv)[16],
+                      int h) {
+        constexpr bool kMask = decltype(mask_tag)::value;
 #pragma unroll
         for (int e2 = 0; e2 < 8; ++e2) {
           const int e = 2 * e2;
@@ -595,7 +605,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
           const float2 dd = __ffma2_rn(
               dl2, m1, make_float2(__uint_as_float(dpv[e]), __uint_as_float(dpv[e + 1])));
           float2 ds = __fmul2_rn(p, dd);
-          if (need_mask) {
+          if constexpr (kMask) {
             const int jg = j0 + kw + 16 * h + e;
             if (jg >= N || ig >= N || (causal && jg > ig)) ds.x = 0.f;
             if (jg + 1 >= N || ig >= N || (causal && jg + 1 > ig)) ds.y = 0.f;
@@ -606,7 +616,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
           wl[wi] = pack_bf16(lo.x, lo.y);
         }
       };
-      math(s0, d0, 0);
+      if (need_mask) math(std::true_type{}, s0, d0, 0);
+      else math(std::false_type{}, s0, d0, 0);
       tmem_wait_ld_tied(s1, d1);
       fence_before_sync();
       mbar_arrive(&sm.s_free[b]);  // S_jt's buffer may take S_jt+2
@@ -619,7 +630,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       store_tile_row32<0, 2>(sm.ds_hi, tl, kw, wh);
       store_tile_row32<0, 2>(sm.ds_lo, tl, kw, wl);
-      math(s1, d1, 1);
+      if (need_mask) math(std::true_type{}, s1, d1, 1);
+      else math(std::false_type{}, s1, d1, 1);
       store_tile_row32<2, 4>(sm.ds_hi, tl, kw, wh);
       store_tile_row32<2, 4>(sm.ds_lo, tl, kw, wl);
       fence_proxy_async_smem();
