@@ -8,10 +8,12 @@
 // Work split: the (targets x sources) pair grid is cut into target tiles of
 // kTargetsPerBlock (kPerThread targets per thread, kept in registers) and
 // source chunks sized so the grid fills every SM several times over.  A
-// block stages its chunk as float4 (x*c, y*c, v, 0) in shared memory, where
-// c = sqrt(log2 e)/h folds the bandwidth and the base change into the
+// block stages its chunk as float4 (-x*c, -y*c, v, 0) in shared memory,
+// where c = sqrt(log2 e)/h folds the bandwidth and the base change into the
 // coordinates, so each pair costs 2 FADD, FMUL, FFMA, one MUFU ex2 (with the
-// sign folded into its operand), FADD and FFMA.  Partial (sum w, sum w v)
+// sign folded into its operand), FADD and FFMA -- the FP32 steps issued two
+// targets at a time as packed f32x2 instructions (bitwise the same sums),
+// which leaves MUFU as the one limit.  Partial (sum w, sum w v)
 // per (chunk, target) go to a float2 workspace; a second kernel adds them in
 // chunk order (deterministic) and divides.  0/0 gives NaN.
 #include "swa_internal.cuh"
@@ -41,39 +43,45 @@ nw_partial_kernel(const float* __restrict__ targets, int64_t M,
   const int ns = (int)imin64(chunk, S - s0);
   for (int e = tid; e < ns; e += kThreads) {
     const float2 xy = reinterpret_cast<const float2*>(sources)[s0 + e];
-    src[e] = make_float4(xy.x * c, xy.y * c, vals[s0 + e], 0.f);
+    src[e] = make_float4(-(xy.x * c), -(xy.y * c), vals[s0 + e], 0.f);
   }
   __syncthreads();
 
-  float tx[kPerThread], ty[kPerThread], sw[kPerThread], swv[kPerThread];
+  // targets in pairs: lane .x of pair u is target 2u, lane .y target 2u + 1
+  constexpr int kPairs = kPerThread / 2;
+  float2 tx[kPairs], ty[kPairs], sw[kPairs], swv[kPairs];
   const int64_t p0 = (int64_t)blockIdx.x * kTargetsPerBlock + tid;
 #pragma unroll
-  for (int t = 0; t < kPerThread; ++t) {
-    const int64_t p = p0 + (int64_t)t * kThreads;
-    float2 xy = make_float2(0.f, 0.f);
-    if (p < M) xy = reinterpret_cast<const float2*>(targets)[p];
-    tx[t] = xy.x * c;
-    ty[t] = xy.y * c;
-    sw[t] = 0.f;
-    swv[t] = 0.f;
+  for (int u = 0; u < kPairs; ++u) {
+    float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
+    const int64_t pa = p0 + (int64_t)(2 * u) * kThreads, pb = pa + kThreads;
+    if (pa < M) a = reinterpret_cast<const float2*>(targets)[pa];
+    if (pb < M) b = reinterpret_cast<const float2*>(targets)[pb];
+    tx[u] = make_float2(a.x * c, b.x * c);
+    ty[u] = make_float2(a.y * c, b.y * c);
+    sw[u] = make_float2(0.f, 0.f);
+    swv[u] = make_float2(0.f, 0.f);
   }
 #pragma unroll 4
   for (int e = 0; e < ns; ++e) {
     const float4 sv = src[e];
+    const float2 nsx = make_float2(sv.x, sv.x), nsy = make_float2(sv.y, sv.y);
+    const float2 v2 = make_float2(sv.z, sv.z);
 #pragma unroll
-    for (int t = 0; t < kPerThread; ++t) {
-      const float dx = tx[t] - sv.x;
-      const float dy = ty[t] - sv.y;
-      const float d2 = fmaf(dy, dy, dx * dx);
-      const float w = ex2_neg(d2);
-      sw[t] += w;
-      swv[t] = fmaf(w, sv.z, swv[t]);
+    for (int u = 0; u < kPairs; ++u) {
+      const float2 dx = __fadd2_rn(tx[u], nsx);
+      const float2 dy = __fadd2_rn(ty[u], nsy);
+      const float2 d2 = __ffma2_rn(dy, dy, __fmul2_rn(dx, dx));
+      const float2 w = make_float2(ex2_neg(d2.x), ex2_neg(d2.y));
+      sw[u] = __fadd2_rn(sw[u], w);
+      swv[u] = __ffma2_rn(w, v2, swv[u]);
     }
   }
 #pragma unroll
-  for (int t = 0; t < kPerThread; ++t) {
-    const int64_t p = p0 + (int64_t)t * kThreads;
-    if (p < M) partials[(int64_t)blockIdx.y * M + p] = make_float2(sw[t], swv[t]);
+  for (int u = 0; u < kPairs; ++u) {
+    const int64_t pa = p0 + (int64_t)(2 * u) * kThreads, pb = pa + kThreads;
+    if (pa < M) partials[(int64_t)blockIdx.y * M + pa] = make_float2(sw[u].x, swv[u].x);
+    if (pb < M) partials[(int64_t)blockIdx.y * M + pb] = make_float2(sw[u].y, swv[u].y);
   }
 }
 
