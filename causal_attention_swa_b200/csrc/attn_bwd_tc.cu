@@ -31,14 +31,19 @@
 //   S^T = K_j Q_i^T      (A = K smem K-major, B = Q smem K-major)
 //   dP^T = V_j dO_i^T    (A = V, B = dO, both K-major)
 //   dV += P^T dO_i       (A = P^T from TMEM, B = dO MN-major)
-//   dK += dS^T Q_i       (A = dS^T tile from smem, K-major; B = Q MN-major)
-// P^T (bf16) goes back over the warpgroup's own S^T columns 32w..32w+15
-// once loaded; dS^T (bf16) into a double-buffered [128 keys][128 queries]
-// tile (two 64-query halves, 128-byte swizzle).
+//   dK += dS^T Q_i       (A = dS^T from TMEM, B = Q MN-major)
+// P^T and dS^T (bf16) go back over the warpgroup's own, already loaded S^T
+// columns 32w..32w+15 and 32w+16..32w+31.
 // dq: thread t of warpgroup w owns query i0 + t (TMEM lane t) and keys
 // 32w..32w+31 of a block.  Per key block:
 //   S = Q_i K_j^T, dP = dO_i V_j^T   (all K-major)
-//   dQ += dS_hi K_j + dS_lo K_j      (A = dS tiles K-major, B = K MN-major)
+//   dQ += dS_hi K_j + dS_lo K_j      (A = dS from TMEM, B = K MN-major)
+// with dS_hi and dS_lo over the warpgroup's own S columns likewise.
+// Operands that a thread computes never pass through shared memory: an SS
+// MMA of N = 64 reads 6 KB of shared memory per 32 tensor cycles, above the
+// 128 bytes per clock the SM's shared memory delivers, while A from TMEM
+// costs none of it.  A later S MMA may overwrite those TMEM columns because
+// one thread's MMAs execute in issue order.
 // dS is carried as hi + lo bf16 (hi = bf16(dS), lo = bf16(dS - hi)) for dq:
 // sum_j dS_ij = 0, and a single bf16 rounding of dS, amplified by that
 // cancellation in sum_j dS_ij k_j, costs dq about 2% of its row RMS at
@@ -67,7 +72,8 @@ constexpr int kComputeThreads = 512;    // four warpgroups
 constexpr int kTmaWarp = 16;
 constexpr int kMmaWarp = 17;
 constexpr int kThreads = 576;
-constexpr int kStages = 3;              // streamed operand ring depth
+constexpr int kStages = 3;              // streamed operand ring depth (dq's K/V)
+constexpr int kQStages = 4;             // dkdv's Q/dO ring depth
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDP = 256;
 constexpr int kHeadGroup = 4;           // heads scheduled together (their operands share L2)
@@ -96,40 +102,21 @@ __device__ __forceinline__ void block_order(int n_blocks, int BH, bool heavy_low
   *blk = heavy_low ? rank : n_blocks - 1 - rank;
 }
 
-// Stores 32 bf16 values of one row (w[0..15], columns col0..col0+31) into a
-// [128 rows][128 columns] bf16 tile kept as two 64-column halves [128][64]
-// with the 128-byte swizzle: 16-byte chunk c of a half-tile row sits at
-// chunk c ^ (row & 7).
-// G0 and G1 select the 8-column chunks stored (0..3: columns col0 + 8g..).
-template <int G0 = 0, int G1 = 4>
-__device__ __forceinline__ void store_tile_row32(const uint8_t (*tile)[kTileBytes], int row,
-                                                 int col0, const uint32_t (&w)[16]) {
-  const uint32_t base = smem_u32(tile[col0 >> 6]) + row * 128;
-  const uint32_t chunk0 = static_cast<uint32_t>((col0 & 63) >> 3);
-#pragma unroll
-  for (int g = G0; g < G1; ++g) {
-    const uint32_t off = ((chunk0 + g) ^ static_cast<uint32_t>(row & 7)) << 4;
-    st_shared_v4(base + off, w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
-  }
-}
-
 // =================================================================== dK, dV
 
 struct __align__(1024) SmemKV {
   uint8_t k[kTileBytes];
   uint8_t v[kTileBytes];
-  uint8_t q[kStages][kTileBytes];
-  uint8_t dout[kStages][kTileBytes];
-  uint8_t ds[2][2][kTileBytes];  // [buffer][query half]: dS^T [128 keys][64 queries]
-  float nlse[kStages][BQ];       // -lse_i * log2(e) of each staged query block (-inf past N)
-  float delta[kStages][BQ];      // delta_i (0 past N)
+  uint8_t q[kQStages][kTileBytes];
+  uint8_t dout[kQStages][kTileBytes];
+  float nlse[kQStages][BQ];      // -lse_i * log2(e) of each staged query block (-inf past N)
+  float delta[kQStages][BQ];     // delta_i (0 past N)
   uint64_t kv_full;
-  uint64_t qd_full[kStages];
-  uint64_t qd_empty[kStages];
+  uint64_t qd_full[kQStages];
+  uint64_t qd_empty[kQStages];
   uint64_t dp_full;  // dP^T (and the S^T issued before it) of the next block
   uint64_t dp_free;
   uint64_t sm_done;
-  uint64_t ds_free[2];
   uint64_t acc_full;
   uint64_t drain;
   uint32_t tmem_base;
@@ -168,11 +155,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   if (tid == 0) {
     mbar_init(&sm.kv_full, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kQStages; ++s) {
       mbar_init(&sm.qd_full[s], 1);
       mbar_init(&sm.qd_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) mbar_init(&sm.ds_free[b], 1);
     mbar_init(&sm.dp_full, 1);
     mbar_init(&sm.dp_free, kComputeThreads);
     mbar_init(&sm.sm_done, kComputeThreads);
@@ -202,8 +188,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       tma_load_3d(sm.k, &tm_k, &sm.kv_full, 0, j0, head);
       tma_load_3d(sm.v, &tm_v, &sm.kv_full, 0, j0, head);
       for (int it = 0; it < n_q; ++it) {
-        const int s = it % kStages;
-        const int round = it / kStages;
+        const int s = it % kQStages;
+        const int round = it / kQStages;
         if (round > 0 && !mbar_wait_parked(&sm.qd_empty[s], (round - 1) & 1, abort, err,
                                            kDevTimeoutEmpty))
           break;
@@ -229,7 +215,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                                id_kk, 0u);
       };
       auto wait_qd = [&](int it) {
-        return mbar_wait_parked(&sm.qd_full[it % kStages], (it / kStages) & 1, abort, err,
+        return mbar_wait_parked(&sm.qd_full[it % kQStages], (it / kQStages) & 1, abort, err,
                                 kDevTimeoutFull);
       };
       bool ok = mbar_wait_parked(&sm.kv_full, 0, abort, err, kDevTimeoutFull) && n_q > 0 &&
@@ -242,10 +228,11 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       for (int it = 0; ok && it < n_q; ++it) {
         const int b = it & 1;
-        const int st = it % kStages;
+        const int st = it % kQStages;
         if (it + 1 < n_q) {
-          const int sn = (it + 1) % kStages;
-          // S^T_it+1 over P^T_it-1: the dV MMA that reads it was issued before
+          const int sn = (it + 1) % kQStages;
+          // S^T_it+1 over P^T_it-1 and dS^T_it-1: the dV and dK MMAs that
+          // read them were issued before
           if (!wait_qd(it + 1)) break;
           fence_after_sync();
           issue_kk(col_s(b ^ 1), k_s, smem_u32(sm.q[sn]));
@@ -261,12 +248,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
         mma_ts_run8<128, 8, 32, 40, 64, 72, 96, 104>(
             tmem + kColDV, tmem + col_s(b), desc_sw128(smem_u32(sm.dout[st]), 8192, 1024),
             id_mn, it > 0 ? 1u : 0u);
-        // dK += dS^T Q_i: A rows = keys, K = queries (K-major; queries 64-127
-        // in the second half tile: step 4 jumps +16 KB = 1024 units in all)
-        mma_ss_run<8, 2, kTileBytes / 16 - 8, 128>(
-            tmem + kColDK, desc_sw128(smem_u32(sm.ds[b][0]), 16, 1024),
-            desc_sw128(smem_u32(sm.q[st]), 8192, 1024), id_mn, it > 0 ? 1u : 0u);
-        mma_commit_elect(&sm.ds_free[b]);
+        // dK += dS^T Q_i: dS^T of 16-query group kk 16 columns further on
+        mma_ts_run8<128, 8, 32, 40, 64, 72, 96, 104>(
+            tmem + kColDK, tmem + col_s(b) + 16, desc_sw128(smem_u32(sm.q[st]), 8192, 1024),
+            id_mn, it > 0 ? 1u : 0u);
         mma_commit_elect(&sm.qd_empty[st]);
       }
       mma_commit_elect(&sm.acc_full);
@@ -284,7 +269,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
     bool ok = true;
     for (int it = 0; it < n_q; ++it) {
       const int b = it & 1;
-      const int st = it % kStages;
+      const int st = it % kQStages;
       const int ib = ib0 + it;
       const int i0 = ib * BQ;
       const bool need_mask = (causal && ib == jb) || (i0 + BQ > N) || (j0 + BK > N);
@@ -341,26 +326,20 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       };
       if (need_mask) math(std::true_type{}, s0, d0, 0);
       else math(std::false_type{}, s0, d0, 0);
-      // P^T of these 16 queries over the warpgroup's own, already loaded,
-      // S^T columns (16-query group 2w at columns 32w..32w+7)
-      tmem_st8(tmem + lane_off + col_s(b) + qw, *reinterpret_cast<const uint32_t(*)[8]>(wp));
+      // P^T and dS^T of these 16 queries over the warpgroup's own S^T
+      // columns: P^T at 32w + 0..7, dS^T at 32w + 16..23 (the latter only
+      // once the second half's load has landed)
+      const uint32_t tw = tmem + lane_off + col_s(b) + qw;
+      tmem_st8(tw, *reinterpret_cast<const uint32_t(*)[8]>(wp));
       tmem_wait_ld_tied(s1, d1);
       fence_before_sync();
       mbar_arrive(&sm.dp_free);  // dP^T's columns may take the next block's
-      // dS^T row of this key into buffer b, once dK of block it-2 has read it
-      if (it >= 2 &&
-          !mbar_wait_parked(&sm.ds_free[b], ((it >> 1) - 1) & 1, abort, err, kDevTimeoutMma)) {
-        ok = false;
-        break;
-      }
-      store_tile_row32<0, 2>(sm.ds[b], tl, qw, wd);
+      tmem_st8(tw + 16, *reinterpret_cast<const uint32_t(*)[8]>(wd));
       if (need_mask) math(std::true_type{}, s1, d1, 1);
       else math(std::false_type{}, s1, d1, 1);
-      tmem_st8(tmem + lane_off + col_s(b) + qw + 8,
-               *reinterpret_cast<const uint32_t(*)[8]>(wp + 8));
-      store_tile_row32<2, 4>(sm.ds[b], tl, qw, wd);
+      tmem_st8(tw + 8, *reinterpret_cast<const uint32_t(*)[8]>(wp + 8));
+      tmem_st8(tw + 24, *reinterpret_cast<const uint32_t(*)[8]>(wd + 8));
       tmem_wait_st();
-      fence_proxy_async_smem();
       fence_before_sync();
       mbar_arrive(&sm.sm_done);
     }
@@ -406,16 +385,12 @@ struct __align__(1024) SmemQ {
   uint8_t dout[kTileBytes];
   uint8_t k[kStages][kTileBytes];
   uint8_t v[kStages][kTileBytes];
-  uint8_t ds_hi[2][kTileBytes];  // [key half]: dS [128 queries][64 keys]
-  uint8_t ds_lo[2][kTileBytes];
   uint64_t q_full;
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
-  uint64_t s_free[2];
   uint64_t dp_full;  // dP (and the S issued before it) of the next block
   uint64_t dp_free;
   uint64_t sm_done;
-  uint64_t ds_free;
   uint64_t acc_full;
   uint64_t drain;
   uint32_t tmem_base;
@@ -457,11 +432,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) mbar_init(&sm.s_free[b], kComputeThreads);
     mbar_init(&sm.dp_full, 1);
     mbar_init(&sm.dp_free, kComputeThreads);
     mbar_init(&sm.sm_done, kComputeThreads);
-    mbar_init(&sm.ds_free, 1);
     mbar_init(&sm.acc_full, 1);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
@@ -509,13 +482,13 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
         mma_ss_run<4, 2, 0, 2>(tmem + d_col, desc_sw128(a0, 16, 1024), desc_sw128(b0, 16, 1024),
                                id_kk, 0u);
       };
-      // dQ (+)= dS K_j from one dS tile pair: A rows = queries, K = keys
-      // (K-major, keys 64-127 in the second half tile), B = K_j rows
-      // (+2048 B per 16 keys)
-      auto issue_dq = [&](const uint8_t (*ds)[kTileBytes], uint32_t k0, bool first) {
-        mma_ss_run<8, 2, kTileBytes / 16 - 8, 128>(
-            tmem + kColDQ, desc_sw128(smem_u32(ds[0]), 16, 1024), desc_sw128(k0, 8192, 1024),
-            id_mn, first ? 0u : 1u);
+      // dQ (+)= dS K_j with dS from TMEM: 16-key group kk's hi words at
+      // S columns 32(kk/2) + 8(kk%2), lo words 16 columns further on; B = K_j
+      // rows (+2048 B per 16 keys)
+      auto issue_dq = [&](uint32_t a_col, uint32_t k0, bool first) {
+        mma_ts_run8<128, 8, 32, 40, 64, 72, 96, 104>(tmem + kColDQ, tmem + a_col,
+                                                     desc_sw128(k0, 8192, 1024), id_mn,
+                                                     first ? 0u : 1u);
       };
       auto wait_kv = [&](int jt) {
         return mbar_wait_parked(&sm.kv_full[jt % kStages], (jt / kStages) & 1, abort, err,
@@ -534,11 +507,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int st = jt % kStages;
         if (jt + 1 < n_k) {
           const int sn = (jt + 1) % kStages;
-          // S_jt+1 into the buffer of S_jt-1 once the compute warps hold it
+          // S_jt+1 over dS_jt-1: the dQ MMAs that read it were issued before
           if (!wait_kv(jt + 1)) break;
-          if (jt >= 1 && !mbar_wait_parked(&sm.s_free[b ^ 1], ((jt - 1) >> 1) & 1, abort, err,
-                                           kDevTimeoutOther))
-            break;
           fence_after_sync();
           issue_kk(col_s(b ^ 1), q_s, smem_u32(sm.k[sn]));
           if (!mbar_wait_parked(&sm.dp_free, jt & 1, abort, err, kDevTimeoutOther)) break;
@@ -549,9 +519,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (!mbar_wait_parked(&sm.sm_done, jt & 1, abort, err, kDevTimeoutOther)) break;
         fence_after_sync();
         const uint32_t k0 = smem_u32(sm.k[st]);
-        issue_dq(sm.ds_hi, k0, jt == 0);
-        issue_dq(sm.ds_lo, k0, false);
-        mma_commit_elect(&sm.ds_free);
+        issue_dq(col_s(b), k0, jt == 0);
+        issue_dq(col_s(b) + 16, k0, false);
         mma_commit_elect(&sm.kv_empty[st]);
       }
       mma_commit_elect(&sm.acc_full);
@@ -618,23 +587,19 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
       };
       if (need_mask) math(std::true_type{}, s0, d0, 0);
       else math(std::false_type{}, s0, d0, 0);
+      // dS of these 16 keys over the warpgroup's own S columns: hi at
+      // 32w + 0..7, lo at 32w + 16..23 (once the second half's load landed)
+      const uint32_t tw = tmem + lane_off + col_s(b) + kw;
+      tmem_st8(tw, *reinterpret_cast<const uint32_t(*)[8]>(wh));
       tmem_wait_ld_tied(s1, d1);
       fence_before_sync();
-      mbar_arrive(&sm.s_free[b]);  // S_jt's buffer may take S_jt+2
-      mbar_arrive(&sm.dp_free);    // dP's columns may take dP_jt+1
-      // dS row of this query, once dQ of block jt-1 has read the tiles
-      if (jt >= 1 &&
-          !mbar_wait_parked(&sm.ds_free, (jt - 1) & 1, abort, err, kDevTimeoutMma)) {
-        ok = false;
-        break;
-      }
-      store_tile_row32<0, 2>(sm.ds_hi, tl, kw, wh);
-      store_tile_row32<0, 2>(sm.ds_lo, tl, kw, wl);
+      mbar_arrive(&sm.dp_free);  // dP's columns may take dP_jt+1
+      tmem_st8(tw + 16, *reinterpret_cast<const uint32_t(*)[8]>(wl));
       if (need_mask) math(std::true_type{}, s1, d1, 1);
       else math(std::false_type{}, s1, d1, 1);
-      store_tile_row32<2, 4>(sm.ds_hi, tl, kw, wh);
-      store_tile_row32<2, 4>(sm.ds_lo, tl, kw, wl);
-      fence_proxy_async_smem();
+      tmem_st8(tw + 8, *reinterpret_cast<const uint32_t(*)[8]>(wh + 8));
+      tmem_st8(tw + 24, *reinterpret_cast<const uint32_t(*)[8]>(wl + 8));
+      tmem_wait_st();
       fence_before_sync();
       mbar_arrive(&sm.sm_done);
     }
