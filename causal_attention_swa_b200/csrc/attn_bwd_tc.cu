@@ -380,14 +380,17 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
 
 // ======================================================================= dQ
 
+// Q_i and dO_i, the A operands of S and dP in every key block, sit in TMEM
+// (columns [448, 480) and [480, 512), written once by the compute warps from
+// their own rows), so those MMAs read only K_j and V_j from shared memory.
+constexpr int kKVStagesQ = 4;
+
 struct __align__(1024) SmemQ {
-  uint8_t q[kTileBytes];
-  uint8_t dout[kTileBytes];
-  uint8_t k[kStages][kTileBytes];
-  uint8_t v[kStages][kTileBytes];
-  uint64_t q_full;
-  uint64_t kv_full[kStages];
-  uint64_t kv_empty[kStages];
+  uint8_t k[kKVStagesQ][kTileBytes];
+  uint8_t v[kKVStagesQ][kTileBytes];
+  uint64_t qt_ready;  // Q_i and dO_i are in TMEM
+  uint64_t kv_full[kKVStagesQ];
+  uint64_t kv_empty[kKVStagesQ];
   uint64_t dp_full;  // dP (and the S issued before it) of the next block
   uint64_t dp_free;
   uint64_t sm_done;
@@ -398,13 +401,12 @@ struct __align__(1024) SmemQ {
 };
 constexpr size_t kSmemQ = sizeof(SmemQ);
 static_assert(kSmemQ <= 232448, "shared memory");
-constexpr uint32_t kColDQ = 384;
+constexpr uint32_t kColDQ = 384, kColQ = 448, kColDO = 480;
 
 __global__ void __launch_bounds__(kThreads, 1)
-attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
-                   const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v,
-                   const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ nlse2,
+attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16* __restrict__ q,
+                   const __nv_bfloat16* __restrict__ dout, const float* __restrict__ nlse2,
                    const float* __restrict__ delta, __nv_bfloat16* __restrict__ dq, int N, int BH,
                    int causal, float scale, float scale_log2, const int* __restrict__ flags,
                    unsigned* __restrict__ err) {
@@ -427,8 +429,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int i0 = ib * BQ;
 
   if (tid == 0) {
-    mbar_init(&sm.q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
+    mbar_init(&sm.qt_ready, kComputeThreads);
+    for (int s = 0; s < kKVStagesQ; ++s) {
       mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
     }
@@ -453,16 +455,11 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      prefetch_tmap(&tm_do);
-      mbar_arrive_expect_tx(&sm.q_full, 2 * kTileBytes);
-      tma_load_3d(sm.q, &tm_q, &sm.q_full, 0, i0, head);
-      tma_load_3d(sm.dout, &tm_do, &sm.q_full, 0, i0, head);
       for (int jt = 0; jt < n_k; ++jt) {
-        const int s = jt % kStages;
-        const int round = jt / kStages;
+        const int s = jt % kKVStagesQ;
+        const int round = jt / kKVStagesQ;
         if (round > 0 && !mbar_wait_parked(&sm.kv_empty[s], (round - 1) & 1, abort, err,
                                            kDevTimeoutEmpty))
           break;
@@ -477,10 +474,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
     {
       constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, 0, 0);  // S, dP: both K-major
       constexpr uint32_t id_mn = idesc_bf16_f32(128, 64, 0, 1);   // dQ: B (K_j) MN-major
-      const uint32_t q_s = smem_u32(sm.q), do_s = smem_u32(sm.dout);
-      auto issue_kk = [&](uint32_t d_col, uint32_t a0, uint32_t b0) {
-        mma_ss_run<4, 2, 0, 2>(tmem + d_col, desc_sw128(a0, 16, 1024), desc_sw128(b0, 16, 1024),
-                               id_kk, 0u);
+      // S = Q K_j^T and dP = dO V_j^T with A from TMEM (8 columns per 16
+      // dims) and B K-major (+32 B per 16 dims)
+      auto issue_kk = [&](uint32_t d_col, uint32_t a_col, uint32_t b0) {
+        mma_ts_run4<8, 2>(tmem + d_col, tmem + a_col, desc_sw128(b0, 16, 1024), id_kk, 0u);
       };
       // dQ (+)= dS K_j with dS from TMEM: 16-key group kk's hi words at
       // S columns 32(kk/2) + 8(kk%2), lo words 16 columns further on; B = K_j
@@ -491,29 +488,29 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                      first ? 0u : 1u);
       };
       auto wait_kv = [&](int jt) {
-        return mbar_wait_parked(&sm.kv_full[jt % kStages], (jt / kStages) & 1, abort, err,
-                                kDevTimeoutFull);
+        return mbar_wait_parked(&sm.kv_full[jt % kKVStagesQ], (jt / kKVStagesQ) & 1, abort,
+                                err, kDevTimeoutFull);
       };
-      bool ok = mbar_wait_parked(&sm.q_full, 0, abort, err, kDevTimeoutFull) && n_k > 0 &&
+      bool ok = mbar_wait_parked(&sm.qt_ready, 0, abort, err, kDevTimeoutOther) && n_k > 0 &&
                 wait_kv(0);
       if (ok) {
         fence_after_sync();
-        issue_kk(col_s(0), q_s, smem_u32(sm.k[0]));
-        issue_kk(kColDP, do_s, smem_u32(sm.v[0]));
+        issue_kk(col_s(0), kColQ, smem_u32(sm.k[0]));
+        issue_kk(kColDP, kColDO, smem_u32(sm.v[0]));
         mma_commit_elect(&sm.dp_full);
       }
       for (int jt = 0; ok && jt < n_k; ++jt) {
         const int b = jt & 1;
-        const int st = jt % kStages;
+        const int st = jt % kKVStagesQ;
         if (jt + 1 < n_k) {
-          const int sn = (jt + 1) % kStages;
+          const int sn = (jt + 1) % kKVStagesQ;
           // S_jt+1 over dS_jt-1: the dQ MMAs that read it were issued before
           if (!wait_kv(jt + 1)) break;
           fence_after_sync();
-          issue_kk(col_s(b ^ 1), q_s, smem_u32(sm.k[sn]));
+          issue_kk(col_s(b ^ 1), kColQ, smem_u32(sm.k[sn]));
           if (!mbar_wait_parked(&sm.dp_free, jt & 1, abort, err, kDevTimeoutOther)) break;
           fence_after_sync();
-          issue_kk(kColDP, do_s, smem_u32(sm.v[sn]));
+          issue_kk(kColDP, kColDO, smem_u32(sm.v[sn]));
           mma_commit_elect(&sm.dp_full);
         }
         if (!mbar_wait_parked(&sm.sm_done, jt & 1, abort, err, kDevTimeoutOther)) break;
@@ -541,6 +538,27 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
     const float2 nl2 = make_float2(nl, nl);
     const float2 dl2 = make_float2(dl, dl);
     const float2 m1 = make_float2(-1.f, -1.f);
+    {  // this thread's 16 dims (16w..16w+15) of Q_i and dO_i into TMEM (0 past N)
+      uint32_t qa[8], da[8];
+      if (ig < N) {
+        const size_t off = ((size_t)head * N + ig) * HD + 16 * w;
+        const uint4* qs = reinterpret_cast<const uint4*>(q + off);
+        const uint4* os = reinterpret_cast<const uint4*>(dout + off);
+        const uint4 q0 = qs[0], q1 = qs[1], e0 = os[0], e1 = os[1];
+        qa[0] = q0.x; qa[1] = q0.y; qa[2] = q0.z; qa[3] = q0.w;
+        qa[4] = q1.x; qa[5] = q1.y; qa[6] = q1.z; qa[7] = q1.w;
+        da[0] = e0.x; da[1] = e0.y; da[2] = e0.z; da[3] = e0.w;
+        da[4] = e1.x; da[5] = e1.y; da[6] = e1.z; da[7] = e1.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) qa[e] = da[e] = 0u;
+      }
+      tmem_st8(tmem + lane_off + kColQ + 8 * w, qa);
+      tmem_st8(tmem + lane_off + kColDO + 8 * w, da);
+      tmem_wait_st();
+      fence_before_sync();
+      mbar_arrive(&sm.qt_ready);
+    }
     bool ok = true;
     for (int jt = 0; jt < n_k; ++jt) {
       const int b = jt & 1;
@@ -660,7 +678,8 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
   *launches += 1;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   attn_bwd_dq_kernel<<<(unsigned)(n_blocks * BH), kThreads, kSmemQ, s>>>(
-      tq, tk, tv, tdo, nlse2, delta, static_cast<__nv_bfloat16*>(dq), (int)N, (int)BH, causal,
+      tk, tv, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dout),
+      nlse2, delta, static_cast<__nv_bfloat16*>(dq), (int)N, (int)BH, causal,
       scale, scale * kLog2e, flags, err);
   *launches += 1;
   return cudaGetLastError();
