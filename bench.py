@@ -334,7 +334,10 @@ def run_ours(args, info):
         "traffic": recorded_traffic(dom),
         "peak_source": f"{pk['source']} bf16 dense (burst)",
         "flops_per_launch": bwd_fl, "ms_per_launch": dom_ms,
+        "launch": "attn_bwd_dkdv_kernel + attn_bwd_dq_kernel (one event pair around both)",
     }
+    if pk.get("bf16_tflops_sustained") and achieved:
+        roofline["frac_of_sustained"] = achieved / pk["bf16_tflops_sustained"]
     # the other main kernels against their own bounds: the forward against the
     # bf16 tensor peak, the regrid against MUFU (148 SMs x 16 ex2/clk x max clock)
     mufu_peak = 148 * 16 * SM_MAX_MHZ * 1e6 / 1e9  # Gpair/s
