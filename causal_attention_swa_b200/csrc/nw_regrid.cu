@@ -22,7 +22,7 @@ namespace swa {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kPerThread = 4;
+constexpr int kPerThread = 8;
 constexpr int kTargetsPerBlock = kThreads * kPerThread;
 constexpr int kTargetBlocks = 148 * 8;   // blocks the grid aims for (SMs x resident blocks)
 constexpr int kMaxChunk = 2048;          // sources per block (32 KB of shared memory)
