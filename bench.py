@@ -323,6 +323,31 @@ def run_ours(args, info):
     e2e_ms = sdist.max_over_ranks(e_start.elapsed_time(e_stop), device) / args.steps
     e2e_value = (fwd_fl + bwd_fl) * info.world / (e2e_ms * 1e-3) / 1e12
 
+    # ---- the first widening row: non-causal attention (every pair, the same
+    # kernels without tile skipping), timed per API call after the step's
+    # measurements (its calls include the small scan and prep kernels)
+    nc_fwd, nc_bwd = [], []
+    for rep in range(5):
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        swa.attn_fwd(q, k, v, causal=False, out=out, lse=lse, workspace=ws_f)
+        e1.record(stream)
+        swa.attn_bwd(q, k, v, out, out, lse, causal=False, dq=dq, dk=dk, dv=dv, workspace=ws_b)
+        e2.record(stream)
+        torch.cuda.synchronize(device)
+        if rep >= 2:  # two warm-up calls
+            nc_fwd.append(e0.elapsed_time(e1))
+            nc_bwd.append(e1.elapsed_time(e2))
+    if swa.get_device_error(device) != swa.SWA_OK:
+        raise RuntimeError("device error word set during the non-causal calls")
+    nc_fl = 4 * D * B * H * N * N
+    nc_f_ms, nc_b_ms = sorted(nc_fwd)[1], sorted(nc_bwd)[1]
+    noncausal = {"workload": f"non-causal attention fwd+bwd B={B} H={H} N={N} D={D} bf16",
+                 "fwd_ms": nc_f_ms, "bwd_ms": nc_b_ms,
+                 "fwd_tflops": nc_fl / (nc_f_ms * 1e-3) / 1e12,
+                 "bwd_tflops": 2.5 * nc_fl / (nc_b_ms * 1e-3) / 1e12,
+                 "timing": "median of 3 API calls after 2 warm-up calls, CUDA events"}
+
     pk = peaks()
     dom = 2  # the backward's main kernel dominates the step
     dom_ms = kernel_ms[dom]
@@ -386,7 +411,7 @@ def run_ours(args, info):
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": timed_launches, "clocks": clocks.summary(),
-            "breakdown": breakdown, "rooflines": rooflines,
+            "breakdown": breakdown, "rooflines": rooflines, "noncausal": noncausal,
         }
         print(json.dumps(line), flush=True)
     sdist.shutdown()

@@ -216,3 +216,41 @@ def test_bf16_long_context_b1_h8_n65536(with_inf):
     heads, rows = sample_rows(np.random.default_rng(3), wl["H"], N, 24)
     check_forward_sampled(out, lse, q, k, v, heads, rows)
     _backward_sampled(qb, kb, vb, out, lse, dq, dk, dv, n_q=12, n_k=3, tail=64, seed=4)
+
+
+# --------------------------------------------------- non-causal (causal = 0)
+
+def test_bf16_noncausal_b1_h4_n2048_every_element():
+    """Every pair exists (the ABI's causal = 0): all tiles, none skipped or
+    masked except past N; compared element by element with the oracle."""
+    bits, (q, k, v) = bf16_case(1, 4, 2048, seed=11)
+    out, lse, (dq, dk, dv) = run_fwd_bwd(*(dev_bf16(b) for b in bits), causal=False)
+    w_out, w_lse = oracle.attn_fwd(q, k, v, causal=False)
+    check_bf16(out, w_out, "out")
+    check_lse(lse, w_lse, "lse")
+    w = oracle.attn_bwd(q, k, v, to_f64(out), causal=False, out=to_f64(out))
+    for name, g, ww in zip(("dq", "dk", "dv"), (dq, dk, dv), w):
+        check_bf16(g, ww, name)
+
+
+def test_bf16_noncausal_b2_h16_n16384_sampled():
+    """The non-causal call at the benchmark's size and launch configuration,
+    checked at sampled rows (keys anywhere: each sees all 16384 queries)."""
+    wl = inputs.WORKLOADS["attn_fwdbwd_b2h16n16384"]
+    qb, kb, vb, _ = inputs.attn_bf16(**wl)
+    out, lse, (dq, dk, dv) = run_fwd_bwd(dev_bf16(qb), dev_bf16(kb), dev_bf16(vb), causal=False)
+    for t in (out, lse, dq, dk, dv):
+        assert bool(torch.isfinite(t).all())
+    q, k, v = (inputs.bf16_to_f64(b) for b in (qb, kb, vb))
+    N = wl["N"]
+    rng = np.random.default_rng(12)
+    heads, rows = sample_rows(rng, 32, N, 16)
+    check_forward_sampled(out, lse, q, k, v, heads, rows, causal=False)
+    o = to_f64(out)
+    qh, qr = sample_rows(rng, 32, N, 8)
+    kh = np.array([5, 5], dtype=np.int64)
+    kr = np.array([0, N // 2 + 17], dtype=np.int64)
+    w_dq, w_dk, w_dv = oracle.attn_bwd_rows(q, k, v, o, qh, qr, kh, kr, causal=False, out=o)
+    check_bf16(to_f64(dq).reshape(-1, N, 64)[qh, qr], w_dq, "dq (sampled rows)")
+    check_bf16(to_f64(dk).reshape(-1, N, 64)[kh, kr], w_dk, "dk (sampled rows)")
+    check_bf16(to_f64(dv).reshape(-1, N, 64)[kh, kr], w_dv, "dv (sampled rows)")
