@@ -72,7 +72,6 @@ constexpr int kComputeThreads = 512;    // four warpgroups
 constexpr int kTmaWarp = 16;
 constexpr int kMmaWarp = 17;
 constexpr int kThreads = 576;
-constexpr int kStages = 3;              // streamed operand ring depth (dq's K/V)
 constexpr int kQStages = 4;             // dkdv's Q/dO ring depth
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDP = 256;

@@ -26,7 +26,7 @@ EXPORTS = (
     "swa_attn_fwd_workspace_size", "swa_attn_fwd", "swa_attn_bwd_workspace_size",
     "swa_attn_bwd", "swa_nw_workspace_size", "swa_nw_regrid", "swa_get_device_error",
     "swa_status_string", "swa_last_error_message", "swa_last_launch_count",
-    "swa_profile_kernel", "swa_attn_fwd_noalloc",
+    "swa_profile_kernel", "swa_attn_fwd_noalloc", "swa_selftest_wait_timeout",
 )
 SWA_KERNEL_NONE, SWA_KERNEL_ATTN_FWD, SWA_KERNEL_ATTN_BWD, SWA_KERNEL_NW = range(4)
 
@@ -71,6 +71,8 @@ def load_library():
     lib.swa_nw_regrid.restype = I
     lib.swa_get_device_error.argtypes = [P]
     lib.swa_get_device_error.restype = I
+    lib.swa_selftest_wait_timeout.argtypes = [P]
+    lib.swa_selftest_wait_timeout.restype = I
     lib.swa_status_string.argtypes = [I]
     lib.swa_status_string.restype = ctypes.c_char_p
     lib.swa_last_error_message.argtypes = []
@@ -198,6 +200,16 @@ def nw_regrid(targets, sources, vals, h: float = 0.5, out=None, workspace=None):
                            _ptr(ws), nbytes, _stream_ptr(targets.device))
     _check(st, "swa_nw_regrid")
     return out
+
+
+def selftest_wait_timeout(device=None) -> None:
+    """swa_selftest_wait_timeout on the current stream (a kernel whose bounded
+    waits run out; read the result with get_device_error)."""
+    dev = torch.device("cuda") if device is None else device
+    st = int(load_library().swa_selftest_wait_timeout(_stream_ptr(dev)))
+    if st != SWA_OK:
+        raise SwaError(st, "swa_selftest_wait_timeout",
+                       load_library().swa_last_error_message().decode())
 
 
 def get_device_error(device=None) -> int:

@@ -152,6 +152,17 @@ swa_status swa_nw_regrid(const float* targets, int64_t M, const float* sources,
  */
 swa_status swa_get_device_error(void* stream);
 
+/*
+ * Diagnostic of the device-side failure path: enqueues on `stream` one small
+ * kernel whose bounded waits (the same code every tensor-core kernel's
+ * waits use) run out, since nothing arrives at the barriers they wait on.
+ * The kernel exits normally after about 2 s of SM clock; a following
+ * swa_get_device_error() reports SWA_ERR_DEVICE_TIMEOUT and clears the
+ * word, and the context stays usable.  Returns SWA_OK once enqueued, or
+ * SWA_ERR_CUDA.
+ */
+swa_status swa_selftest_wait_timeout(void* stream);
+
 /* Static string naming a status code. */
 const char* swa_status_string(swa_status status);
 
