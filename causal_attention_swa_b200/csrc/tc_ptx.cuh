@@ -82,26 +82,11 @@ __device__ __forceinline__ bool mbar_try_wait_parked(uint64_t* bar, uint32_t par
   return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete.  Gives up (returns
-// false) when *abort becomes non-zero or after kWaitCycles; on a timeout it
-// records `code` in the device error word and raises *abort so that every
-// other role of the block leaves its loop too.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          unsigned* err, unsigned code) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if (clock64() - t0 > kWaitCycles) {
-      atomicCAS(err, 0u, code);
-      *abort = 1;
-      return false;
-    }
-  }
-}
-
-// mbar_wait that parks between polls (see mbar_try_wait_parked).
+// Waits for the phase with the given parity to complete, parking between
+// polls (see mbar_try_wait_parked).  Gives up (returns false) when *abort
+// becomes non-zero or after kWaitCycles; on a timeout it records `code` in
+// the device error word and raises *abort, so that every role of the block
+// leaves its loop instead of waiting for a partner that gave up.
 __device__ __forceinline__ bool mbar_wait_parked(uint64_t* bar, uint32_t parity,
                                                  volatile int* abort, unsigned* err,
                                                  unsigned code) {
@@ -116,19 +101,6 @@ __device__ __forceinline__ bool mbar_wait_parked(uint64_t* bar, uint32_t parity,
       return false;
     }
   }
-}
-
-// mbar_wait by lane 0 only (one shared-memory poll per warp instead of 32),
-// result broadcast; the warp barrier orders the other lanes after lane 0's
-// acquire.  All 32 lanes of the warp must call it.
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
-                                               volatile int* abort, unsigned* err,
-                                               unsigned code) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, err, code) ? 1 : 0;
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  __syncwarp();
-  return ok != 0;
 }
 
 // ----------------------------------------------------------------------- TMA
@@ -181,53 +153,6 @@ __device__ __forceinline__ void fence_before_sync() {
 
 __device__ __forceinline__ void fence_after_sync() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// D[tmem] (+)= A[smem desc] * B[smem desc]
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// D[tmem] (+)= A[tmem] * B[smem desc]
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Warp-converged issue: every lane of the warp executes these with the same
-// (uniform) operands and one elected lane issues the instruction, so the
-// descriptors stay in uniform registers.
-__device__ __forceinline__ void mma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                             uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                             uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
 }
 
 // A run of kN MMAs into one accumulator from one asm block (one elect.sync):
@@ -345,15 +270,6 @@ __device__ __forceinline__ void mma_commit_elect(uint64_t* bar) {
       : "memory");
 }
 
-// Arrive on an mbarrier once every tcgen05 operation this thread issued
-// before has completed.
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_u32(bar))
-      : "memory");
-}
-
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -415,58 +331,6 @@ __device__ __forceinline__ void regs_increase() {
 template <int kRegs>
 __device__ __forceinline__ void regs_decrease() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
-}
-
-// ------------------------------------------------------ bulk copies, proxies
-
-// Make this thread's generic-proxy shared-memory writes visible to the
-// async proxy (tcgen05.mma operands, bulk copies).
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// Element-wise f32 add of `bytes` contiguous shared-memory bytes into global
-// memory (16-byte aligned addresses, bytes a multiple of 16).
-__device__ __forceinline__ void bulk_reduce_add_f32(float* gdst, const void* ssrc,
-                                                    uint32_t bytes) {
-  asm volatile(
-      "cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
-          reinterpret_cast<uint64_t>(gdst)),
-      "r"(smem_u32(ssrc)), "r"(bytes)
-      : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit_group() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// Wait until every committed bulk group has finished reading its source.
-__device__ __forceinline__ void bulk_wait_group_read0() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-
-// Wait until every committed bulk group has completed.
-__device__ __forceinline__ void bulk_wait_group0() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
-// Vector float32 atomic add (no return) into global memory, 16-byte aligned.
-__device__ __forceinline__ void red_add_v4(float* gdst, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(gdst), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
-
-// Named barrier among `nthreads` threads (a multiple of 32).
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-__device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
 }
 
 // ---------------------------------------------------------------- descriptors
