@@ -245,14 +245,17 @@ def run_ours(args, info):
     ws_n = torch.empty(swa.nw_workspace_size(NW_M, NW_S), dtype=torch.uint8, device=device)
     launches = [0]
 
-    def step(src):
-        swa.attn_fwd(src["q"], src["k"], src["v"], causal=True, out=out, lse=lse,
+    main_out = {"out": out, "lse": lse, "dq": dq, "dk": dk, "dv": dv, "nw": nw_out}
+
+    def step(src, dst=None):
+        d = main_out if dst is None else dst
+        swa.attn_fwd(src["q"], src["k"], src["v"], causal=True, out=d["out"], lse=d["lse"],
                      workspace=ws_f)
         launches[0] += swa.last_launch_count()
-        swa.attn_bwd(src["q"], src["k"], src["v"], out, out, lse, causal=True, dq=dq, dk=dk,
-                     dv=dv, workspace=ws_b)
+        swa.attn_bwd(src["q"], src["k"], src["v"], d["out"], d["out"], d["lse"], causal=True,
+                     dq=d["dq"], dk=d["dk"], dv=d["dv"], workspace=ws_b)
         launches[0] += swa.last_launch_count()
-        swa.nw_regrid(src["nt"], src["ns"], src["ny"], h=H_BW, out=nw_out, workspace=ws_n)
+        swa.nw_regrid(src["nt"], src["ns"], src["ny"], h=H_BW, out=d["nw"], workspace=ws_n)
         launches[0] += swa.last_launch_count()
 
     stream = torch.cuda.current_stream(device)
@@ -295,29 +298,50 @@ def run_ours(args, info):
     ms_per_step = elapsed_ms / args.steps
     value = (fwd_fl + bwd_fl) * info.world / (elapsed_ms / args.steps * 1e-3) / 1e12
 
-    # ---- end to end through the public API with host buffers: H2D of the
-    # step's inputs from pinned memory, the step, D2H of its results.
+    # ---- end to end through the public API with host buffers: every step
+    # copies its inputs in from pinned host memory and its results back out.
+    # The copies run on streams of their own with the device side
+    # double-buffered, so step s+1's inputs go in and step s-1's results come
+    # out while step s computes (the link is full duplex); the bytes each
+    # step moves are the same as with no overlap.
     host_out = {"out": torch.empty_like(out, device="cpu").pin_memory(),
                 "lse": torch.empty_like(lse, device="cpu").pin_memory(),
                 "dq": torch.empty_like(dq, device="cpu").pin_memory(),
                 "dk": torch.empty_like(dk, device="cpu").pin_memory(),
                 "dv": torch.empty_like(dv, device="cpu").pin_memory(),
                 "nw": torch.empty_like(nw_out, device="cpu").pin_memory()}
-    dev_out = {"out": out, "lse": lse, "dq": dq, "dk": dk, "dv": dv, "nw": nw_out}
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-    e2e_in = {name: torch.empty_like(t) for name, t in dev_in.items()}
+    bufs = [({name: torch.empty_like(t) for name, t in dev_in.items()},
+             {name: torch.empty_like(t) for name, t in main_out.items()}) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
+    for e in comp_done + out_done:
+        e.record(stream)
     e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sdist.barrier(device)
     torch.cuda.synchronize(device)
-    e_start.record(stream)
-    for _ in range(args.steps):
-        for name, t in host_in.items():
-            e2e_in[name].copy_(t, non_blocking=True)
-        step(e2e_in)
-        for name, t in dev_out.items():
-            host_out[name].copy_(t, non_blocking=True)
-    e_stop.record(stream)
+    e_start.record(s_in)
+    for i in range(args.steps):
+        b = i % 2
+        ins, outs = bufs[b]
+        s_in.wait_event(comp_done[b])  # step i-2, the last reader of these inputs, is done
+        with torch.cuda.stream(s_in):
+            for name, t in host_in.items():
+                ins[name].copy_(t, non_blocking=True)
+        in_ready[b].record(s_in)
+        stream.wait_event(in_ready[b])
+        stream.wait_event(out_done[b])  # step i-2's results have left this buffer
+        step(ins, outs)
+        comp_done[b].record(stream)
+        s_out.wait_event(comp_done[b])
+        with torch.cuda.stream(s_out):
+            for name, t in outs.items():
+                host_out[name].copy_(t, non_blocking=True)
+        out_done[b].record(s_out)
+    e_stop.record(s_out)
     torch.cuda.synchronize(device)
     sdist.barrier(device)
     e2e_ms = sdist.max_over_ranks(e_start.elapsed_time(e_stop), device) / args.steps
