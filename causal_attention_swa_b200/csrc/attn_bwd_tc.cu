@@ -36,7 +36,7 @@
 // columns 32w..32w+15 and 32w+16..32w+31.
 // dq: thread t of warpgroup w owns query i0 + t (TMEM lane t) and keys
 // 32w..32w+31 of a block.  Per key block:
-//   S = Q_i K_j^T, dP = dO_i V_j^T   (all K-major)
+//   S = Q_i K_j^T, dP = dO_i V_j^T   (A from TMEM, B K-major)
 //   dQ += dS_hi K_j + dS_lo K_j      (A = dS from TMEM, B = K MN-major)
 // with dS_hi and dS_lo over the warpgroup's own S columns likewise.
 // Operands that a thread computes never pass through shared memory: an SS
