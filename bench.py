@@ -390,12 +390,18 @@ def run_ours(args, info):
     # the other main kernels against their own bounds: the forward against the
     # bf16 tensor peak, the regrid against MUFU (148 SMs x 16 ex2/clk x max clock)
     mufu_peak = 148 * 16 * SM_MAX_MHZ * 1e6 / 1e9  # Gpair/s
+    n_tiles = (N + 127) // 128
+    fwd_ex2 = B * H * (n_tiles * (n_tiles + 1) // 2) * 128 * 128
     nw_rate = NW_M * NW_S / (kernel_ms[3] * 1e-3) / 1e9 if kernel_ms[3] else None
     fwd_rate = fwd_fl / (kernel_ms[1] * 1e-3) / 1e12 if kernel_ms[1] else None
     rooflines = {
         "attn_fwd": {"bound": "tensor", "achieved": fwd_rate, "peak": pk["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": fwd_rate / pk["bf16_tflops"] if fwd_rate else None,
-                     "traffic": recorded_traffic(1)},
+                     "traffic": recorded_traffic(1),
+                     # the forward's actual limit: one MUFU ex2 per element of every causal
+                     # 128 x 128 tile it visits, against 148 SMs x 16 ex2/clk x max clock
+                     "mufu_frac": (fwd_ex2 / (kernel_ms[1] * 1e-3) / (mufu_peak * 1e9)
+                                   if kernel_ms[1] else None)},
         "nw_regrid": {"bound": "alu", "achieved": nw_rate, "peak": mufu_peak, "unit": "Gpair/s",
                       "frac": nw_rate / mufu_peak if nw_rate else None,
                       "traffic": recorded_traffic(3),
