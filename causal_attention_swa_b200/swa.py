@@ -107,6 +107,18 @@ def _ptr(t):
     return ctypes.c_void_p(0 if t is None else t.data_ptr())
 
 
+def _require_like(ref, named, what):
+    """The C ABI takes sizes from `ref` only, so every other tensor must have
+    the shape, dtype and device that it implies (checked before any launch)."""
+    for name, t in named.items():
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor")
+        shape, dtype = what(name)
+        if tuple(t.shape) != tuple(shape) or t.dtype != dtype or t.device != ref.device:
+            raise ValueError(f"{name}: expected shape {tuple(shape)}, dtype {dtype} on "
+                             f"{ref.device}; got {tuple(t.shape)}, {t.dtype} on {t.device}")
+
+
 def _require_cuda(*ts):
     for t in ts:
         if not (isinstance(t, torch.Tensor) and t.is_cuda and t.is_contiguous()):
@@ -152,15 +164,18 @@ def _workspace(nbytes: int, device, ws):
 def attn_fwd(q, k, v, causal: bool = True, out=None, lse=None, workspace=None):
     """swa_attn_fwd: q, k, v [B,H,N,64] bf16 or fp32 CUDA tensors ->
     (out [B,H,N,64] same dtype, lse [B,H,N] fp32)."""
-    lib = load_library()
-    _require_cuda(q, k, v)
+    if not isinstance(q, torch.Tensor) or q.dim() != 4:
+        raise ValueError("q must be a [B, H, N, D] tensor")
     B, H, N, D = q.shape
     dt = _dtype_code(q)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    _require_cuda(out, lse)
+    _require_like(q, {"k": k, "v": v, "out": out, "lse": lse},
+                  lambda n: ((B, H, N), torch.float32) if n == "lse" else (q.shape, q.dtype))
+    lib = load_library()
+    _require_cuda(q, k, v, out, lse)
     nbytes = attn_fwd_workspace_size(B, H, N, D, dt)
     ws = _workspace(nbytes, q.device, workspace)
     st = lib.swa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, D,
@@ -172,13 +187,18 @@ def attn_fwd(q, k, v, causal: bool = True, out=None, lse=None, workspace=None):
 def attn_bwd(q, k, v, out, dout, lse, causal: bool = True, dq=None, dk=None, dv=None,
              workspace=None):
     """swa_attn_bwd -> (dq, dk, dv), each [B,H,N,64] of q's dtype."""
-    lib = load_library()
-    _require_cuda(q, k, v, out, dout, lse)
+    if not isinstance(q, torch.Tensor) or q.dim() != 4:
+        raise ValueError("q must be a [B, H, N, D] tensor")
     B, H, N, D = q.shape
     dt = _dtype_code(q)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
+    _require_like(q, {"k": k, "v": v, "out": out, "dout": dout, "lse": lse, "dq": dq, "dk": dk,
+                      "dv": dv},
+                  lambda n: ((B, H, N), torch.float32) if n == "lse" else (q.shape, q.dtype))
+    lib = load_library()
+    _require_cuda(q, k, v, out, dout, lse, dq, dk, dv)
     nbytes = attn_bwd_workspace_size(B, H, N, D, dt)
     ws = _workspace(nbytes, q.device, workspace)
     st = lib.swa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
@@ -190,10 +210,16 @@ def attn_bwd(q, k, v, out, dout, lse, causal: bool = True, dq=None, dk=None, dv=
 
 def nw_regrid(targets, sources, vals, h: float = 0.5, out=None, workspace=None):
     """swa_nw_regrid: targets [M,2], sources [S,2], vals [S] fp32 -> out [M] fp32."""
-    lib = load_library()
-    _require_cuda(targets, sources, vals)
+    if not isinstance(targets, torch.Tensor) or targets.dim() != 2 or \
+            not isinstance(sources, torch.Tensor) or sources.dim() != 2:
+        raise ValueError("targets and sources must be [M, 2] and [S, 2] tensors")
     M, S = targets.shape[0], sources.shape[0]
     out = torch.empty((M,), dtype=torch.float32, device=targets.device) if out is None else out
+    shapes = {"targets": (M, 2), "sources": (S, 2), "vals": (S,), "out": (M,)}
+    _require_like(targets, {"targets": targets, "sources": sources, "vals": vals, "out": out},
+                  lambda n: (shapes[n], torch.float32))
+    lib = load_library()
+    _require_cuda(targets, sources, vals, out)
     nbytes = nw_workspace_size(M, S)
     ws = _workspace(nbytes, targets.device, workspace)
     st = lib.swa_nw_regrid(_ptr(targets), M, _ptr(sources), _ptr(vals), S, float(h), _ptr(out),

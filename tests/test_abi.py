@@ -110,3 +110,34 @@ def test_product_path_does_not_import_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "swa_oracle" not in text and "liboracle" not in text, f
+
+
+@pytest.mark.parametrize("bad", ["k_shape", "v_dtype", "out_shape", "lse_dtype"])
+def test_binding_rejects_mismatched_tensors_before_any_launch(bad):
+    """The C ABI takes B, H, N, D from q alone; the binding must refuse any
+    other tensor whose shape or dtype disagrees (it would be read out of
+    bounds), before touching the GPU."""
+    import torch
+    q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
+    k, v = q.clone(), q.clone()
+    out, lse = q.clone(), torch.zeros(1, 2, 8, dtype=torch.float32)
+    if bad == "k_shape":
+        k = torch.zeros(1, 2, 7, 64, dtype=torch.bfloat16)
+    elif bad == "v_dtype":
+        v = v.float()
+    elif bad == "out_shape":
+        out = torch.zeros(1, 2, 8, 32, dtype=torch.bfloat16)
+    else:
+        lse = lse.double()
+    with pytest.raises(ValueError, match="expected shape"):
+        swa.attn_fwd(q, k, v, out=out, lse=lse)
+    with pytest.raises(ValueError, match="expected shape"):
+        swa.attn_bwd(q, k, v, out, out, lse)
+
+
+def test_binding_rejects_mismatched_regrid_tensors():
+    import torch
+    t = torch.zeros(5, 2)
+    src = torch.zeros(7, 2)
+    with pytest.raises(ValueError, match="expected shape"):
+        swa.nw_regrid(t, src, torch.zeros(6))
