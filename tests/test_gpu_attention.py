@@ -191,6 +191,14 @@ def test_bf16_forward_backward_b2_h16_n16384():
     heads, rows = sample_rows(np.random.default_rng(1), 32, wl["N"], 48)
     check_forward_sampled(out, lse, q, k, v, heads, rows)
     _backward_sampled(qb, kb, vb, out, lse, dq, dk, dv, n_q=24, n_k=6, tail=256, seed=2)
+    # the heaviest keys too: key 0 and key 129 each collect dk, dv from ~16384 queries
+    o = to_f64(out)
+    N = wl["N"]
+    kh, kr = np.array([7, 7], dtype=np.int64), np.array([0, 129], dtype=np.int64)
+    _, w_dk, w_dv = oracle.attn_bwd_rows(q, k, v, o, np.zeros(0, np.int64),
+                                         np.zeros(0, np.int64), kh, kr, out=o)
+    check_bf16(to_f64(dk).reshape(-1, N, 64)[kh, kr], w_dk, "dk (first keys)")
+    check_bf16(to_f64(dv).reshape(-1, N, 64)[kh, kr], w_dv, "dv (first keys)")
 
 
 @pytest.mark.parametrize("with_inf", [False, True])
