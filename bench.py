@@ -152,7 +152,16 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- CPU oracle
 
-def oracle_sample(head_tokens, nw_targets, seed=SEED):
+def host_threads():
+    """Threads for the oracle: every core this process may run on (torchrun sets
+    OMP_NUM_THREADS=1 for its ranks; the oracle leg runs on rank 0 alone)."""
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except (AttributeError, OSError):
+        return max(1, os.cpu_count() or 1)
+
+
+def oracle_sample(head_tokens, nw_targets, seed=SEED, threads=0):
     """Time the float64 oracle on a bounded sample of the step: one head of
     the attention batch (its first `head_tokens` tokens as a causal problem)
     forward + backward, and `nw_targets` regrid targets against all sources.
@@ -163,9 +172,9 @@ def oracle_sample(head_tokens, nw_targets, seed=SEED):
     q, k, v = (inputs.bf16_to_f64(b) for b in (qb, kb, vb))
     t, s, y = inputs.nw_grid(NW_M, NW_S, NW_SEED)
     t0 = time.perf_counter()
-    out, _ = oracle.attn_fwd(q, k, v)
-    oracle.attn_bwd(q, k, v, out, out=out)
-    oracle.nw_regrid(t[:nw_targets], s, y, h=H_BW)
+    out, _ = oracle.attn_fwd(q, k, v, threads=threads)
+    oracle.attn_bwd(q, k, v, out, out=out, threads=threads)
+    oracle.nw_regrid(t[:nw_targets], s, y, h=H_BW, threads=threads)
     dt = time.perf_counter() - t0
     fwd, bwd = attn_flops(1, 1, head_tokens)
     return dt, fwd + bwd
@@ -176,14 +185,13 @@ def run_reference(args, info):
     from causal_attention_swa_b200 import dist as sdist
     if not info.is_root:
         return 0
-    import oracle
-    threads = oracle.max_threads()
+    threads = host_threads()
     head_tokens, nw_targets = 4096, 128
     for _ in range(args.warmup):
-        oracle_sample(1024, 16)
+        oracle_sample(1024, 16, threads=threads)
     times, flops = [], 0.0
     for _ in range(args.steps):
-        dt, fl = oracle_sample(head_tokens, nw_targets)
+        dt, fl = oracle_sample(head_tokens, nw_targets, threads=threads)
         times.append(dt)
         flops = fl
     mean_s = sum(times) / len(times)
@@ -417,9 +425,9 @@ def run_ours(args, info):
 
     cpu = None
     if info.is_root and info.world == 1 and not args.no_cpu_baseline:
-        import oracle
-        dt, fl = oracle_sample(N, NW_M // 32)
-        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(),
+        threads = host_threads()
+        dt, fl = oracle_sample(N, NW_M // 32, threads=threads)
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads,
                "kind": "oracle",
                "sample": f"1/32 of one step: head 0 of {B * H} ({N} tokens, forward + "
                          f"backward) and {NW_M // 32} of {NW_M} regrid targets; "
