@@ -64,9 +64,12 @@ def _load():
         lib.oracle_attn_bwd_rows.argtypes = [P, P, P, P, P, I64, I64, I, Dbl, P, P, I64, P,
                                              P, P, I64, P, P, I]
         lib.oracle_nw.argtypes = [P, I64, P, P, I64, Dbl, P, I]
+        lib.oracle_nw_nd.argtypes = [P, I64, P, P, I64, I, Dbl, P, P, I]
+        lib.oracle_nw_bwd.argtypes = [P, I64, P, P, I64, I, Dbl, P, P, P, P, I]
         lib.oracle_max_threads.argtypes = []
         for f in (lib.oracle_attn_fwd, lib.oracle_attn_fwd_rows, lib.oracle_attn_bwd,
-                  lib.oracle_attn_bwd_rows, lib.oracle_nw, lib.oracle_max_threads):
+                  lib.oracle_attn_bwd_rows, lib.oracle_nw, lib.oracle_nw_nd,
+                  lib.oracle_nw_bwd, lib.oracle_max_threads):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -187,3 +190,47 @@ def nw_regrid(targets, sources, vals, h: float = 0.5, threads: int = 0):
                            _ptr(out), int(threads))
     _check(rc, False)
     return out
+
+
+def nw_regrid_nd(targets, sources, vals, h: float = 0.5, threads: int = 0, with_z=False):
+    """Regrid with points of 1, 2 or 3 coordinates: targets [M, d], sources
+    [S, d], vals [S] -> out [M] (and Z [M] = sum of weights if with_z)."""
+    targets, sources, vals = _f64(targets), _f64(sources), _f64(vals)
+    M, dims = targets.shape
+    S = sources.shape[0]
+    assert sources.shape[1] == dims
+    out = np.empty((M,), dtype=np.float64)
+    z = np.empty((M,), dtype=np.float64)
+    rc = _load().oracle_nw_nd(_ptr(targets), M, _ptr(sources), _ptr(vals), S, dims, float(h),
+                              _ptr(out), _ptr(z), int(threads))
+    _check(rc, False)
+    return (out, z) if with_z else out
+
+
+def nw_regrid_bwd(targets, sources, vals, gout, h: float = 0.5, threads: int = 0):
+    """Gradient of a loss with dL/dout = gout [M] with respect to targets
+    [M, d], sources [S, d] and vals [S]: returns (dtargets, dsources, dvals)."""
+    targets, sources, vals, gout = _f64(targets), _f64(sources), _f64(vals), _f64(gout)
+    M, dims = targets.shape
+    S = sources.shape[0]
+    dt, ds = np.empty_like(targets), np.empty_like(sources)
+    dv = np.empty((S,), dtype=np.float64)
+    rc = _load().oracle_nw_bwd(_ptr(targets), M, _ptr(sources), _ptr(vals), S, dims, float(h),
+                               _ptr(gout), _ptr(dt), _ptr(ds), _ptr(dv), int(threads))
+    _check(rc, False)
+    return dt, ds, dv
+
+
+def qkv_proj(x, w, H: int, D: int = 64):
+    """Fused QKV projection in front of attention ("Wiki notes", page 5,
+    mini_attention: Q = x Wq, K = x Wk, V = x Wv), float64.  x [B, N, C];
+    w [3 H D, C] stacks the output features of Wq, Wk, Wv, one row per
+    feature (q feature h*D + d is row h*D + d, k's rows follow, then v's).
+    Returns q, k, v as [B, H, N, D].  One library matmul, then the head split
+    (no blocking or fusion)."""
+    x, w = _f64(x), _f64(w)
+    B, N, C = x.shape
+    assert w.shape == (3 * H * D, C)
+    y = x.reshape(B * N, C) @ w.T                     # [B*N, 3 H D]
+    y = y.reshape(B, N, 3, H, D).transpose(2, 0, 3, 1, 4)
+    return tuple(np.ascontiguousarray(y[i]) for i in range(3))

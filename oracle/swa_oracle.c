@@ -408,6 +408,115 @@ int oracle_nw(const double* targets, int64_t M, const double* sources,
     return OR_OK;
 }
 
+/*
+ * Nadaraya-Watson regrid with points of `dims` coordinates (1, 2 or 3):
+ * the NADARAYA_WATSON query's weight with the squared distance summed over
+ * every coordinate (the pages' points are (x, y); a point table with more
+ * coordinate columns gives the same view with more terms):
+ *   w_pq  = exp(-sum_c (t_pc - s_qc)^2 / h^2)
+ *   Z_p   = sum_q w_pq
+ *   out_p = (sum_q w_pq v_q) / Z_p
+ * targets [M, dims], sources [S, dims]; z_out (may be NULL) receives Z_p.
+ */
+static void nw_row(const double* tp, const double* sources, const double* vals, int64_t S,
+                   int dims, double h2, double* z, double* o) {
+    double sw = 0.0, swv = 0.0;
+    for (int64_t q = 0; q < S; ++q) {
+        double d2 = 0.0;
+        for (int c = 0; c < dims; ++c) {
+            double d = tp[c] - sources[q * dims + c];
+            d2 += d * d;
+        }
+        double w = exp(-d2 / h2);
+        sw += w;
+        swv += w * vals[q];
+    }
+    *z = sw;
+    *o = swv / sw;
+}
+
+int oracle_nw_nd(const double* targets, int64_t M, const double* sources, const double* vals,
+                 int64_t S, int dims, double h, double* out, double* z_out, int nthreads) {
+    if (!targets || !sources || !vals || !out || M < 0 || S < 0 || dims < 1 || dims > 3 ||
+        !(h > 0.0))
+        return OR_EINVAL;
+    set_threads(nthreads);
+    double h2 = h * h;
+#pragma omp parallel for schedule(static)
+    for (int64_t p = 0; p < M; ++p) {
+        double z;
+        nw_row(targets + p * dims, sources, vals, S, dims, h2, &z, out + p);
+        if (z_out) z_out[p] = z;
+    }
+    return OR_OK;
+}
+
+/*
+ * Backward of the regrid for an upstream gradient g_p = dL/dout_p,
+ * hand-derived from the definition above (every sum over all pairs):
+ *   P_pq  = w_pq / Z_p                       (so out_p = sum_q P_pq v_q)
+ *   dv_q  = sum_p g_p P_pq
+ *   dw_pq = g_p (v_q - out_p) / Z_p          (dL/dw_pq through Z_p and the sum)
+ *   dw_pq/dt_p = w_pq (-2 / h^2) (t_p - s_q),  dw_pq/ds_q = -dw_pq/dt_p
+ *   dt_p  = sum_q dw_pq w_pq (-2 / h^2) (t_p - s_q)
+ *   ds_q  = sum_p dw_pq w_pq (+2 / h^2) (t_p - s_q)
+ * Phase 1 (per target): Z_p, out_p and dt_p.  Phase 2 (per source): ds_q and
+ * dv_q from every target's (Z_p, out_p).  dtargets [M, dims], dsources
+ * [S, dims], dvals [S].
+ */
+int oracle_nw_bwd(const double* targets, int64_t M, const double* sources, const double* vals,
+                  int64_t S, int dims, double h, const double* gout, double* dtargets,
+                  double* dsources, double* dvals, int nthreads) {
+    if (!targets || !sources || !vals || !gout || !dtargets || !dsources || !dvals || M < 0 ||
+        S < 0 || dims < 1 || dims > 3 || !(h > 0.0))
+        return OR_EINVAL;
+    set_threads(nthreads);
+    double h2 = h * h;
+    double* zo = (double*)malloc(sizeof(double) * (size_t)(2 * (M > 0 ? M : 1)));
+    if (!zo) return OR_ENOMEM;
+#pragma omp parallel for schedule(static)
+    for (int64_t p = 0; p < M; ++p) {
+        const double* tp = targets + p * dims;
+        double z, o;
+        nw_row(tp, sources, vals, S, dims, h2, &z, &o);
+        zo[2 * p] = z;
+        zo[2 * p + 1] = o;
+        double acc[3] = {0.0, 0.0, 0.0};
+        for (int64_t q = 0; q < S; ++q) {
+            double d2 = 0.0, diff[3];
+            for (int c = 0; c < dims; ++c) {
+                diff[c] = tp[c] - sources[q * dims + c];
+                d2 += diff[c] * diff[c];
+            }
+            double w = exp(-d2 / h2);
+            double dw = gout[p] * (vals[q] - o) / z;
+            for (int c = 0; c < dims; ++c) acc[c] += dw * w * (-2.0 / h2) * diff[c];
+        }
+        for (int c = 0; c < dims; ++c) dtargets[p * dims + c] = acc[c];
+    }
+#pragma omp parallel for schedule(static)
+    for (int64_t q = 0; q < S; ++q) {
+        const double* sq = sources + q * dims;
+        double acc[3] = {0.0, 0.0, 0.0}, dv = 0.0;
+        for (int64_t p = 0; p < M; ++p) {
+            double d2 = 0.0, diff[3];
+            for (int c = 0; c < dims; ++c) {
+                diff[c] = targets[p * dims + c] - sq[c];
+                d2 += diff[c] * diff[c];
+            }
+            double w = exp(-d2 / h2);
+            double z = zo[2 * p], o = zo[2 * p + 1];
+            dv += gout[p] * w / z;
+            double dw = gout[p] * (vals[q] - o) / z;
+            for (int c = 0; c < dims; ++c) acc[c] += dw * w * (2.0 / h2) * diff[c];
+        }
+        for (int c = 0; c < dims; ++c) dsources[q * dims + c] = acc[c];
+        dvals[q] = dv;
+    }
+    free(zo);
+    return OR_OK;
+}
+
 int oracle_max_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

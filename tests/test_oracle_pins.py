@@ -380,3 +380,123 @@ def test_delta_on_a_given_output_moves_gradients_by_the_closed_form():
         want_dk = -(P.T @ (delta[:, None] * q[0, 0])) / 8.0
         assert np.abs((dq1 - dq0)[0, 0] - want_dq).max() < 1e-12
         assert np.abs((dk1 - dk0)[0, 0] - want_dk).max() < 1e-12
+
+
+# ------------------------------------------------- regrid in 1-3 dimensions
+
+def _nw_points(seed, M, S, dims, lo=0.0, hi=1.5):
+    rng = np.random.default_rng(seed)
+    return (rng.uniform(lo, hi, size=(M, dims)), rng.uniform(lo, hi, size=(S, dims)),
+            rng.normal(size=S), rng.normal(size=M))
+
+
+def test_nw_nd_two_dims_is_the_pages_regrid():
+    """In two dimensions the generalised regrid is the NADARAYA_WATSON view
+    itself (the demo's numpy check's inputs)."""
+    t, s, y = inputs.pages_nw()
+    assert np.abs(oracle.nw_regrid_nd(t, s, y, h=0.5) - oracle.nw_regrid(t, s, y, h=0.5)).max() \
+        < 1e-15
+
+
+def test_nw_nd_zero_coordinates_reduce_the_dimension():
+    """A coordinate that is 0 for every point adds 0 to every squared
+    distance: 3-D with z = 0 gives the 2-D result, 2-D with y = 0 the 1-D."""
+    t, s, y, _ = _nw_points(21, 9, 13, 2)
+    pad = lambda a: np.concatenate([a, np.zeros((a.shape[0], 1))], axis=1)  # noqa: E731
+    assert np.abs(oracle.nw_regrid_nd(pad(t), pad(s), y) - oracle.nw_regrid_nd(t, s, y)).max() \
+        < 1e-15
+    assert np.abs(oracle.nw_regrid_nd(pad(t[:, :1]), pad(s[:, :1]), y)
+                  - oracle.nw_regrid_nd(t[:, :1], s[:, :1], y)).max() < 1e-15
+
+
+def test_nw_nd_closed_forms():
+    """3-D: a source at squared distance h^2 weighs exp(-1) against a
+    coincident one; one source gives out = v everywhere."""
+    s = np.array([[0.0, 0.0, 0.0], [0.3, 0.4, 0.0]])    # |s1 - s0| = 0.5 = h
+    vals = np.array([1.0, 4.0])
+    got = oracle.nw_regrid_nd(np.zeros((1, 3)), s, vals, h=0.5)
+    e = math.exp(-1.0)
+    assert abs(got[0] - (1.0 + 4.0 * e) / (1.0 + e)) < 1e-15
+    t = np.random.default_rng(3).uniform(-1, 1, size=(7, 3))
+    assert np.all(oracle.nw_regrid_nd(t, s[:1], vals[:1]) == 1.0)
+
+
+@pytest.mark.parametrize("dims", [1, 2, 3])
+def test_nw_backward_matches_central_differences(dims):
+    """L = sum_p g_p out_p: dL/dtargets, dL/dsources and dL/dvals against
+    central differences of the forward (relative error <= 1e-6)."""
+    t, s, y, g = _nw_points(30 + dims, 5, 7, dims)
+    h = 0.7
+    dt, ds, dv = oracle.nw_regrid_bwd(t, s, y, g, h=h)
+
+    def loss(t_, s_, y_):
+        return float(np.dot(g, oracle.nw_regrid_nd(t_, s_, y_, h=h)))
+
+    eps = 1e-6
+    for arr, grad, which in ((t, dt, 0), (s, ds, 1), (y, dv, 2)):
+        fd = np.zeros_like(arr)
+        flat, fflat = arr.reshape(-1), fd.reshape(-1)
+        for i in range(flat.size):
+            old = flat[i]
+            args = [t, s, y]
+            flat[i] = old + eps
+            lp = loss(*args)
+            flat[i] = old - eps
+            lm = loss(*args)
+            flat[i] = old
+            fflat[i] = (lp - lm) / (2 * eps)
+        err = np.abs(grad - fd).max() / max(np.abs(fd).max(), 1e-12)
+        assert err <= 1e-6, (which, err)
+
+
+def test_nw_backward_invariants_and_closed_forms():
+    """Shifting every point by one vector leaves out unchanged, so the
+    position gradients sum to zero; sum_q dv_q = sum_p g_p (each row of P
+    sums to 1); one source: out = v for every target, so the position
+    gradients vanish and dv = sum_p g_p; constant values likewise."""
+    t, s, y, g = _nw_points(40, 11, 17, 3)
+    dt, ds, dv = oracle.nw_regrid_bwd(t, s, y, g, h=0.6)
+    tot = dt.sum(axis=0) + ds.sum(axis=0)
+    assert np.abs(tot).max() < 1e-12 * (np.abs(dt).max() + np.abs(ds).max())
+    assert abs(dv.sum() - g.sum()) < 1e-12 * np.abs(g).sum()
+    dt1, ds1, dv1 = oracle.nw_regrid_bwd(t, s[:1], y[:1], g, h=0.6)
+    # out = (w v) / w is v up to one rounding, so v - out is 0 or one ulp of v
+    assert np.abs(dt1).max() < 1e-14 and np.abs(ds1).max() < 1e-14
+    assert abs(dv1[0] - g.sum()) < 1e-13
+    dtc, dsc, _ = oracle.nw_regrid_bwd(t, s, np.full(17, 0.25), g, h=0.6)
+    assert np.abs(dtc).max() < 1e-15 and np.abs(dsc).max() < 1e-15
+
+
+# ------------------------------------------------------- QKV projection
+
+def test_qkv_projection_brute_force():
+    """q[b,h,n,d] = sum_c x[b,n,c] w[h D + d, c], k and v from the next row
+    blocks: against a plain triple loop on a tiny case."""
+    rng = np.random.default_rng(50)
+    B, N, C, H, D = 2, 3, 5, 2, 3
+    x = rng.normal(size=(B, N, C))
+    w = rng.normal(size=(3 * H * D, C))
+    q, k, v = oracle.qkv_proj(x, w, H, D)
+    for which, t in enumerate((q, k, v)):
+        for b in range(B):
+            for h in range(H):
+                for n in range(N):
+                    for d in range(D):
+                        want = sum(x[b, n, c] * w[which * H * D + h * D + d, c] for c in range(C))
+                        assert abs(t[b, h, n, d] - want) < 1e-13
+
+
+def test_qkv_projection_is_mini_attentions_x_times_w():
+    """Page 5's mini_attention (seq 4, d_model 8, d_k = d_v = 4): with the
+    rows of w taken from the columns of Wq, Wk, Wv (one head), the projection
+    gives x Wq, x Wk, x Wv; selecting rows of the identity picks features."""
+    rng = np.random.default_rng(5)
+    x = rng.normal(size=(4, 8))
+    wq, wk, wv = (rng.normal(size=(8, 4)) for _ in range(3))
+    q, k, v = oracle.qkv_proj(x[None], np.concatenate([wq.T, wk.T, wv.T]), 1, 4)
+    for got, wm in ((q, wq), (k, wk), (v, wv)):
+        assert np.abs(got[0, 0] - x @ wm).max() < 1e-14
+    eye = np.eye(8)[[0, 1, 2, 3, 4, 5, 6, 7, 0, 1, 2, 3]]   # q, k: features 0-3, 4-7; v: 0-3
+    q, k, v = oracle.qkv_proj(x[None], eye, 1, 4)
+    assert np.array_equal(q[0, 0], x[:, :4]) and np.array_equal(k[0, 0], x[:, 4:])
+    assert np.array_equal(v[0, 0], x[:, :4])
