@@ -2,20 +2,25 @@
 """Benchmark of the fused softmax-weighted average on B200.
 
 One step = one pass of the whole hot path over one batch of synthetic input:
-  * causal attention forward (bf16, B=2 H=16 N=16384 D=64, scale 1/8):
-    out and lse;
-  * its backward for loss = 1/2 sum out^2 (dout = out): dq, dk, dv;
+  * the GRADIENT query (swa_attn_grad): causal attention forward (bf16,
+    B=2 H=16 N=16384 D=64, scale 1/8) -- out and lse -- and the gradient of
+    loss = 1/2 sum out^2 with respect to q, k, v;
   * the Nadaraya-Watson regrid (fp32, 16384 targets x 16384 sources in
     [0,10]^2, h = 0.5).
+The other workloads (the 4x16x4096 forward, the 1x8x65536 forward + gradient
+with and without 0.01% of V set to +inf, the float32 256-token call) are
+timed after the step, each beside a bounded oracle sample, under "configs".
 The metric is attention TFLOP/s with FLOPs counted causally (N(N+1)/2 pairs
 per head; forward 4*D per pair, backward 2.5x forward), over the whole
 step's device time.  Inputs (201 MB of Q, K, V) exceed the 126 MB L2.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-N > 1: launched by torchrun, one process per GPU; each rank runs its own
-seeded replica of the batch (weak scaling, no collective in the data path);
-the elapsed time is the max over ranks.  --impl reference times the float64
+N > 1: launched by torchrun, one process per GPU; the problem is one batch
+of B*N sequences (and N blocks of regrid targets), split across the ranks by
+sequences -- rank r computes sequences [rB, rB+B), its heads -- with no
+collective in the data path (weak scaling: per-rank work fixed); the
+elapsed time is the max over ranks.  --impl reference times the float64
 CPU oracle on the host cores instead (rank 0 only).
 """
 from __future__ import annotations
@@ -42,6 +47,7 @@ NW_SEED = 2
 H_BW = 0.5
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 SM_MAX_MHZ = 1965.0
+MUFU_GPAIRS = 148 * 16 * SM_MAX_MHZ * 1e6 / 1e9  # one ex2 per pair, Gpair/s
 
 # kernel id -> (name, source file whose hash keys the recorded ncu traffic)
 KERNELS = {
@@ -219,6 +225,217 @@ def run_reference(args, info):
 
 # ----------------------------------------------------------------- our arm
 
+def timed_grad(swa, q, k, v, causal, stream, device, ws, reps=5, warm=2):
+    """Median of (reps - warm) gradient calls: whole-call, forward-kernel and
+    backward-kernel times (CUDA events, the library's profiling hook)."""
+    import torch
+    out, lse = torch.empty_like(q), torch.empty(q.shape[:3], dtype=torch.float32, device=device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    rows = []
+    for rep in range(reps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        for e in ev:
+            e.record(stream)
+        ev[0].record(stream)
+        swa.profile_kernel(swa.SWA_KERNEL_ATTN_FWD, ev[2], ev[3])
+        swa.attn_grad(q, k, v, causal=causal, out=out, lse=lse, dq=dq, dk=dk, dv=dv,
+                      workspace=ws)
+        ev[1].record(stream)
+        swa.profile_kernel(swa.SWA_KERNEL_ATTN_BWD, ev[4], ev[5])
+        swa.attn_grad(q, k, v, causal=causal, out=out, lse=lse, dq=dq, dk=dk, dv=dv,
+                      workspace=ws)
+        swa.profile_kernel(swa.SWA_KERNEL_NONE)
+        torch.cuda.synchronize(device)
+        if rep >= warm:
+            rows.append((ev[0].elapsed_time(ev[1]), ev[2].elapsed_time(ev[3]),
+                         ev[4].elapsed_time(ev[5])))
+    if swa.get_device_error(device) != swa.SWA_OK:
+        raise RuntimeError("device error word set during the gradient calls")
+    med = lambda i: statistics.median(r[i] for r in rows)  # noqa: E731
+    return {"call_ms": med(0), "fwd_ms": med(1), "bwd_ms": med(2)}
+
+
+def timed_call(fn, stream, device, reps=7, warm=2):
+    import torch
+    ts = []
+    for rep in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        if rep >= warm:
+            ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def oracle_attn_rate(qb, kb, vb, heads, tokens, backward, threads, v_f64=None):
+    """Oracle TFLOP/s (causal count) on heads[...]'s first `tokens` tokens."""
+    import oracle
+    from causal_attention_swa_b200 import inputs
+    q, k, v = (inputs.bf16_to_f64(b[:, :, :tokens]) for b in (qb, kb, vb))
+    B_, H_ = qb.shape[:2]
+    q, k, v = (a.reshape(B_ * H_, 1, tokens, 64)[heads] for a in (q, k, v))
+    t0 = time.perf_counter()
+    out, _ = oracle.attn_fwd(q, k, v, threads=threads, allow_underflow=True)
+    if backward:
+        oracle.attn_bwd(q, k, v, out, threads=threads, allow_underflow=True)
+    dt = time.perf_counter() - t0
+    fwd, bwd = attn_flops(len(heads), 1, tokens)
+    return (fwd + (bwd if backward else 0)) / dt / 1e12, dt
+
+
+def other_configs(swa, inputs, torch, stream, device, pk, info, cpu):
+    """The workloads besides the step's: each timed on the GPU with its
+    roofline fraction, and (rank 0, one GPU) the oracle on a bounded sample."""
+    peak = pk["bf16_tflops"]
+    threads = host_threads()
+    res = {}
+
+    def dev16(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(device)
+
+    # 4x16x4096 causal forward (out + lse)
+    wl = inputs.WORKLOADS["attn_fwd_b4h16n4096"]
+    qb, kb, vb, _ = inputs.attn_bf16(**wl)
+    q, k, v = dev16(qb), dev16(kb), dev16(vb)
+    ws = torch.empty(max(swa.attn_fwd_workspace_size(wl["B"], wl["H"], wl["N"], D, swa.SWA_BF16),
+                         16), dtype=torch.uint8, device=device)
+    o, l = torch.empty_like(q), torch.empty(q.shape[:3], dtype=torch.float32, device=device)
+    ms = timed_call(lambda: swa.attn_fwd(q, k, v, out=o, lse=l, workspace=ws), stream, device)
+    fl, _ = attn_flops(wl["B"], wl["H"], wl["N"])
+    entry = {"workload": "causal attention forward B=4 H=16 N=4096 D=64 bf16 (out + lse)",
+             "ms": ms, "tflops": fl / (ms * 1e-3) / 1e12,
+             "frac": fl / (ms * 1e-3) / 1e12 / peak, "bound": "tensor",
+             "timing": "median of 5 calls after 2 warm-up calls (V scan + kernel), CUDA events; "
+                       "inputs 101 MB (< L2, not flushed)"}
+    if cpu:
+        rate, dt = oracle_attn_rate(qb, kb, vb, [0, 1], wl["N"], False, threads)
+        entry["cpu_baseline"] = {"value": rate, "unit": "TFLOP/s", "cores": threads,
+                                 "kind": "oracle", "sample": f"2 of 64 heads, forward; {dt:.1f} s"}
+    res["fwd_b4h16n4096"] = entry
+    del q, k, v, o, l, ws
+
+    # 1x8x65536 forward + gradient, without and with 0.01% +inf in V
+    wl = inputs.WORKLOADS["attn_fwdbwd_b1h8n65536"]
+    for with_inf in (False, True):
+        qb, kb, vb, _ = inputs.attn_bf16(**wl, n_inf=inputs.LONG_CONTEXT_N_INF if with_inf else 0)
+        q, k, v = dev16(qb), dev16(kb), dev16(vb)
+        ws = torch.empty(swa.attn_grad_workspace_size(wl["B"], wl["H"], wl["N"], D, swa.SWA_BF16),
+                         dtype=torch.uint8, device=device)
+        t = timed_grad(swa, q, k, v, True, stream, device, ws)
+        fwd, bwd = attn_flops(wl["B"], wl["H"], wl["N"])
+        entry = {"workload": "causal attention forward + gradient B=1 H=8 N=65536 D=64 bf16, "
+                             "Q, K ~ N(0, 0.5^2)" + (", 3355 V entries +inf" if with_inf else ""),
+                 "call_ms": t["call_ms"], "fwd_ms": t["fwd_ms"], "bwd_ms": t["bwd_ms"],
+                 "tflops": (fwd + bwd) / (t["call_ms"] * 1e-3) / 1e12,
+                 "fwd_tflops": fwd / (t["fwd_ms"] * 1e-3) / 1e12,
+                 "bwd_tflops": bwd / (t["bwd_ms"] * 1e-3) / 1e12,
+                 "fwd_frac": fwd / (t["fwd_ms"] * 1e-3) / 1e12 / peak,
+                 "bwd_frac": bwd / (t["bwd_ms"] * 1e-3) / 1e12 / peak, "bound": "tensor",
+                 "timing": "median of 3 gradient calls after 2 warm-up calls, CUDA events"}
+        if cpu:
+            rate, dt = oracle_attn_rate(qb, kb, vb, [0], 8192, True, threads)
+            entry["cpu_baseline"] = {"value": rate, "unit": "TFLOP/s", "cores": threads,
+                                     "kind": "oracle",
+                                     "sample": f"head 0, first 8192 tokens, forward + gradient; "
+                                               f"{dt:.1f} s"}
+        res["fwdbwd_b1h8n65536" + ("_inf" if with_inf else "")] = entry
+        del q, k, v, ws
+
+    # float32, one head of 256 tokens (the demo's size): latency of the
+    # forward + gradient call on CUDA cores
+    q64, k64, v64 = inputs.single_head_f64(256)
+    q, k, v = (torch.from_numpy(a.astype(np.float32)).to(device) for a in (q64, k64, v64))
+    ws = torch.empty(swa.attn_grad_workspace_size(1, 1, 256, D, swa.SWA_F32), dtype=torch.uint8,
+                     device=device)
+    o, l = torch.empty_like(q), torch.empty((1, 1, 256), dtype=torch.float32, device=device)
+    g = [torch.empty_like(q) for _ in range(3)]
+    ms = timed_call(lambda: swa.attn_grad(q, k, v, out=o, lse=l, dq=g[0], dk=g[1], dv=g[2],
+                                          workspace=ws), stream, device, reps=22)
+    fwd, bwd = attn_flops(1, 1, 256)
+    entry = {"workload": "causal attention forward + gradient B=1 H=1 N=256 D=64 float32 "
+                         "(CUDA cores)",
+             "us": ms * 1e3, "tflops": (fwd + bwd) / (ms * 1e-3) / 1e12, "bound": "latency",
+             "timing": "median of 20 calls after 2 warm-up calls, CUDA events"}
+    if cpu:
+        import oracle
+        ts = []
+        for _ in range(5):
+            t0 = time.perf_counter()
+            out, _ = oracle.attn_fwd(q64, k64, v64, threads=threads)
+            oracle.attn_bwd(q64, k64, v64, out, threads=threads)
+            ts.append(time.perf_counter() - t0)
+        entry["cpu_baseline"] = {"value": statistics.median(ts) * 1e6, "unit": "us",
+                                 "cores": threads, "kind": "oracle",
+                                 "sample": "the whole call, median of 5"}
+    res["f32_b1h1n256"] = entry
+
+    # the regrid generalised: 3-D points, and the gradient (2-D, loss 1/2 sum out^2)
+    t3, s3, v3 = (torch.from_numpy(a).to(device) for a in inputs.nw_grid_nd(NW_M, NW_S, 3))
+    ms = timed_call(lambda: swa.nw_regrid_nd(t3, s3, v3, h=H_BW), stream, device)
+    rate = NW_M * NW_S / (ms * 1e-3) / 1e9
+    entry = {"workload": f"Nadaraya-Watson regrid, 3-D points, {NW_M}x{NW_S} fp32 h={H_BW}",
+             "ms": ms, "gpairs_per_s": rate, "points_per_s": NW_M / (ms * 1e-3),
+             "frac": rate / MUFU_GPAIRS, "bound": "alu (MUFU: one ex2 per pair)",
+             "timing": "median of 5 calls after 2 warm-up calls (both kernels)"}
+    if cpu:
+        import oracle
+        tn, sn, vn = inputs.nw_grid_nd(NW_M, NW_S, 3)
+        t0 = time.perf_counter()
+        oracle.nw_regrid_nd(tn[:512], sn, vn, h=H_BW, threads=threads)
+        dt = time.perf_counter() - t0
+        entry["cpu_baseline"] = {"value": 512 * NW_S / dt / 1e9, "unit": "Gpair/s",
+                                 "cores": threads, "kind": "oracle",
+                                 "sample": f"512 of {NW_M} targets; {dt:.1f} s"}
+    res["nw3d_16384"] = entry
+    t2, s2, v2 = (torch.from_numpy(a).to(device) for a in inputs.nw_grid(NW_M, NW_S, NW_SEED))
+    g2 = swa.nw_regrid(t2, s2, v2, h=H_BW)
+    ms = timed_call(lambda: swa.nw_regrid_bwd(t2, s2, v2, g2, h=H_BW), stream, device)
+    rate = 2 * NW_M * NW_S / (ms * 1e-3) / 1e9
+    entry = {"workload": f"Nadaraya-Watson regrid gradient (targets, sources, values), 2-D, "
+                         f"{NW_M}x{NW_S} fp32, gout = out",
+             "ms": ms, "gpairs_per_s": rate, "frac": rate / MUFU_GPAIRS,
+             "bound": "alu (MUFU: one ex2 per pair in each of the two passes)",
+             "timing": "median of 5 calls after 2 warm-up calls (all four kernels)"}
+    if cpu:
+        import oracle
+        tn, sn, vn = inputs.nw_grid(NW_M, NW_S, NW_SEED)
+        sub_t, sub_s = tn[:1024], sn[:1024]
+        t0 = time.perf_counter()
+        oracle.nw_regrid_bwd(sub_t, sub_s, vn[:1024], np.ones(1024), h=H_BW, threads=threads)
+        dt = time.perf_counter() - t0
+        entry["cpu_baseline"] = {"value": 2 * 1024 * 1024 / dt / 1e9, "unit": "Gpair/s",
+                                 "cores": threads, "kind": "oracle",
+                                 "sample": f"1024 targets x 1024 sources; {dt:.2f} s"}
+    res["nw_grad_16384"] = entry
+    del t3, s3, v3, t2, s2, v2, g2
+
+    # the QKV projection at the step's shape (x [2*16384, 1024], w [3072, 1024])
+    Cq = H * D
+    xb, wb = inputs.qkv_inputs(B, N, Cq, H, seed=6)
+    x, w = dev16(xb), dev16(wb)
+    qo, ko, vo = (torch.empty((B, H, N, D), dtype=torch.bfloat16, device=device) for _ in range(3))
+    ms = timed_call(lambda: swa.qkv_proj(x, w, H, q=qo, k=ko, v=vo), stream, device)
+    fl = 2.0 * B * N * Cq * 3 * Cq
+    entry = {"workload": f"QKV projection B={B} N={N} C={Cq} H={H} bf16 (x w^T into [B,H,N,64])",
+             "ms": ms, "tflops": fl / (ms * 1e-3) / 1e12, "frac": fl / (ms * 1e-3) / 1e12 / peak,
+             "bound": "tensor", "timing": "median of 5 calls after 2 warm-up calls"}
+    if cpu:
+        import oracle
+        xs = inputs.bf16_to_f64(xb[:, :512])
+        t0 = time.perf_counter()
+        oracle.qkv_proj(xs, inputs.bf16_to_f64(wb), H)
+        dt = time.perf_counter() - t0
+        entry["cpu_baseline"] = {"value": 2.0 * B * 512 * Cq * 3 * Cq / dt / 1e12,
+                                 "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                 "sample": f"512 of {N} tokens per sequence; {dt:.2f} s"}
+    res["qkv_proj_b2n16384c1024"] = entry
+    del x, w, qo, ko, vo
+    if swa.get_device_error(device) != swa.SWA_OK:
+        raise RuntimeError("device error word set during the other workloads")
+    return res
+
 def run_ours(args, info):
     import torch
     from causal_attention_swa_b200 import dist as sdist
@@ -230,9 +447,13 @@ def run_ours(args, info):
     sdist.init("nccl", info)
     swa.load_library()
 
-    seed = sdist.replica_seed(SEED, info.rank)
-    qb, kb, vb, _ = inputs.attn_bf16(B, H, N, seed=seed)
-    nt, ns, ny = inputs.nw_grid(NW_M, NW_S, sdist.replica_seed(NW_SEED, info.rank))
+    # this rank's block of one global problem: sequences [rank*B, rank*B + B)
+    # of a batch of B*world (every sequence drawn from its own seed) and
+    # target block `rank` against the shared source set
+    qb, kb, vb = inputs.attn_bf16_batch(B, H, N, seed=SEED,
+                                        first=sdist.sequence_block(B, info.rank))
+    _, ns, ny = inputs.nw_grid(NW_M, NW_S, NW_SEED)
+    nt = inputs.nw_targets_block(NW_M, info.rank, NW_SEED)
 
     def bf16_host(bits):
         return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
@@ -246,9 +467,7 @@ def run_ours(args, info):
     lse = torch.empty((B, H, N), dtype=torch.float32, device=device)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
     nw_out = torch.empty((NW_M,), dtype=torch.float32, device=device)
-    ws_f = torch.empty(max(swa.attn_fwd_workspace_size(B, H, N, D, swa.SWA_BF16), 16),
-                       dtype=torch.uint8, device=device)
-    ws_b = torch.empty(swa.attn_bwd_workspace_size(B, H, N, D, swa.SWA_BF16),
+    ws_g = torch.empty(swa.attn_grad_workspace_size(B, H, N, D, swa.SWA_BF16),
                        dtype=torch.uint8, device=device)
     ws_n = torch.empty(swa.nw_workspace_size(NW_M, NW_S), dtype=torch.uint8, device=device)
     launches = [0]
@@ -257,11 +476,8 @@ def run_ours(args, info):
 
     def step(src, dst=None):
         d = main_out if dst is None else dst
-        swa.attn_fwd(src["q"], src["k"], src["v"], causal=True, out=d["out"], lse=d["lse"],
-                     workspace=ws_f)
-        launches[0] += swa.last_launch_count()
-        swa.attn_bwd(src["q"], src["k"], src["v"], d["out"], d["out"], d["lse"], causal=True,
-                     dq=d["dq"], dk=d["dk"], dv=d["dv"], workspace=ws_b)
+        swa.attn_grad(src["q"], src["k"], src["v"], causal=True, out=d["out"], lse=d["lse"],
+                      dq=d["dq"], dk=d["dk"], dv=d["dv"], workspace=ws_g)
         launches[0] += swa.last_launch_count()
         swa.nw_regrid(src["nt"], src["ns"], src["ny"], h=H_BW, out=d["nw"], workspace=ws_n)
         launches[0] += swa.last_launch_count()
@@ -356,31 +572,20 @@ def run_ours(args, info):
     e2e_value = (fwd_fl + bwd_fl) * info.world / (e2e_ms * 1e-3) / 1e12
 
     # ---- the first widening row: non-causal attention (every pair, the same
-    # kernels without tile skipping), timed per API call after the step's
-    # measurements (its calls include the small scan and prep kernels)
-    nc_fwd, nc_bwd = [], []
-    for rep in range(5):
-        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-        e0.record(stream)
-        swa.attn_fwd(q, k, v, causal=False, out=out, lse=lse, workspace=ws_f)
-        e1.record(stream)
-        swa.attn_bwd(q, k, v, out, out, lse, causal=False, dq=dq, dk=dk, dv=dv, workspace=ws_b)
-        e2.record(stream)
-        torch.cuda.synchronize(device)
-        if rep >= 2:  # two warm-up calls
-            nc_fwd.append(e0.elapsed_time(e1))
-            nc_bwd.append(e1.elapsed_time(e2))
-    if swa.get_device_error(device) != swa.SWA_OK:
-        raise RuntimeError("device error word set during the non-causal calls")
+    # kernels without tile skipping), timed per kernel group inside the
+    # gradient call after the step's measurements
+    nc = timed_grad(swa, q, k, v, False, stream, device, ws_g)
     nc_fl = 4 * D * B * H * N * N
-    nc_f_ms, nc_b_ms = sorted(nc_fwd)[1], sorted(nc_bwd)[1]
     noncausal = {"workload": f"non-causal attention fwd+bwd B={B} H={H} N={N} D={D} bf16",
-                 "fwd_ms": nc_f_ms, "bwd_ms": nc_b_ms,
-                 "fwd_tflops": nc_fl / (nc_f_ms * 1e-3) / 1e12,
-                 "bwd_tflops": 2.5 * nc_fl / (nc_b_ms * 1e-3) / 1e12,
-                 "timing": "median of 3 API calls after 2 warm-up calls, CUDA events"}
+                 "fwd_ms": nc["fwd_ms"], "bwd_ms": nc["bwd_ms"],
+                 "fwd_tflops": nc_fl / (nc["fwd_ms"] * 1e-3) / 1e12,
+                 "bwd_tflops": 2.5 * nc_fl / (nc["bwd_ms"] * 1e-3) / 1e12,
+                 "timing": "median of 3 gradient calls after 2 warm-up calls; CUDA events "
+                           "around the forward and the backward kernels"}
 
     pk = peaks()
+    configs = other_configs(swa, inputs, torch, stream, device, pk, info,
+                            cpu=info.is_root and info.world == 1 and not args.no_cpu_baseline)
     dom = 2  # the backward's main kernel dominates the step
     dom_ms = kernel_ms[dom]
     achieved = bwd_fl / (dom_ms * 1e-3) / 1e12 if dom_ms else None
@@ -391,13 +596,14 @@ def run_ours(args, info):
         "traffic": recorded_traffic(dom),
         "peak_source": f"{pk['source']} bf16 dense (burst)",
         "flops_per_launch": bwd_fl, "ms_per_launch": dom_ms,
-        "launch": "attn_bwd_dkdv_kernel + attn_bwd_dq_kernel (one event pair around both)",
+        "launch": "attn_bwd_dkdv_kernel + attn_bwd_dq_kernel, f16- and bf16-operand "
+                  "instances (one event pair around the four launches of the gradient call)",
     }
     if pk.get("bf16_tflops_sustained") and achieved:
         roofline["frac_of_sustained"] = achieved / pk["bf16_tflops_sustained"]
     # the other main kernels against their own bounds: the forward against the
     # bf16 tensor peak, the regrid against MUFU (148 SMs x 16 ex2/clk x max clock)
-    mufu_peak = 148 * 16 * SM_MAX_MHZ * 1e6 / 1e9  # Gpair/s
+    mufu_peak = MUFU_GPAIRS
     n_tiles = (N + 127) // 128
     fwd_ex2 = B * H * (n_tiles * (n_tiles + 1) // 2) * 128 * 128
     nw_rate = NW_M * NW_S / (kernel_ms[3] * 1e-3) / 1e9 if kernel_ms[3] else None
@@ -413,7 +619,8 @@ def run_ours(args, info):
         "nw_regrid": {"bound": "alu", "achieved": nw_rate, "peak": mufu_peak, "unit": "Gpair/s",
                       "frac": nw_rate / mufu_peak if nw_rate else None,
                       "traffic": recorded_traffic(3),
-                      "peak_source": "148 SMs x 16 MUFU ex2/clk x 1965 MHz (one ex2 per pair)"},
+                      "peak_source": "148 SMs x 16 MUFU ex2/clk x 1965 MHz (one ex2 per pair)",
+                      "timing": "the whole call: pair-grid kernel and final sum"},
     }
     breakdown = {
         "attn_fwd_ms": kernel_ms[1], "attn_bwd_ms": kernel_ms[2], "nw_ms": kernel_ms[3],
@@ -443,13 +650,16 @@ def run_ours(args, info):
                                    f"(dout = out) + Nadaraya-Watson regrid {NW_M}x{NW_S} "
                                    f"fp32 h={H_BW}",
                        "global_batch": B * info.world, "seq_len": N,
-                       "parallelism": f"replicas x{info.world} (independent heads)",
+                       "parallelism": f"heads split over {info.world} GPU(s): rank r takes "
+                                      f"sequences [{B}r, {B}r+{B}) of a {B * info.world}-"
+                                      f"sequence batch (no data-path collective)",
                        "l2": "inputs larger than L2 (Q, K, V = 201 MB per rank)"},
             "roofline": roofline, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": timed_launches, "clocks": clocks.summary(),
             "breakdown": breakdown, "rooflines": rooflines, "noncausal": noncausal,
+            "configs": configs,
         }
         print(json.dumps(line), flush=True)
     sdist.shutdown()

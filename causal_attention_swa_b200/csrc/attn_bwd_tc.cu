@@ -10,6 +10,13 @@
 //   dv_j += P_ij dout_i   dk_j += scale dS_ij q_i   dq_i += scale dS_ij k_j
 // over the pairs that exist (j <= i when causal).
 //
+// Operands: the kernels are instantiated for f16 and for bf16 operands.  The
+// f16 instance reads f16 copies of q, k, v and dout (made by the caller's
+// prep pass, exact for values below 2^15 in magnitude) and takes P and dS as
+// f16 (10 fraction bits), which keeps the end-to-end gradient of
+// 1/2 sum out^2 inside the bf16 path's tolerance with one dS per dQ product;
+// the bf16 instance (heads with larger values) takes P and dS^T as bf16 and
+// dS for dQ as bf16 hi + lo (below).  Each launch takes the heads of its type.
 // Two kernels, neither with atomics:
 //   attn_bwd_dkdv_kernel  block = one 128-key block j; it walks the query
 //                         blocks i that see j and keeps dV_j, dK_j in TMEM
@@ -44,15 +51,27 @@
 // 128 bytes per clock the SM's shared memory delivers, while A from TMEM
 // costs none of it.  A later S MMA may overwrite those TMEM columns because
 // one thread's MMAs execute in issue order.
-// dS is carried as hi + lo bf16 (hi = bf16(dS), lo = bf16(dS - hi)) for dq:
-// sum_j dS_ij = 0, and a single bf16 rounding of dS, amplified by that
-// cancellation in sum_j dS_ij k_j, costs dq about 2% of its row RMS at
-// N = 2048.  dk has no such cancellation (its sum runs over queries), so
-// dS^T enters dK at bf16.
+// In the bf16 instance dS is carried as hi + lo bf16 (hi = bf16(dS),
+// lo = bf16(dS - hi)) for dq: sum_j dS_ij = 0, and a single bf16 rounding of
+// dS, amplified by that cancellation in sum_j dS_ij k_j, costs dq about 2% of
+// its row RMS at N = 2048.  An f16 dS (three more fraction bits) needs no lo.
 // Causal: a key block meets only the query blocks i >= j; inside a diagonal
 // block (and past N on a ragged tail) P and dS of a masked pair are set to
-// 0 by select.  These kernels take only heads whose V and dout are all
-// finite, so 0 times a finite value is the same as skipping the pair.
+// 0 by select, so dS never carries a masked pair into dK or dQ.
+// Non-finite V or dout (absent rows, "check_masks_are_absent_rows": a masked
+// pair must never enter a product).  Every product over existing pairs is
+// the IEEE one: S, dP, dS and the dK, dQ sums run on the values as given
+// (tcgen05 propagates infinities and NaN), and for dq the lo word of a
+// non-finite dS is 0 (hi - hi would be NaN).  The one product that meets
+// masked pairs is dV += P^T dO_i of the diagonal block: its zero weights
+// meet dout rows of queries before the key.  For a head whose V or dout
+// holds an infinity or NaN (the scan's flag), the dK/dV kernel therefore
+// loads the diagonal block's dO a second time into a buffer of its own,
+// the producer warp replaces its non-finite entries by 0 (recording, per
+// column d, the last query row of the block holding +inf, -inf and NaN),
+// and dV of that block reads the clean copy; the epilogue then merges the
+// IEEE class those rows give dV_jd (rows i >= j of the block, each with a
+// weight > 0) into the value the other blocks accumulated.
 // Every mbarrier wait is bounded (device error word on expiry).
 #include <type_traits>
 
@@ -76,6 +95,29 @@ constexpr int kQStages = 4;             // dkdv's Q/dO ring depth
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDP = 256;
 constexpr int kHeadGroup = 4;           // heads scheduled together (their operands share L2)
+
+// Per-head information (four int32 per head, from the prep pass):
+//   [0] bit 0: V holds an infinity or NaN; bit 1: dout does
+//   [1] [2] [3] largest biased exponent of the finite values of V, of Q and
+//       K, and of dout.
+// A head takes the f16 instance when all three exponents are below 2^15's.
+constexpr int kInfoInts = 4;
+constexpr int kF16ExpLimit = 127 + 15;
+__device__ __forceinline__ bool head_is_f16(const int* info, int head) {
+  const int* hi = info + kInfoInts * head;
+  return max(hi[1], max(hi[2], hi[3])) < kF16ExpLimit;
+}
+
+// A 16-bit value (f16 or bf16) that is +-inf or NaN, and its class
+// (0 = +inf, 1 = -inf, 2 = NaN).
+template <bool kF16>
+__device__ __forceinline__ bool nonfinite16(uint32_t b) {
+  return kF16 ? (b & 0x7C00u) == 0x7C00u : (b & 0x7F80u) == 0x7F80u;
+}
+template <bool kF16>
+__device__ __forceinline__ int class16(uint32_t b) {
+  return (b & (kF16 ? 0x03FFu : 0x7Fu)) ? 2 : ((b & 0x8000u) ? 1 : 0);
+}
 
 __device__ __forceinline__ uint32_t col_s(int b) { return b ? 128u : 0u; }
 
@@ -108,8 +150,12 @@ struct __align__(1024) SmemKV {
   uint8_t v[kTileBytes];
   uint8_t q[kQStages][kTileBytes];
   uint8_t dout[kQStages][kTileBytes];
+  uint8_t dout_diag[kTileBytes];  // non-finite heads: the diagonal block's dO, cleaned
   float nlse[kQStages][BQ];      // -lse_i * log2(e) of each staged query block (-inf past N)
   float delta[kQStages][BQ];     // delta_i (0 past N)
+  int last_cls[3][HD];           // per column: last diagonal-block row with +inf, -inf, NaN
+  uint64_t diag_full;
+  uint64_t diag_clean;
   uint64_t kv_full;
   uint64_t qd_full[kQStages];
   uint64_t qd_empty[kQStages];
@@ -125,6 +171,7 @@ constexpr size_t kSmemKV = sizeof(SmemKV);
 static_assert(kSmemKV <= 232448, "shared memory");
 constexpr uint32_t kColDV = 384, kColDK = 448;
 
+template <bool kF16>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
@@ -132,12 +179,15 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ nlse2,
                      const float* __restrict__ delta, __nv_bfloat16* __restrict__ dk,
                      __nv_bfloat16* __restrict__ dv, int N, int BH, int causal, float scale,
-                     float scale_log2, const int* __restrict__ flags, unsigned* __restrict__ err) {
+                     float scale_log2, const int* __restrict__ info, unsigned* __restrict__ err) {
   const int n_blocks = (N + BQ - 1) / BQ;
   const int Npad = n_blocks * BQ;
   int head, jb;
   block_order(n_blocks, BH, true, &head, &jb);
-  if (flags[head] != 0) return;
+  if (head_is_f16(info, head) != kF16) return;  // the other instance's head
+  // a head with a non-finite V or dout: dV of the diagonal block reads a
+  // cleaned copy of its dO (non-causal: no masked pair meets dO at all)
+  const bool clean_diag = info[kInfoInts * head] != 0 && causal;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (smem_u32(smem_raw) & 1023u) {  // the swizzled tiles need 1024-byte alignment
@@ -159,13 +209,16 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(&sm.qd_empty[s], 1);
     }
     mbar_init(&sm.dp_full, 1);
-    mbar_init(&sm.dp_free, kComputeThreads);
-    mbar_init(&sm.sm_done, kComputeThreads);
+    mbar_init(&sm.dp_free, kComputeThreads / 32);  // one arrival per compute warp
+    mbar_init(&sm.sm_done, kComputeThreads / 32);
     mbar_init(&sm.acc_full, 1);
     mbar_init(&sm.drain, 1);
+    mbar_init(&sm.diag_full, 1);
+    mbar_init(&sm.diag_clean, 1);
     sm.abort = 0;
     fence_mbar_init();
   }
+  if (tid < 3 * HD) (&sm.last_cls[0][0])[tid] = -1;
   if (warp == kMmaWarp) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
@@ -178,6 +231,40 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ producer
+    if (clean_diag) {
+      // the diagonal block's dO once more, into a buffer of its own; every
+      // lane then cleans it (non-finite -> 0, rows recorded per column)
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&sm.diag_full, kTileBytes);
+        tma_load_3d(sm.dout_diag, &tm_do, &sm.diag_full, 0, j0, head);
+      }
+      __syncwarp();
+      if (mbar_wait_parked(&sm.diag_full, 0, abort, err, kDevTimeoutFull)) {
+        uint4* base = reinterpret_cast<uint4*>(sm.dout_diag);
+        for (int c = lane; c < kTileBytes / 16; c += 32) {
+          const uint4 x = base[c];
+          uint32_t w[4] = {x.x, x.y, x.z, x.w};
+          const int r = c >> 3;                      // query row of the block
+          const int d0 = ((c & 7) ^ (r & 7)) * 8;    // first column (swizzle undone)
+          bool changed = false;
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+              const uint32_t bits = (w[e] >> (16 * p)) & 0xFFFFu;
+              if (nonfinite16<kF16>(bits)) {
+                atomicMax(&sm.last_cls[class16<kF16>(bits)][d0 + 2 * e + p], j0 + r);
+                w[e] &= ~(0xFFFFu << (16 * p));
+                changed = true;
+              }
+            }
+          if (changed) base[c] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      fence_proxy_async_smem();  // the dV MMA (async proxy) reads the cleaned tile
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.diag_clean);
+    }
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
@@ -204,8 +291,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
   } else if (warp == kMmaWarp) {
     // --------------------------------------------------------- MMA issuer
     {  // the whole warp runs the issue loop; one elected lane issues
-      constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T: both K-major
-      constexpr uint32_t id_mn = idesc_bf16_f32(128, 64, 0, 1);   // dV, dK: B MN-major
+      constexpr uint32_t fmt = kF16 ? 0u : 1u;
+      constexpr uint32_t id_kk = idesc_f32acc(128, 128, 0, 0, fmt);  // S^T, dP^T: both K-major
+      constexpr uint32_t id_mn = idesc_f32acc(128, 64, 0, 1, fmt);   // dV, dK: B MN-major
       const uint32_t k_s = smem_u32(sm.k), v_s = smem_u32(sm.v);
       // descriptor steps in 16-byte units: K-major +32 B (2) per K = 16
       // step, MN-major +2048 B (128)
@@ -242,11 +330,14 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
           mma_commit_elect(&sm.dp_full);
         }
         if (!mbar_wait_parked(&sm.sm_done, it & 1, abort, err, kDevTimeoutOther)) break;
+        const bool diag = clean_diag && it == 0;  // dV of the diagonal block: the clean dO
+        if (diag && !mbar_wait_parked(&sm.diag_clean, 0, abort, err, kDevTimeoutOther)) break;
         fence_after_sync();
         // dV += P^T dO_i: 16-query group kk's P^T is in S^T columns 32(kk/2) + 8(kk%2)
         mma_ts_run8<128, 8, 32, 40, 64, 72, 96, 104>(
-            tmem + kColDV, tmem + col_s(b), desc_sw128(smem_u32(sm.dout[st]), 8192, 1024),
-            id_mn, it > 0 ? 1u : 0u);
+            tmem + kColDV, tmem + col_s(b),
+            desc_sw128(smem_u32(diag ? sm.dout_diag : sm.dout[st]), 8192, 1024), id_mn,
+            it > 0 ? 1u : 0u);
         // dK += dS^T Q_i: dS^T of 16-query group kk 16 columns further on
         mma_ts_run8<128, 8, 32, 40, 64, 72, 96, 104>(
             tmem + kColDK, tmem + col_s(b) + 16, desc_sw128(smem_u32(sm.q[st]), 8192, 1024),
@@ -318,8 +409,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
               if (ig >= N || jg >= N || (causal && ig < jg)) p.x = ds.x = 0.f;
               if (ig + 1 >= N || jg >= N || (causal && ig + 1 < jg)) p.y = ds.y = 0.f;
             }
-            wp[8 * h + 2 * e4 + u] = pack_bf16(p.x, p.y);
-            wd[8 * h + 2 * e4 + u] = pack_bf16(ds.x, ds.y);
+            wp[8 * h + 2 * e4 + u] = pack_p<kF16>(p.x, p.y);
+            wd[8 * h + 2 * e4 + u] = pack_p<kF16>(ds.x, ds.y);
           }
         }
       };
@@ -332,7 +423,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       tmem_st8(tw, *reinterpret_cast<const uint32_t(*)[8]>(wp));
       tmem_wait_ld_tied(s1, d1);
       fence_before_sync();
-      mbar_arrive(&sm.dp_free);  // dP^T's columns may take the next block's
+      warp_arrive(&sm.dp_free);  // dP^T's columns may take the next block's
       tmem_st8(tw + 16, *reinterpret_cast<const uint32_t(*)[8]>(wd));
       if (need_mask) math(std::true_type{}, s1, d1, 1);
       else math(std::false_type{}, s1, d1, 1);
@@ -340,7 +431,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       tmem_st8(tw + 24, *reinterpret_cast<const uint32_t(*)[8]>(wd + 8));
       tmem_wait_st();
       fence_before_sync();
-      mbar_arrive(&sm.sm_done);
+      warp_arrive(&sm.sm_done);
     }
     // ---- columns 16w..16w+15 of this key's dv and dk
     if (ok && mbar_wait_parked(&sm.acc_full, 0, abort, err, kDevTimeoutMma)) {
@@ -349,6 +440,20 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       tmem_ld16(tmem + lane_off + kColDV + 16 * w, av);
       tmem_ld16(tmem + lane_off + kColDK + 16 * w, ak);
       tmem_wait_ld();
+      if (clean_diag && mbar_wait_parked(&sm.diag_clean, 0, abort, err, kDevTimeoutOther)) {
+        // merge the IEEE class of the diagonal block's rows i >= jg into dv
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int d = 16 * w + e;
+          const float x = __uint_as_float(av[e]);
+          const bool pinf = sm.last_cls[0][d] >= jg || x == INFINITY;
+          const bool ninf = sm.last_cls[1][d] >= jg || x == -INFINITY;
+          const bool nan = sm.last_cls[2][d] >= jg || x != x || (pinf && ninf);
+          if (nan) av[e] = 0x7FC00000u;
+          else if (pinf) av[e] = 0x7F800000u;
+          else if (ninf) av[e] = 0xFF800000u;
+        }
+      }
       if (jg < N) {
         uint4* dvd = reinterpret_cast<uint4*>(dv + ((size_t)head * N + jg) * HD + 16 * w);
         uint4* dkd = reinterpret_cast<uint4*>(dk + ((size_t)head * N + jg) * HD + 16 * w);
@@ -402,18 +507,20 @@ constexpr size_t kSmemQ = sizeof(SmemQ);
 static_assert(kSmemQ <= 232448, "shared memory");
 constexpr uint32_t kColDQ = 384, kColQ = 448, kColDO = 480;
 
+template <bool kF16>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16* __restrict__ q,
-                   const __nv_bfloat16* __restrict__ dout, const float* __restrict__ nlse2,
+                   const __grid_constant__ CUtensorMap tm_v, const uint16_t* __restrict__ q,
+                   const uint16_t* __restrict__ dout, const float* __restrict__ nlse2,
                    const float* __restrict__ delta, __nv_bfloat16* __restrict__ dq, int N, int BH,
-                   int causal, float scale, float scale_log2, const int* __restrict__ flags,
+                   int causal, float scale, float scale_log2, const int* __restrict__ info,
                    unsigned* __restrict__ err) {
   const int n_blocks = (N + BQ - 1) / BQ;
   const int Npad = n_blocks * BQ;
   int head, ib;
   block_order(n_blocks, BH, false, &head, &ib);
-  if (flags[head] != 0) return;
+  if (head_is_f16(info, head) != kF16) return;  // the other instance's head
+  const bool nonfinite = info[kInfoInts * head] != 0;  // V or dout holds an infinity or NaN
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (smem_u32(smem_raw) & 1023u) {
@@ -428,14 +535,14 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
   const int i0 = ib * BQ;
 
   if (tid == 0) {
-    mbar_init(&sm.qt_ready, kComputeThreads);
+    mbar_init(&sm.qt_ready, kComputeThreads / 32);
     for (int s = 0; s < kKVStagesQ; ++s) {
       mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
     }
     mbar_init(&sm.dp_full, 1);
-    mbar_init(&sm.dp_free, kComputeThreads);
-    mbar_init(&sm.sm_done, kComputeThreads);
+    mbar_init(&sm.dp_free, kComputeThreads / 32);  // one arrival per compute warp
+    mbar_init(&sm.sm_done, kComputeThreads / 32);
     mbar_init(&sm.acc_full, 1);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
@@ -471,8 +578,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
   } else if (warp == kMmaWarp) {
     // --------------------------------------------------------- MMA issuer
     {
-      constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, 0, 0);  // S, dP: both K-major
-      constexpr uint32_t id_mn = idesc_bf16_f32(128, 64, 0, 1);   // dQ: B (K_j) MN-major
+      constexpr uint32_t fmt = kF16 ? 0u : 1u;
+      constexpr uint32_t id_kk = idesc_f32acc(128, 128, 0, 0, fmt);  // S, dP: both K-major
+      constexpr uint32_t id_mn = idesc_f32acc(128, 64, 0, 1, fmt);   // dQ: B (K_j) MN-major
       // S = Q K_j^T and dP = dO V_j^T with A from TMEM (8 columns per 16
       // dims) and B K-major (+32 B per 16 dims)
       auto issue_kk = [&](uint32_t d_col, uint32_t a_col, uint32_t b0) {
@@ -516,7 +624,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
         fence_after_sync();
         const uint32_t k0 = smem_u32(sm.k[st]);
         issue_dq(col_s(b), k0, jt == 0);
-        issue_dq(col_s(b) + 16, k0, false);
+        if constexpr (!kF16) issue_dq(col_s(b) + 16, k0, false);  // + the lo words
         mma_commit_elect(&sm.kv_empty[st]);
       }
       mma_commit_elect(&sm.acc_full);
@@ -541,7 +649,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
       uint32_t qa[8], da[8];
       if (ig < N) {
         const size_t off = ((size_t)head * N + ig) * HD + 16 * w;
-        const uint4* qs = reinterpret_cast<const uint4*>(q + off);
+        const uint4* qs = reinterpret_cast<const uint4*>(q + off);  // 16-bit words as given
         const uint4* os = reinterpret_cast<const uint4*>(dout + off);
         const uint4 q0 = qs[0], q1 = qs[1], e0 = os[0], e1 = os[1];
         qa[0] = q0.x; qa[1] = q0.y; qa[2] = q0.z; qa[3] = q0.w;
@@ -556,7 +664,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
       tmem_st8(tmem + lane_off + kColDO + 8 * w, da);
       tmem_wait_st();
       fence_before_sync();
-      mbar_arrive(&sm.qt_ready);
+      warp_arrive(&sm.qt_ready);
     }
     bool ok = true;
     for (int jt = 0; jt < n_k; ++jt) {
@@ -579,9 +687,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
       tmem_ld16(tmem + lane_off + kColDP + kw + 16, d1);
       // two keys at a time in packed f32x2 arithmetic; lo = dS - hi is exact
       uint32_t wh[16], wl[16];
-      auto math = [&](auto mask_tag, const uint32_t (&sv)[16], const uint32_t (&dpv)[16],
-                      int h) {
+      auto math = [&](auto mask_tag, auto nonfinite_tag, const uint32_t (&sv)[16],
+                      const uint32_t (&dpv)[16], int h) {
         constexpr bool kMask = decltype(mask_tag)::value;
+        [[maybe_unused]] constexpr bool kNonFinite = decltype(nonfinite_tag)::value;
 #pragma unroll
         for (int e2 = 0; e2 < 8; ++e2) {
           const int e = 2 * e2;
@@ -597,28 +706,43 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
             if (jg + 1 >= N || ig >= N || (causal && jg + 1 > ig)) ds.y = 0.f;
           }
           const int wi = 8 * h + e2;
-          wh[wi] = pack_bf16(ds.x, ds.y);
-          const float2 lo = __ffma2_rn(make_float2(bf16lo(wh[wi]), bf16hi(wh[wi])), m1, ds);
-          wl[wi] = pack_bf16(lo.x, lo.y);
+          if constexpr (kF16) {
+            wh[wi] = pack_f16(ds.x, ds.y);
+          } else {
+            wh[wi] = pack_bf16(ds.x, ds.y);
+            float2 lo = __ffma2_rn(make_float2(bf16lo(wh[wi]), bf16hi(wh[wi])), m1, ds);
+            if constexpr (kNonFinite) {  // inf - inf: the hi word carries the class alone
+              if (!isfinite(ds.x)) lo.x = 0.f;
+              if (!isfinite(ds.y)) lo.y = 0.f;
+            }
+            wl[wi] = pack_bf16(lo.x, lo.y);
+          }
         }
       };
-      if (need_mask) math(std::true_type{}, s0, d0, 0);
-      else math(std::false_type{}, s0, d0, 0);
+      auto math_any = [&](const uint32_t (&sv)[16], const uint32_t (&dpv)[16], int h) {
+        if (nonfinite) {
+          if (need_mask) math(std::true_type{}, std::true_type{}, sv, dpv, h);
+          else math(std::false_type{}, std::true_type{}, sv, dpv, h);
+        } else {
+          if (need_mask) math(std::true_type{}, std::false_type{}, sv, dpv, h);
+          else math(std::false_type{}, std::false_type{}, sv, dpv, h);
+        }
+      };
+      math_any(s0, d0, 0);
       // dS of these 16 keys over the warpgroup's own S columns: hi at
       // 32w + 0..7, lo at 32w + 16..23 (once the second half's load landed)
       const uint32_t tw = tmem + lane_off + col_s(b) + kw;
       tmem_st8(tw, *reinterpret_cast<const uint32_t(*)[8]>(wh));
       tmem_wait_ld_tied(s1, d1);
       fence_before_sync();
-      mbar_arrive(&sm.dp_free);  // dP's columns may take dP_jt+1
-      tmem_st8(tw + 16, *reinterpret_cast<const uint32_t(*)[8]>(wl));
-      if (need_mask) math(std::true_type{}, s1, d1, 1);
-      else math(std::false_type{}, s1, d1, 1);
+      warp_arrive(&sm.dp_free);  // dP's columns may take dP_jt+1
+      if constexpr (!kF16) tmem_st8(tw + 16, *reinterpret_cast<const uint32_t(*)[8]>(wl));
+      math_any(s1, d1, 1);
       tmem_st8(tw + 8, *reinterpret_cast<const uint32_t(*)[8]>(wh + 8));
-      tmem_st8(tw + 24, *reinterpret_cast<const uint32_t(*)[8]>(wl + 8));
+      if constexpr (!kF16) tmem_st8(tw + 24, *reinterpret_cast<const uint32_t(*)[8]>(wl + 8));
       tmem_wait_st();
       fence_before_sync();
-      mbar_arrive(&sm.sm_done);
+      warp_arrive(&sm.sm_done);
     }
     // ---- columns 16w..16w+15 of this query's dq
     if (ok && mbar_wait_parked(&sm.acc_full, 0, abort, err, kDevTimeoutMma)) {
@@ -649,39 +773,51 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
   }
 }
 
-}  // namespace
-
-cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* dout,
-                               const float* nlse2, const float* delta, void* dq, void* dk,
-                               void* dv, int64_t B, int64_t H, int64_t N, int causal,
-                               float scale, const int* flags, unsigned* err, cudaStream_t s,
-                               int* launches) {
-  const int64_t BH = B * H;
+template <bool kF16>
+cudaError_t launch_bwd_instance(const void* q, const void* k, const void* v, const void* dout,
+                                const float* nlse2, const float* delta, void* dq, void* dk,
+                                void* dv, int64_t BH, int64_t N, int causal, float scale,
+                                const int* info, unsigned* err, cudaStream_t s, int* launches) {
   CUtensorMap tq, tk, tv, tdo;
   cudaError_t e;
   if ((e = make_tmap_bf16_rows(&tq, q, BH, N, BQ)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_rows(&tk, k, BH, N, BK)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_rows(&tv, v, BH, N, BK)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_rows(&tdo, dout, BH, N, BQ)) != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kSmemKV);
+  e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel<kF16>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemKV);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(attn_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(attn_bwd_dq_kernel<kF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)kSmemQ);
   if (e != cudaSuccess) return e;
   const int64_t n_blocks = (N + BK - 1) / BK;
-  attn_bwd_dkdv_kernel<<<(unsigned)(n_blocks * BH), kThreads, kSmemKV, s>>>(
+  attn_bwd_dkdv_kernel<kF16><<<(unsigned)(n_blocks * BH), kThreads, kSmemKV, s>>>(
       tq, tk, tv, tdo, nlse2, delta, static_cast<__nv_bfloat16*>(dk),
-      static_cast<__nv_bfloat16*>(dv), (int)N, (int)BH, causal, scale, scale * kLog2e, flags,
+      static_cast<__nv_bfloat16*>(dv), (int)N, (int)BH, causal, scale, scale * kLog2e, info,
       err);
   *launches += 1;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  attn_bwd_dq_kernel<<<(unsigned)(n_blocks * BH), kThreads, kSmemQ, s>>>(
-      tk, tv, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dout),
-      nlse2, delta, static_cast<__nv_bfloat16*>(dq), (int)N, (int)BH, causal,
-      scale, scale * kLog2e, flags, err);
+  attn_bwd_dq_kernel<kF16><<<(unsigned)(n_blocks * BH), kThreads, kSmemQ, s>>>(
+      tk, tv, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(dout), nlse2, delta,
+      static_cast<__nv_bfloat16*>(dq), (int)N, (int)BH, causal, scale, scale * kLog2e, info,
+      err);
   *launches += 1;
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bwd_tc(const BwdOperands& f16, const BwdOperands& bf16,
+                               const float* nlse2, const float* delta, void* dq, void* dk,
+                               void* dv, int64_t B, int64_t H, int64_t N, int causal,
+                               float scale, const int* info, unsigned* err, cudaStream_t s,
+                               int* launches) {
+  const int64_t BH = B * H;
+  cudaError_t e = launch_bwd_instance<true>(f16.q, f16.k, f16.v, f16.dout, nlse2, delta, dq, dk,
+                                            dv, BH, N, causal, scale, info, err, s, launches);
+  if (e != cudaSuccess) return e;
+  return launch_bwd_instance<false>(bf16.q, bf16.k, bf16.v, bf16.dout, nlse2, delta, dq, dk, dv,
+                                    BH, N, causal, scale, info, err, s, launches);
 }
 
 }  // namespace swa

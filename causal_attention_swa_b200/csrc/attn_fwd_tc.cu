@@ -1,6 +1,6 @@
 // attn_fwd_tc.cu -- causal / non-causal attention forward on the sm_100a
-// tensor cores (tcgen05.mma kind::f16, bf16 operands, f32 accumulators in
-// TMEM, TMA-staged K/V).
+// tensor cores (tcgen05.mma kind::f16: bf16 Q K^T, f16 or bf16 P V; f32
+// accumulators in TMEM; TMA-staged K/V).
 //
 // The method: "Show HN: Automatic deduction of FlashAttention kernel from
 // ~25 lines of SQL" (page 2, the demo's docstring): FlashAttention streams
@@ -17,7 +17,10 @@
 //   warp  16    TMA producer: Q0, Q1 once, then K_j, V_j into 4 stages
 //   warp  17    MMA issuer for query tile 0 (one elected lane), TMEM owner
 //   warp  18    MMA issuer for query tile 1
-//   warp  19    idle (gives its registers to the softmax warps of its scheduler)
+//   warp  19    V converter: rewrites each staged V tile in place (bf16 ->
+//               f16, and a non-finite entry -> 0 with its row recorded), then
+//               releases it to the issuers; it also gives its registers to
+//               the softmax warps of its scheduler
 // Each query tile has an issuer of its own, so neither tile's MMAs queue
 // behind the other tile's barriers; each issuer releases a K/V stage on a
 // barrier of its own and the producer waits for the issuers that read it.
@@ -27,8 +30,8 @@
 // that the kernel was built with exactly 96: a larger claim than the
 // scheduler holds would stall setmaxnreg.inc.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384)
-// O0 [384,448) O1 [448,512).  P_t (bf16, two per column) has columns of its
-// own and is the A operand of O_t += P_t V_j straight from TMEM.
+// O0 [384,448) O1 [448,512).  P_t (16-bit, two per column) has columns of
+// its own and is the A operand of O_t += P_t V_j straight from TMEM.
 // The softmax warps copy S_t,j into registers and release its columns
 // (s_free) first, so the MMA warp computes S_t,j+1 while they exponentiate
 // S_t,j: the tensor work hides under the softmax instead of alternating
@@ -47,14 +50,44 @@
 // Online softmax in the log2 domain with a lazy rescale: the reference max
 // of a row moves (and O, l are rescaled) only when the new row max exceeds
 // it by more than 8, so P <= 2^8 (exact after the final division by l).
+// Precision of O += P V: P enters the MMA as f16 (10 fraction bits) with V
+// converted to f16 in shared memory, for every head whose finite V values
+// lie below 2^15 in magnitude (f16 holds them exactly, up to f16's
+// subnormal spacing of 2^-24); a head with larger values keeps both in
+// bf16.  A bf16 P (7 fraction bits) is exact enough for the output itself,
+// but the output is what the gradient of loss = 1/2 sum out^2 feeds back
+// as dout, and the rounding of few-key rows (early rows) reaches the
+// gradient amplified by the cancellation in sum_j dS_ij k_j; with the f16 P
+// the end-to-end gradient stays inside the bf16 path's tolerance.  Rows
+// that see few keys (the first rows of a causal head) average no rounding
+// away, so on the diagonal tile -- the last key tile of every causal query
+// tile -- P also enters as the sum of two 16-bit words: its rounding
+// residual goes into that tile's S columns (free then: no later S is
+// computed for the query tile) and a second P V product adds it.  The
+// kernel is instantiated for both operand types; each launch takes the
+// heads of its type (the per-head scan of V decides).
+// For the gradient of loss = 1/2 sum out^2 (dout = out) the epilogue can
+// also write what the backward reads: an f16 copy of the float32 output,
+// delta_i = sum_d out_id^2 in float32, and -lse_i log2 e, the last two
+// padded to whole 128-row blocks.
 // Causal: key tiles past the diagonal are never loaded; inside the
 // diagonal tile (and past N on a ragged tail) a masked score is replaced by
-// -inf before the max, so its weight is exactly 0; V is all-finite in the
-// heads this kernel takes (the caller's scan), so 0 * v = 0 and the product
-// is the same as skipping the pair.
+// -inf before the max, so its weight is exactly 0.
+// Non-finite V (absent rows: a masked pair must never enter a product,
+// "check_masks_are_absent_rows"): a masked weight of a diagonal tile meets
+// the V rows of keys after the query, and 0 * inf would be NaN.  For a head
+// whose V holds an infinity or NaN (the scan's flag) the converter warp
+// replaces every non-finite V entry by 0 before the MMA reads the tile and
+// records, per column d, the first key row holding +inf, -inf and NaN; the
+// epilogue then sets out[i, d] to the IEEE class that the sum over the
+// existing pairs j in J(i) takes (every existing weight is > 0): NaN if a
+// NaN, or both infinities, lie in rows J(i), else the infinity that does,
+// else the finite value computed from the sanitised V.
 // Every mbarrier wait is bounded; on expiry the block records an error code
 // in the device error word, all roles leave their loops, and TMEM is freed.
 #include <cudaTypedefs.h>
+
+#include <climits>
 
 #include "attn_tc.cuh"
 #include "tc_ptx.cuh"
@@ -84,7 +117,14 @@ constexpr int kMmaWarp = kSoftmaxWarps + 1;  // issuer of tile 0; kMmaWarp + 1 i
 constexpr int kHalf = BN / 2;                // score columns per softmax thread
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
-constexpr float kFastRange = 64.0f;  // P < 2^64 against a stale max still fits
+// A P computed against a stale reference max must still fit the operand
+// type before it is moved to the new max: < 2^15 in f16, < 2^64 in bf16.
+template <bool kF16> constexpr float kFastRange = kF16 ? 15.0f : 64.0f;
+constexpr int kConvWarp = kSoftmaxWarps + 3;  // warp 19
+// Per-head information (kHeadInfoInts int32 per head): bit 0 of [0] is set if
+// V holds an infinity or NaN, [1] is the largest biased exponent of its
+// finite values.  f16 operands are used when that exponent is below 2^15's.
+constexpr int kF16ExpLimit = 127 + 15;
 
 
 struct __align__(1024) Smem {
@@ -99,6 +139,9 @@ struct __align__(1024) Smem {
   uint64_t s_free[2];
   uint64_t p_full[2];
   uint64_t pv_done[2];
+  uint64_t v_ready[kStages];    // the converter has rewritten the stage's V tile
+  uint64_t cls_done;            // the converter has recorded every tile's classes
+  int first_cls[3][HD];         // per column: first key row with +inf, -inf, NaN
   uint64_t pair[2][4];          // the two threads of a row: tile t, lanes 32w..
   float part[2][2][2][BM];      // [tile][parity][half][row]: partial row max / sum
   uint64_t drain[2];
@@ -120,16 +163,56 @@ __device__ __forceinline__ bool wait_unbounded_by_abort(uint64_t* bar, uint32_t 
   return true;
 }
 
+// Rewrites one staged V tile (128 rows of 128 bytes, 128-byte swizzle) in
+// place: a non-finite entry becomes 0 with its row recorded in first_cls
+// (when `nonfinite`), and every entry is converted to f16 (when kF16).
+template <bool kF16>
+__device__ __forceinline__ void convert_v_tile(uint8_t* tile, int lane, int key0, bool nonfinite,
+                                               int (*first_cls)[HD]) {
+  uint4* base = reinterpret_cast<uint4*>(tile);
+#pragma unroll 4
+  for (int c = lane; c < kTileBytes / 16; c += 32) {
+    const uint4 x = base[c];
+    uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    if (nonfinite) {
+      const int r = c >> 3;                      // row of the tile
+      const int d0 = ((c & 7) ^ (r & 7)) * 8;    // its first column (swizzle undone)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+          const uint32_t b = (w[e] >> (16 * p)) & 0xFFFFu;
+          if ((b & 0x7F80u) == 0x7F80u) {
+            const int cls = (b & 0x7Fu) ? 2 : ((b & 0x8000u) ? 1 : 0);
+            atomicMin(&first_cls[cls][d0 + 2 * e + p], key0 + r);
+            w[e] &= ~(0xFFFFu << (16 * p));
+          }
+        }
+    }
+    if constexpr (kF16) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) w[e] = pack_f16(bf16lo(w[e]), bf16hi(w[e]));
+    }
+    base[c] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+template <bool kF16>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
                    float* __restrict__ lse, int N, int BH, int n_ctiles, int causal,
-                   float scale_log2, const int* __restrict__ flags, unsigned* __restrict__ err) {
+                   float scale_log2, const int* __restrict__ vinfo, uint16_t* __restrict__ do16,
+                   float* __restrict__ delta, float* __restrict__ nlse2,
+                   unsigned* __restrict__ err) {
   // Longest first: every head's latest (heaviest) query tiles, then the next.
   const int head = blockIdx.x % BH;
   const int c = n_ctiles - 1 - blockIdx.x / BH;
-  if (flags[head] != 0) return;         // a non-finite head: the pair-by-pair kernel's
+  const bool nonfinite = (vinfo[kHeadInfoInts * head] & 1) != 0;
+  if ((vinfo[kHeadInfoInts * head + 1] < kF16ExpLimit) != kF16) return;  // the other instance's head
+  // the converter rewrites V tiles for f16 operands or to remove non-finite values
+  const bool convert = kF16 || nonfinite;
 
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -158,16 +241,19 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&sm.s_full[t], 1);
-      mbar_init(&sm.s_free[t], 256);
-      mbar_init(&sm.p_full[t], 256);
+      mbar_init(&sm.s_free[t], kSoftmaxWarps / 2);  // one arrival per softmax warp of tile t
+      mbar_init(&sm.p_full[t], kSoftmaxWarps / 2);
       mbar_init(&sm.pv_done[t], 1);
-      for (int w = 0; w < 4; ++w) mbar_init(&sm.pair[t][w], 64);
+      for (int w = 0; w < 4; ++w) mbar_init(&sm.pair[t][w], 2);  // the row's two warps
     }
     mbar_init(&sm.drain[0], 1);
     mbar_init(&sm.drain[1], 1);
+    for (int s = 0; s < kStages; ++s) mbar_init(&sm.v_ready[s], 1);
+    mbar_init(&sm.cls_done, 1);
     sm.abort = 0;
     fence_mbar_init();
   }
+  if (tid < 3 * HD) (&sm.first_cls[0][0])[tid] = INT_MAX;
   if (warp == kMmaWarp) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
@@ -211,7 +297,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     {  // the whole warp runs the issue loop; one elected lane issues
       const int t = warp - kMmaWarp;
       constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BN, 0, 0);  // Q, K both K-major
-      constexpr uint32_t idesc_o = idesc_bf16_f32(BM, HD, 0, 1);  // V is MN-major (dims contiguous)
+      // V is MN-major (dims contiguous); P and V are f16 or bf16 together
+      constexpr uint32_t idesc_o = kF16 ? idesc_f16_f32(BM, HD, 0, 1) : idesc_bf16_f32(BM, HD, 0, 1);
       const uint64_t q_desc = desc_sw128(smem_u32(sm.q[t]), 16, 1024);
       auto issue_s = [&](int j) {
         // one asm block of 4 MMAs; K steps of 32 B = 2 descriptor units
@@ -220,10 +307,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         mma_commit_elect(&sm.s_full[t]);
       };
       auto issue_pv = [&](int j) {
+        const uint64_t v_desc = desc_sw128(smem_u32(sm.v[j % kStages]), 8192, 1024);
         // 8 MMAs: P columns 8k, V rows 16k (+2048 B = 128 units)
-        mma_ts_run8<128, 8, 16, 24, 32, 40, 48, 56>(
-            tmem + col_o(t), tmem + col_p(t), desc_sw128(smem_u32(sm.v[j % kStages]), 8192, 1024),
-            idesc_o, j > 0 ? 1u : 0u);
+        mma_ts_run8<128, 8, 16, 24, 32, 40, 48, 56>(tmem + col_o(t), tmem + col_p(t), v_desc,
+                                                    idesc_o, j > 0 ? 1u : 0u);
+        if (causal && j == n_t[t] - 1)  // the diagonal tile: + P's residual (in S's columns)
+          mma_ts_run8<128, 8, 16, 24, 64, 72, 80, 88>(tmem + col_o(t), tmem + col_s(t), v_desc,
+                                                      idesc_o, 1u);
         mma_commit_elect(&sm.pv_done[t]);
         mma_commit_elect(&sm.kv_empty[t][j % kStages]);
       };
@@ -246,8 +336,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           fence_after_sync();
           issue_s(j + 1);
         }
-        if (!mbar_wait_parked(&sm.v_full[j % kStages], (j / kStages) & 1, abort, err,
-                              kDevTimeoutFull) ||
+        if (!mbar_wait_parked(convert ? &sm.v_ready[j % kStages] : &sm.v_full[j % kStages],
+                              (j / kStages) & 1, abort, err, kDevTimeoutFull) ||
             !mbar_wait_parked(&sm.p_full[t], j & 1, abort, err, kDevTimeoutOther))
           break;
         fence_after_sync();
@@ -256,6 +346,22 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       // every MMA this warp issued has finished before TMEM is released
       mma_commit_elect(&sm.drain[t]);
       wait_unbounded_by_abort(&sm.drain[t], 0);
+    }
+    __syncwarp();
+  } else if (warp == kConvWarp) {
+    // ---------------------------------------------------------- converter
+    if (convert) {
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j % kStages;
+        if (!mbar_wait_parked(&sm.v_full[s], (j / kStages) & 1, abort, err, kDevTimeoutFull))
+          break;
+        convert_v_tile<kF16>(sm.v[s], lane, j * BN, nonfinite, sm.first_cls);
+        fence_proxy_async_smem();  // the MMA (async proxy) reads what was written
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.v_ready[s]);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.cls_done);
     }
     __syncwarp();
   } else if (warp < kSoftmaxWarps) {
@@ -277,7 +383,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     auto exchange = [&](float v, float& other) -> bool {
       const int slot = pair_phase & 1;
       sm.part[t][slot][h][r] = v;
-      mbar_arrive(pair);
+      warp_arrive(pair);
       if (!mbar_wait_parked(pair, pair_phase & 1, abort, err, kDevTimeoutOther)) return false;
       other = sm.part[t][slot][h ^ 1][r];
       ++pair_phase;
@@ -306,7 +412,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           for (int e = 0; e < 16; ++e) x[i * 16 + e] = __uint_as_float(u[i][e]);
       }
       fence_before_sync();
-      mbar_arrive(&sm.s_free[t]);  // S_t,j is in registers: its columns may take S_t,j+1
+      warp_arrive(&sm.s_free[t]);  // S_t,j is in registers: its columns may take S_t,j+1
       const bool need_mask = (j * BN + BN > N) || (causal && j == g);
       if (need_mask) {
 #pragma unroll
@@ -339,7 +445,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint32_t par = static_cast<uint32_t>(pair_phase & 1);
       ++pair_phase;
       sm.part[t][slot][h][r] = mine_l2;
-      mbar_arrive(pair);
+      warp_arrive(pair);
       float m_new = m_used;
       bool pair_seen = false;  // set by an earlier successful probe
       auto fetch_and_decide = [&]() -> bool {
@@ -352,7 +458,11 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (j == 0 || mc > m_used + kRescaleThreshold) m_new = mc;
         return true;
       };
-      const bool early = __any_sync(0xffffffffu, j == 0 || !(mine_l2 <= m_used + kFastRange));
+      // the diagonal tile (last of a causal query tile) recomputes P below
+      // for its residual, against the final reference max: fetch it first
+      const bool diag_lo = causal && j == n_t[t] - 1;
+      const bool early = diag_lo ||
+          __any_sync(0xffffffffu, j == 0 || !(mine_l2 <= m_used + kFastRange<kF16>));
       if (early && !fetch_and_decide()) { ok = false; break; }
       const float m_exp = m_new;  // the reference the ex2 loop uses
       // O_t += P_t,j-1 V_j-1 (issued at the end of the last tile) is probed
@@ -368,7 +478,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           const float2 a = __ffma2_rn(make_float2(x[2 * e], x[2 * e + 1]), sc2, nm2);
           const float2 pe = make_float2(ex2(a.x), ex2(a.y));
           rsp[e & 1] = __fadd2_rn(rsp[e & 1], pe);
-          pk[i][e & 15] = pack_bf16(pe.x, pe.y);
+          pk[i][e & 15] = pack_p<kF16>(pe.x, pe.y);
         }
       };
       exps(0);
@@ -382,7 +492,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int i = 0; i < kHalf / 32; ++i)
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            pk[i][e] = pack_bf16(bf16lo(pk[i][e]) * beta, bf16hi(pk[i][e]) * beta);
+            pk[i][e] = pack_p<kF16>(unpack_lo<kF16>(pk[i][e]) * beta,
+                                    unpack_hi<kF16>(pk[i][e]) * beta);
         rsp[0].x *= beta; rsp[0].y *= beta; rsp[1].x *= beta; rsp[1].y *= beta;
       }
       // O_t += P_t,j-1 V_j-1 must finish before O_t is rescaled or P_t is
@@ -411,36 +522,96 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       m_used = m_new;
 #pragma unroll
       for (int i = 0; i < kHalf / 32; ++i) tmem_st16(tP + i * 16, pk[i]);
+      if (diag_lo) {
+        // P's rounding residual P - hi(P), 16 keys per 8 columns, over this
+        // thread's own S columns (each chunk is read before it is written)
+#pragma unroll 1
+        for (int cidx = 0; cidx < kHalf / 16; ++cidx) {
+          uint32_t u[16];
+          tmem_ld16(tS + 16 * cidx, u);
+          tmem_wait_ld();
+          uint32_t lo[8];
+#pragma unroll
+          for (int e2 = 0; e2 < 8; ++e2) {
+            float2 sv = make_float2(__uint_as_float(u[2 * e2]), __uint_as_float(u[2 * e2 + 1]));
+            const int key = j * BN + kHalf * h + 16 * cidx + 2 * e2;
+            if (key >= N || key > row) sv.x = -INFINITY;
+            if (key + 1 >= N || key + 1 > row) sv.y = -INFINITY;
+            const float2 a = __ffma2_rn(sv, sc2, nm2);
+            const float2 pe = make_float2(ex2(a.x), ex2(a.y));
+            const uint32_t hi = pack_p<kF16>(pe.x, pe.y);
+            lo[e2] = pack_p<kF16>(pe.x - unpack_lo<kF16>(hi), pe.y - unpack_hi<kF16>(hi));
+          }
+          tmem_st8(tS + 8 * cidx, lo);
+        }
+      }
       // S_t,j+1 was issued early in this tile: probe it while the stores land
       s_ready = j + 1 < n_t[t] && mbar_test_wait(&sm.s_full[t], (j + 1) & 1);
       tmem_wait_st();
       fence_before_sync();
-      mbar_arrive(&sm.p_full[t]);
+      warp_arrive(&sm.p_full[t]);
       l += (rsp[0].x + rsp[0].y) + (rsp[1].x + rsp[1].y);
     }
     float l_other = 0.f;
     if (ok && n_t[t] > 0 && exchange(l, l_other) &&
         mbar_wait_parked(&sm.pv_done[t], (n_t[t] - 1) & 1, abort, err, kDevTimeoutMma)) {
       fence_after_sync();
-      const float inv = 1.f / (h == 0 ? l + l_other : l_other + l);
-      uint32_t packed[HD / 4];
+      const float l_row = h == 0 ? l + l_other : l_other + l;
+      const float inv = 1.f / l_row;
+      float o[HD / 2];  // this thread's 32 columns of out_row, float32
 #pragma unroll
       for (int i = 0; i < HD / 32; ++i) {
         uint32_t u[16];
         tmem_ld16(tO + i * 16, u);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          packed[i * 8 + e] = pack_bf16(__uint_as_float(u[2 * e]) * inv,
-                                        __uint_as_float(u[2 * e + 1]) * inv);
+        for (int e = 0; e < 16; ++e) o[i * 16 + e] = __uint_as_float(u[e]) * inv;
       }
+      if (nonfinite && mbar_wait_parked(&sm.cls_done, 0, abort, err, kDevTimeoutOther)) {
+        // IEEE class of sum_{j in J(row)} P_ij v_jd with every P_ij > 0
+        const int last = causal ? row : N - 1;
+#pragma unroll
+        for (int e = 0; e < HD / 2; ++e) {
+          const int d = (HD / 2) * h + e;
+          const bool pinf = sm.first_cls[0][d] <= last, ninf = sm.first_cls[1][d] <= last;
+          const bool nan = sm.first_cls[2][d] <= last || (pinf && ninf);
+          if (nan) o[e] = __uint_as_float(0x7FC00000u);
+          else if (pinf) o[e] = INFINITY;
+          else if (ninf) o[e] = -INFINITY;
+        }
+      }
+      const float lse2 = m_used + __log2f(l_row);  // lse * log2 e
       if (row < N) {
         uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)head * N + row) * HD + (HD / 2) * h);
 #pragma unroll
         for (int i = 0; i < HD / 16; ++i)
-          dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2],
-                              packed[4 * i + 3]);
-        if (h == 0) lse[(size_t)head * N + row] = (m_used + __log2f(l + l_other)) * kLn2;
+          dst[i] = make_uint4(pack_bf16(o[8 * i], o[8 * i + 1]), pack_bf16(o[8 * i + 2], o[8 * i + 3]),
+                              pack_bf16(o[8 * i + 4], o[8 * i + 5]),
+                              pack_bf16(o[8 * i + 6], o[8 * i + 7]));
+        if (h == 0) lse[(size_t)head * N + row] = lse2 * kLn2;
+      }
+      if (do16 != nullptr) {
+        // what the backward of loss = 1/2 sum out^2 reads: dout = out as f16,
+        // delta = sum_d out_d^2, -lse log2 e (rows past N: 0 and -inf)
+        float sq = 0.f;
+#pragma unroll
+        for (int e = 0; e < HD / 2; ++e) sq = fmaf(o[e], o[e], sq);
+        float sq_other = 0.f;
+        const bool got = exchange(sq, sq_other);
+        const int64_t Npad = pad128(N);
+        if (row < N) {
+          uint4* dst = reinterpret_cast<uint4*>(do16 + ((size_t)head * N + row) * HD + (HD / 2) * h);
+#pragma unroll
+          for (int i = 0; i < HD / 16; ++i)
+            dst[i] = make_uint4(pack_f16(o[8 * i], o[8 * i + 1]), pack_f16(o[8 * i + 2], o[8 * i + 3]),
+                                pack_f16(o[8 * i + 4], o[8 * i + 5]),
+                                pack_f16(o[8 * i + 6], o[8 * i + 7]));
+        }
+        if (got && h == 0 && row < Npad) {
+          const bool real = row < N;
+          delta[(size_t)head * Npad + row] = real ? sq + sq_other : 0.f;
+          nlse2[(size_t)head * Npad + row] = real ? -lse2 : -INFINITY;
+        }
       }
     }
   }
@@ -486,30 +657,48 @@ cudaError_t make_tmap_bf16_rows(CUtensorMap* map, const void* base, int64_t BH, 
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+template <bool kF16>
+cudaError_t launch_fwd_instance(const CUtensorMap& tq, const CUtensorMap& tk,
+                                const CUtensorMap& tv, void* out, float* lse, int64_t BH,
+                                int64_t N, int causal, float scale, const int* vinfo,
+                                const FwdSaved& saved, unsigned* err, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<kF16>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, attn_fwd_tc_kernel<kF16>);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;  // register split unsafe
+  const int n_ctiles = (int)((N + 2 * BM - 1) / (2 * BM));
+  const int64_t grid = (int64_t)n_ctiles * BH;
+  attn_fwd_tc_kernel<kF16><<<(unsigned)grid, kThreads, kSmemBytes, s>>>(
+      tq, tk, tv, static_cast<__nv_bfloat16*>(out), lse, (int)N, (int)BH, n_ctiles, causal,
+      scale * kLog2e, vinfo, static_cast<uint16_t*>(saved.do16), saved.delta, saved.nlse2, err);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_attn_fwd_tc(const void* q, const void* k, const void* v, void* out,
                                float* lse, int64_t B, int64_t H, int64_t N, int causal,
-                               float scale, const int* flags, unsigned* err, cudaStream_t s,
-                               int* launches) {
+                               float scale, const int* vinfo, const FwdSaved& saved,
+                               unsigned* err, cudaStream_t s, int* launches) {
   const int64_t BH = B * H;
   CUtensorMap tq, tk, tv;
   cudaError_t e;
   if ((e = make_tmap_bf16_rows(&tq, q, BH, N, BM)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_rows(&tk, k, BH, N, BN)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_rows(&tv, v, BH, N, BN)) != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kSmemBytes);
-  if (e != cudaSuccess) return e;
-  cudaFuncAttributes fa;
-  e = cudaFuncGetAttributes(&fa, attn_fwd_tc_kernel);
-  if (e != cudaSuccess) return e;
-  if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;  // register split unsafe
-  const int n_ctiles = (int)((N + 2 * BM - 1) / (2 * BM));
-  const int64_t grid = (int64_t)n_ctiles * BH;
-  attn_fwd_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(
-      tq, tk, tv, static_cast<__nv_bfloat16*>(out), lse, (int)N, (int)BH, n_ctiles, causal,
-      scale * kLog2e, flags, err);
+  // f16-operand heads (the usual case) first; the bf16 instance's blocks of
+  // those heads exit at once, and the other way round
+  if ((e = launch_fwd_instance<true>(tq, tk, tv, out, lse, BH, N, causal, scale, vinfo, saved,
+                                     err, s)) != cudaSuccess)
+    return e;
   *launches += 1;
-  return cudaGetLastError();
+  if ((e = launch_fwd_instance<false>(tq, tk, tv, out, lse, BH, N, causal, scale, vinfo, saved,
+                                      err, s)) != cudaSuccess)
+    return e;
+  *launches += 1;
+  return cudaSuccess;
 }
 
 }  // namespace swa

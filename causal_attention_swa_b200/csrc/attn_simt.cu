@@ -6,13 +6,14 @@
 // lines of SQL", view ATTENTION_WINDOW and check_masks_are_absent_rows): a
 // masked pair is skipped by a branch, never multiplied by a zero weight, so
 // non-finite values in V or dout propagate exactly as IEEE sums over the
-// existing pairs.  They serve the float32 path and the heads of the bf16
-// path that hold a non-finite value.
+// existing pairs.  They are the float32 path.
 //
 // Forward: one thread per query row keeps q (pre-scaled into the log2
 // domain), the output accumulator and the running (max, sum) in registers,
 // and streams 32-key K/V tiles through shared memory; the online softmax
-// rescales once per 16-key chunk.
+// rescales once per 16-key chunk, and leaves an accumulator that is already
+// +-inf or NaN as it is (a weight > 0 keeps its class; a rescale factor that
+// underflows to 0 must not turn it into 0 * inf = NaN).
 // Backward: delta_i = dout_i . out_i (prep kernel, also lse * log2 e, both
 // padded to whole 128-row blocks for the tensor-core kernel); a key-major kernel
 // accumulates dk_j, dv_j over the rows i that see j; a query-major kernel
@@ -86,9 +87,8 @@ template <typename T>
 __global__ void __launch_bounds__(kFwdRows)
 attn_fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                      T* __restrict__ out, float* __restrict__ lse, int64_t N, int causal,
-                     float scale_log2, const int* __restrict__ flags, int select) {
+                     float scale_log2) {
   const int64_t head = blockIdx.y;
-  if (!head_selected(flags, head, select)) return;
   __shared__ __align__(16) float Ks[kFwdKeys][D];
   __shared__ __align__(16) float Vs[kFwdKeys][D];
 
@@ -146,7 +146,7 @@ attn_fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
         const float alpha = exp2f(m - mc);  // 0 on the first chunk (m = -inf)
         l *= alpha;
 #pragma unroll
-        for (int d = 0; d < D; ++d) o[d] *= alpha;
+        for (int d = 0; d < D; ++d) o[d] = isfinite(o[d]) ? o[d] * alpha : o[d];
         m = mc;
       }
 #pragma unroll
@@ -219,10 +219,8 @@ attn_bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
                           const T* __restrict__ v, const T* __restrict__ dout,
                           const float* __restrict__ lse, const float* __restrict__ delta,
                           T* __restrict__ dk, T* __restrict__ dv, int64_t N, int64_t dstride,
-                          int causal, float scale, float scale_log2,
-                          const int* __restrict__ flags, int select) {
+                          int causal, float scale, float scale_log2) {
   const int64_t head = blockIdx.y;
-  if (!head_selected(flags, head, select)) return;
   __shared__ __align__(16) float Qs[kBwdTile][D];
   __shared__ __align__(16) float Ds[kBwdTile][D];
   __shared__ float Ls[kBwdTile];
@@ -293,10 +291,8 @@ attn_bwd_dq_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
                         const T* __restrict__ v, const T* __restrict__ dout,
                         const float* __restrict__ lse, const float* __restrict__ delta,
                         T* __restrict__ dq, int64_t N, int64_t dstride, int causal,
-                        float scale, float scale_log2, const int* __restrict__ flags,
-                        int select) {
+                        float scale, float scale_log2) {
   const int64_t head = blockIdx.y;
-  if (!head_selected(flags, head, select)) return;
   __shared__ __align__(16) float Ks[kBwdTile][D];
   __shared__ __align__(16) float Vs[kBwdTile][D];
 
@@ -379,31 +375,180 @@ scan_nonfinite_kernel(const uint4* __restrict__ x, int64_t total_vec, int64_t ve
   }
 }
 
+// Per-head information of a bf16 attention call: four int32 per head h
+// (zeroed first), info[4h + 0] bit 0 = V holds an infinity or NaN, bit 1 =
+// dout does; info[4h + 1], [4h + 2], [4h + 3] = the largest biased exponent
+// of the finite values of V, of Q and K, and of dout.
+
+// bf16x8 helpers: the largest biased exponent among the finite values, and
+// whether any value is +-inf or NaN.
+__device__ __forceinline__ unsigned maxexp8(const uint4& u) {
+  const unsigned w[4] = {u.x, u.y, u.z, u.w};
+  unsigned m = 0u;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const unsigned lo = (w[e] >> 7) & 0xFFu, hi = (w[e] >> 23) & 0xFFu;
+    m = max(m, lo == 0xFFu ? 0u : lo);
+    m = max(m, hi == 0xFFu ? 0u : hi);
+  }
+  return m;
+}
+__device__ __forceinline__ bool nonfinite8(const uint4& u) {
+  const unsigned w[4] = {u.x, u.y, u.z, u.w};
+  bool bad = false;
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    bad |= ((w[e] & 0x7F80u) == 0x7F80u) | ((w[e] & 0x7F800000u) == 0x7F800000u);
+  return bad;
+}
+// bf16x8 -> f16x8, round to nearest even (infinities and NaN keep their class).
+__device__ __forceinline__ uint4 to_f16x8(const uint4& u) {
+  const unsigned w[4] = {u.x, u.y, u.z, u.w};
+  unsigned r[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xFFFF0000u);
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r[e]) : "f"(hi), "f"(lo));
+  }
+  return make_uint4(r[0], r[1], r[2], r[3]);
+}
+__device__ __forceinline__ float dot8(const uint4& a, const uint4& b) {
+  const unsigned x[4] = {a.x, a.y, a.z, a.w}, y[4] = {b.x, b.y, b.z, b.w};
+  float acc = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    acc = fmaf(__uint_as_float(x[e] << 16), __uint_as_float(y[e] << 16), acc);
+    acc = fmaf(__uint_as_float(x[e] & 0xFFFF0000u), __uint_as_float(y[e] & 0xFFFF0000u), acc);
+  }
+  return acc;
+}
+
+// Block-level reduction of the four info fields of one head, then one
+// global atomic per field.
+__device__ __forceinline__ void flush_info(unsigned fl, unsigned ve, unsigned qke, unsigned de,
+                                           int* info_h, unsigned* sh) {
+  fl = __reduce_or_sync(0xffffffffu, fl);
+  ve = __reduce_max_sync(0xffffffffu, ve);
+  qke = __reduce_max_sync(0xffffffffu, qke);
+  de = __reduce_max_sync(0xffffffffu, de);
+  if ((threadIdx.x & 31) == 0) {
+    atomicOr(&sh[0], fl);
+    atomicMax(&sh[1], ve);
+    atomicMax(&sh[2], qke);
+    atomicMax(&sh[3], de);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (sh[0]) atomicOr(&info_h[0], (int)sh[0]);
+    if (sh[1]) atomicMax(&info_h[1], (int)sh[1]);
+    if (sh[2]) atomicMax(&info_h[2], (int)sh[2]);
+    if (sh[3]) atomicMax(&info_h[3], (int)sh[3]);
+  }
+}
+
+// Forward scan of V: info fields 0 (bit 0) and 1.  Grid (x: blocks over the
+// head's 16-byte vectors, y: head).
+__global__ void __launch_bounds__(256)
+scan_v_info_kernel(const uint4* __restrict__ v, int64_t vec_per_head, int* __restrict__ info) {
+  __shared__ unsigned sh[4];
+  if (threadIdx.x < 4) sh[threadIdx.x] = 0u;
+  __syncthreads();
+  const int64_t head = blockIdx.y;
+  const uint4* vh = v + head * vec_per_head;
+  unsigned nonfinite = 0u, maxexp = 0u;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < vec_per_head;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 u = vh[idx];
+    nonfinite |= nonfinite8(u) ? 1u : 0u;
+    maxexp = max(maxexp, maxexp8(u));
+  }
+  flush_info(nonfinite, maxexp, 0u, 0u, info + 4 * head, sh);
+}
+
+// Prep pass of the bf16 backward.  8 threads per row (16 bytes of each
+// tensor per thread) over the padded rows [BH][Npad] (Npad = N rounded up to
+// 128), 128 rows per block, so a block never spans two heads:
+//   * f16 copies (round to nearest even; exact below 2^15 in magnitude) of
+//     q, k, v and, when given, dout -- the operands of the f16 instance;
+//   * when `out` is given: delta = sum_d dout_d out_d and nlse2 = -lse log2 e
+//     (padding rows: 0 and -inf);
+//   * the per-head info (all four fields; dout's only when dout is given).
+constexpr int kConvRows = 128;
+__global__ void __launch_bounds__(256)
+attn_convert_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
+                    const uint4* __restrict__ v, const uint4* __restrict__ dout,
+                    const uint4* __restrict__ out, const float* __restrict__ lse,
+                    uint4* __restrict__ q16, uint4* __restrict__ k16, uint4* __restrict__ v16,
+                    uint4* __restrict__ do16, float* __restrict__ delta,
+                    float* __restrict__ nlse2, int* __restrict__ info, int64_t N, int64_t Npad) {
+  __shared__ unsigned sh[4];
+  if (threadIdx.x < 4) sh[threadIdx.x] = 0u;
+  __syncthreads();
+  const int64_t rp0 = (int64_t)blockIdx.x * kConvRows;
+  const int64_t head = rp0 / Npad;
+  const int part = threadIdx.x & 7;
+  unsigned fl = 0u, ve = 0u, qke = 0u, de = 0u;
+#pragma unroll 1
+  for (int it = 0; it < kConvRows / 32; ++it) {
+    const int64_t rp = rp0 + it * 32 + (threadIdx.x >> 3);
+    const int64_t i = rp - head * Npad;
+    const bool real = i < N;
+    float acc = 0.f;
+    if (real) {
+      const int64_t vec = (head * N + i) * 8 + part;
+      uint4 x = q[vec];
+      q16[vec] = to_f16x8(x);
+      qke = max(qke, maxexp8(x));
+      x = k[vec];
+      k16[vec] = to_f16x8(x);
+      qke = max(qke, maxexp8(x));
+      x = v[vec];
+      v16[vec] = to_f16x8(x);
+      ve = max(ve, maxexp8(x));
+      fl |= nonfinite8(x) ? 1u : 0u;
+      if (dout != nullptr) {
+        x = dout[vec];
+        do16[vec] = to_f16x8(x);
+        de = max(de, maxexp8(x));
+        fl |= nonfinite8(x) ? 2u : 0u;
+        if (out != nullptr) acc = dot8(x, out[vec]);
+      }
+    }
+    if (out != nullptr) {
+      acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      if (part == 0) {
+        delta[rp] = real ? acc : 0.f;
+        nlse2[rp] = real ? -lse[head * N + i] * kLog2e : -INFINITY;
+      }
+    }
+  }
+  flush_info(fl, ve, qke, de, info + 4 * head, sh);
+}
+
 template <typename T>
 cudaError_t fwd_simt(const void* q, const void* k, const void* v, void* out, float* lse,
-                     int64_t BH, int64_t N, int causal, float scale, const int* flags,
-                     int select, cudaStream_t s) {
+                     int64_t BH, int64_t N, int causal, float scale, cudaStream_t s) {
   dim3 grid((unsigned)((N + kFwdRows - 1) / kFwdRows), (unsigned)BH);
   attn_fwd_simt_kernel<T><<<grid, kFwdRows, 0, s>>>(
-      (const T*)q, (const T*)k, (const T*)v, (T*)out, lse, N, causal, scale * kLog2e, flags,
-      select);
+      (const T*)q, (const T*)k, (const T*)v, (T*)out, lse, N, causal, scale * kLog2e);
   return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t bwd_simt(const void* q, const void* k, const void* v, const void* dout,
                      const float* lse, const float* delta, int64_t dstride, void* dq, void* dk,
-                     void* dv, int64_t BH, int64_t N, int causal, float scale, const int* flags,
-                     int select, cudaStream_t s) {
+                     void* dv, int64_t BH, int64_t N, int causal, float scale, cudaStream_t s) {
   dim3 grid((unsigned)((N + kBwdRows - 1) / kBwdRows), (unsigned)BH);
   attn_bwd_dkdv_simt_kernel<T><<<grid, 2 * kBwdRows, 0, s>>>(
       (const T*)q, (const T*)k, (const T*)v, (const T*)dout, lse, delta, (T*)dk, (T*)dv, N,
-      dstride, causal, scale, scale * kLog2e, flags, select);
+      dstride, causal, scale, scale * kLog2e);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   attn_bwd_dq_simt_kernel<T><<<grid, 2 * kBwdRows, 0, s>>>(
       (const T*)q, (const T*)k, (const T*)v, (const T*)dout, lse, delta, (T*)dq, N, dstride,
-      causal, scale, scale * kLog2e, flags, select);
+      causal, scale, scale * kLog2e);
   return cudaGetLastError();
 }
 
@@ -428,14 +573,38 @@ cudaError_t launch_scan_nonfinite(swa_dtype dt, const void* x, int64_t heads,
   return cudaGetLastError();
 }
 
+cudaError_t launch_scan_v_info(const void* v, int64_t heads, int64_t elems_per_head,
+                               int* info, cudaStream_t s, int* launches) {
+  const int64_t vec_per_head = elems_per_head * 2 / 16;
+  int64_t bx = (vec_per_head + 256 * 4 - 1) / (256 * 4);  // about four vectors per thread
+  if (bx > 1024) bx = 1024;
+  if (bx < 1) bx = 1;
+  dim3 grid((unsigned)bx, (unsigned)heads);
+  scan_v_info_kernel<<<grid, 256, 0, s>>>((const uint4*)v, vec_per_head, info);
+  *launches += 1;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_convert(const void* q, const void* k, const void* v, const void* dout,
+                                const void* out, const float* lse, void* q16, void* k16,
+                                void* v16, void* do16, float* delta, float* nlse2, int* info,
+                                int64_t BH, int64_t N, cudaStream_t s, int* launches) {
+  const int64_t Npad = pad128(N);
+  const int64_t blocks = BH * Npad / kConvRows;
+  attn_convert_kernel<<<(unsigned)blocks, 256, 0, s>>>(
+      (const uint4*)q, (const uint4*)k, (const uint4*)v, (const uint4*)dout, (const uint4*)out,
+      lse, (uint4*)q16, (uint4*)k16, (uint4*)v16, (uint4*)do16, delta, nlse2, info, N, Npad);
+  *launches += 1;
+  return cudaGetLastError();
+}
+
 cudaError_t launch_attn_fwd_simt(swa_dtype dt, const void* q, const void* k, const void* v,
                                  void* out, float* lse, int64_t BH, int64_t N, int causal,
-                                 float scale, const int* flags, int select, cudaStream_t s,
-                                 int* launches) {
+                                 float scale, cudaStream_t s, int* launches) {
   *launches += 1;
   if (dt == SWA_BF16)
-    return fwd_simt<__nv_bfloat16>(q, k, v, out, lse, BH, N, causal, scale, flags, select, s);
-  return fwd_simt<float>(q, k, v, out, lse, BH, N, causal, scale, flags, select, s);
+    return fwd_simt<__nv_bfloat16>(q, k, v, out, lse, BH, N, causal, scale, s);
+  return fwd_simt<float>(q, k, v, out, lse, BH, N, causal, scale, s);
 }
 
 cudaError_t launch_attn_bwd_prep(swa_dtype dt, const void* out, const void* dout,
@@ -457,14 +626,14 @@ cudaError_t launch_attn_bwd_prep(swa_dtype dt, const void* out, const void* dout
 cudaError_t launch_attn_bwd_simt(swa_dtype dt, const void* q, const void* k, const void* v,
                                  const void* dout, const float* lse, const float* delta,
                                  int64_t dstride, void* dq, void* dk, void* dv, int64_t BH,
-                                 int64_t N, int causal, float scale, const int* flags, int select,
-                                 cudaStream_t s, int* launches) {
+                                 int64_t N, int causal, float scale, cudaStream_t s,
+                                 int* launches) {
   *launches += 2;
   if (dt == SWA_BF16)
     return bwd_simt<__nv_bfloat16>(q, k, v, dout, lse, delta, dstride, dq, dk, dv, BH, N, causal,
-                                   scale, flags, select, s);
+                                   scale, s);
   return bwd_simt<float>(q, k, v, dout, lse, delta, dstride, dq, dk, dv, BH, N, causal, scale,
-                         flags, select, s);
+                         s);
 }
 
 }  // namespace swa

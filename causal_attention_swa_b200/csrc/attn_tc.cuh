@@ -1,6 +1,6 @@
 // attn_tc.cuh -- launchers of the tensor-core (tcgen05) attention kernels.
-// They handle only the heads whose flag is 0 (V, and for the backward dout,
-// all finite); the pair-by-pair kernels take the others.
+// They take every head of a bf16 call; heads whose V (or, in the backward,
+// dout) holds an infinity or NaN get the kernels' non-finite handling.
 #pragma once
 
 #include <cuda.h>
@@ -9,24 +9,56 @@
 
 namespace swa {
 
-// [BH][N][64] bf16 as a 3-D TMA tensor map (64, N, BH) with 64 x box_rows x 1
-// boxes and 128-byte swizzle; rows past N read as zeros.
+// [BH][N][64] of a 16-bit type (bf16 or f16: the copy does not convert) as
+// a 3-D TMA tensor map (64, N, BH) with 64 x box_rows x 1 boxes and 128-byte
+// swizzle; rows past N read as zeros.
 cudaError_t make_tmap_bf16_rows(CUtensorMap* map, const void* base, int64_t BH, int64_t N,
                                 int box_rows);
 
+// What the forward saves for the backward of loss = 1/2 sum out^2 (all
+// null for a plain forward): do16 [BH][N][64] f16 copy of out; delta and
+// nlse2 [BH][Npad] float32 (sum_d out_d^2 and -lse log2 e; padding rows 0
+// and -inf).
+struct FwdSaved {
+  void* do16 = nullptr;
+  float* delta = nullptr;
+  float* nlse2 = nullptr;
+};
+
+// vinfo: the per-head V information of launch_scan_v_info.  Two launches
+// (f16-operand and bf16-operand instances; each takes the heads of its type).
 cudaError_t launch_attn_fwd_tc(const void* q, const void* k, const void* v, void* out,
                                float* lse, int64_t B, int64_t H, int64_t N, int causal,
-                               float scale, const int* flags, unsigned* err, cudaStream_t s,
-                               int* launches);
+                               float scale, const int* vinfo, const FwdSaved& saved,
+                               unsigned* err, cudaStream_t s, int* launches);
 
-// Backward of the finite heads: a key-major kernel writes dk and dv, a
-// query-major kernel writes dq (both directly in bf16, no accumulator in
-// memory).  nlse2 = -lse * log2 e and delta are the prep kernel's [BH][Npad]
-// arrays.
-cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* dout,
+// The four 16-bit operand tensors of a backward instance, [BH][N][64] each.
+struct BwdOperands {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* dout;
+};
+
+// Backward: a key-major kernel writes dk and dv, a query-major kernel writes
+// dq (both directly in bf16, no accumulator in memory); f16-operand heads
+// read `f16` (copies), the others `bf16`.  Four launches.  nlse2 = -lse *
+// log2 e and delta are [BH][Npad] float32; info holds four int32 per head
+// (non-finite flags of V and dout, largest exponents of V, Q/K and dout).
+cudaError_t launch_attn_bwd_tc(const BwdOperands& f16, const BwdOperands& bf16,
                                const float* nlse2, const float* delta, void* dq, void* dk,
                                void* dv, int64_t B, int64_t H, int64_t N, int causal,
-                               float scale, const int* flags, unsigned* err, cudaStream_t s,
+                               float scale, const int* info, unsigned* err, cudaStream_t s,
                                int* launches);
+
+}  // namespace swa
+
+namespace swa {
+
+// q, k, v [B][H][N][64] bf16 = x [B*N][C] times the rows of w [3*H*64][C]
+// (q's features, then k's, then v's); C a multiple of 64.  One launch.
+cudaError_t launch_qkv_proj(const void* x, const void* w, void* q, void* k, void* v, int64_t B,
+                            int64_t N, int64_t C, int64_t H, unsigned* err, cudaStream_t s,
+                            int* launches);
 
 }  // namespace swa

@@ -3,7 +3,9 @@
 // "Show HN: Automatic deduction of FlashAttention kernel from ~25 lines of
 // SQL", query NADARAYA_WATSON: w_pq = exp(-((tx-sx)^2 + (ty-sy)^2) / h^2)
 // ("bandwidth h = 0.5", divisor 0.25), out_p = sum_q w_pq v_q / sum_q w_pq.
-// Every weight is <= 1, so no running max is needed.
+// Every weight is <= 1, so no running max is needed.  The kernels take
+// points of DIMS = 1, 2 or 3 coordinates (the squared distance summed over
+// them); the pages' points, and the benchmark's, have two.
 //
 // Work split: the (targets x sources) pair grid is cut into target tiles of
 // kTargetsPerBlock (kPerThread targets per thread, kept in registers) and
@@ -13,9 +15,12 @@
 // coordinates, so each pair costs 2 FADD, FMUL, FFMA, one MUFU ex2 (with the
 // sign folded into its operand), FADD and FFMA -- the FP32 steps issued two
 // targets at a time as packed f32x2 instructions (bitwise the same sums),
-// which leaves MUFU as the one limit.  Partial (sum w, sum w v)
-// per (chunk, target) go to a float2 workspace; a second kernel adds them in
-// chunk order (deterministic) and divides.  0/0 gives NaN.
+// which leaves MUFU as the one limit.  A chunk longer than the shared-memory
+// stage (2048 sources) is staged in turns, so any S fits the grid.  Partial
+// (sum w, sum w v) per (chunk, target) go to a float2 workspace; a second
+// kernel adds them in a fixed order (deterministic) and divides: eight
+// threads per target each add every eighth chunk, then the eight sums are
+// added in order.  0/0 gives NaN.
 #include "swa_internal.cuh"
 
 namespace swa {
@@ -25,7 +30,8 @@ constexpr int kThreads = 256;
 constexpr int kPerThread = 8;
 constexpr int kTargetsPerBlock = kThreads * kPerThread;
 constexpr int kTargetBlocks = 148 * 8;   // blocks the grid aims for (SMs x resident blocks)
-constexpr int kMaxChunk = 2048;          // sources per block (32 KB of shared memory)
+constexpr int kStage = 2048;             // sources staged at a time (32 KB of shared memory)
+constexpr int64_t kMaxChunks = 65535;    // grid.y limit
 
 __device__ __forceinline__ float ex2_neg(float x) {
   float y;
@@ -33,48 +39,61 @@ __device__ __forceinline__ float ex2_neg(float x) {
   return y;
 }
 
+template <int DIMS>
 __global__ void __launch_bounds__(kThreads)
 nw_partial_kernel(const float* __restrict__ targets, int64_t M,
                   const float* __restrict__ sources, const float* __restrict__ vals,
                   int64_t S, float c, int64_t chunk, float2* __restrict__ partials) {
+  static_assert(DIMS >= 1 && DIMS <= 3, "1 to 3 coordinates");
   extern __shared__ float4 src[];
   const int tid = threadIdx.x;
-  const int64_t s0 = (int64_t)blockIdx.y * chunk;
-  const int ns = (int)imin64(chunk, S - s0);
-  for (int e = tid; e < ns; e += kThreads) {
-    const float2 xy = reinterpret_cast<const float2*>(sources)[s0 + e];
-    src[e] = make_float4(-(xy.x * c), -(xy.y * c), vals[s0 + e], 0.f);
-  }
-  __syncthreads();
+  const int64_t c0 = (int64_t)blockIdx.y * chunk;
+  const int64_t c1 = imin64(c0 + chunk, S);
 
   // targets in pairs: lane .x of pair u is target 2u, lane .y target 2u + 1
   constexpr int kPairs = kPerThread / 2;
-  float2 tx[kPairs], ty[kPairs], sw[kPairs], swv[kPairs];
+  float2 tc[DIMS][kPairs], sw[kPairs], swv[kPairs];
   const int64_t p0 = (int64_t)blockIdx.x * kTargetsPerBlock + tid;
 #pragma unroll
   for (int u = 0; u < kPairs; ++u) {
-    float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
     const int64_t pa = p0 + (int64_t)(2 * u) * kThreads, pb = pa + kThreads;
-    if (pa < M) a = reinterpret_cast<const float2*>(targets)[pa];
-    if (pb < M) b = reinterpret_cast<const float2*>(targets)[pb];
-    tx[u] = make_float2(a.x * c, b.x * c);
-    ty[u] = make_float2(a.y * c, b.y * c);
+#pragma unroll
+    for (int d = 0; d < DIMS; ++d)
+      tc[d][u] = make_float2(pa < M ? targets[pa * DIMS + d] * c : 0.f,
+                             pb < M ? targets[pb * DIMS + d] * c : 0.f);
     sw[u] = make_float2(0.f, 0.f);
     swv[u] = make_float2(0.f, 0.f);
   }
-#pragma unroll 4
-  for (int e = 0; e < ns; ++e) {
-    const float4 sv = src[e];
-    const float2 nsx = make_float2(sv.x, sv.x), nsy = make_float2(sv.y, sv.y);
-    const float2 v2 = make_float2(sv.z, sv.z);
+  for (int64_t s0 = c0; s0 < c1; s0 += kStage) {
+    const int ns = (int)imin64(kStage, c1 - s0);
+    if (s0 != c0) __syncthreads();  // the previous stage is no longer read
+    for (int e = tid; e < ns; e += kThreads) {
+      // (-s c per coordinate, then v): the value sits right after the coordinates
+      float f[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int u = 0; u < kPairs; ++u) {
-      const float2 dx = __fadd2_rn(tx[u], nsx);
-      const float2 dy = __fadd2_rn(ty[u], nsy);
-      const float2 d2 = __ffma2_rn(dy, dy, __fmul2_rn(dx, dx));
-      const float2 w = make_float2(ex2_neg(d2.x), ex2_neg(d2.y));
-      sw[u] = __fadd2_rn(sw[u], w);
-      swv[u] = __ffma2_rn(w, v2, swv[u]);
+      for (int d = 0; d < DIMS; ++d) f[d] = -(sources[(s0 + e) * DIMS + d] * c);
+      f[DIMS] = vals[s0 + e];
+      src[e] = make_float4(f[0], f[1], f[2], f[3]);
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int e = 0; e < ns; ++e) {
+      const float4 sv = src[e];
+      const float sf[4] = {sv.x, sv.y, sv.z, sv.w};
+      const float2 v2 = make_float2(sf[DIMS], sf[DIMS]);
+#pragma unroll
+      for (int u = 0; u < kPairs; ++u) {
+        // squared scaled distance: (t0 - s0)^2 first, then + (t_d - s_d)^2
+        float2 d2;
+#pragma unroll
+        for (int d = 0; d < DIMS; ++d) {
+          const float2 dd = __fadd2_rn(tc[d][u], make_float2(sf[d], sf[d]));
+          d2 = d == 0 ? __fmul2_rn(dd, dd) : __ffma2_rn(dd, dd, d2);
+        }
+        const float2 w = make_float2(ex2_neg(d2.x), ex2_neg(d2.y));
+        sw[u] = __fadd2_rn(sw[u], w);
+        swv[u] = __ffma2_rn(w, v2, swv[u]);
+      }
     }
   }
 #pragma unroll
@@ -85,18 +104,37 @@ nw_partial_kernel(const float* __restrict__ targets, int64_t M,
   }
 }
 
-__global__ void __launch_bounds__(256)
+// Block = 32 targets x 8 chunk groups: thread (g, t) adds chunks g, g + 8,
+// ... of target t (32 consecutive targets per chunk: coalesced 256-byte
+// reads), then thread (0, t) adds the eight group sums in order.
+constexpr int kFinTargets = 32;
+constexpr int kFinGroups = 8;
+__global__ void __launch_bounds__(kFinTargets * kFinGroups)
 nw_finalize_kernel(const float2* __restrict__ partials, int nchunks, int64_t M,
                    float* __restrict__ out) {
-  const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (p >= M) return;
-  float sw = 0.f, swv = 0.f;
-  for (int ch = 0; ch < nchunks; ++ch) {
-    const float2 a = partials[(int64_t)ch * M + p];
-    sw += a.x;
-    swv += a.y;
+  __shared__ float2 part[kFinGroups][kFinTargets];
+  const int t = threadIdx.x % kFinTargets, g = threadIdx.x / kFinTargets;
+  const int64_t p = (int64_t)blockIdx.x * kFinTargets + t;
+  float2 acc = make_float2(0.f, 0.f);
+  if (p < M) {
+#pragma unroll 4
+    for (int ch = g; ch < nchunks; ch += kFinGroups) {
+      const float2 a = partials[(int64_t)ch * M + p];
+      acc.x += a.x;
+      acc.y += a.y;
+    }
   }
-  out[p] = swv / sw;
+  part[g][t] = acc;
+  __syncthreads();
+  if (g == 0 && p < M) {
+    float sw = 0.f, swv = 0.f;
+#pragma unroll
+    for (int i = 0; i < kFinGroups; ++i) {
+      sw += part[i][t].x;
+      swv += part[i][t].y;
+    }
+    out[p] = swv / sw;
+  }
 }
 
 struct Plan {
@@ -109,7 +147,9 @@ Plan plan(int64_t M, int64_t S) {
   int64_t want = (kTargetBlocks + pl.mtiles - 1) / pl.mtiles;
   if (want < 1) want = 1;
   int64_t chunk = (S + want - 1) / want;
-  if (chunk > kMaxChunk) chunk = kMaxChunk;
+  if (chunk > kStage) chunk = kStage;         // one stage per block when S allows
+  const int64_t min_chunk = (S + kMaxChunks - 1) / kMaxChunks;
+  if (chunk < min_chunk) chunk = min_chunk;   // else several stages: grid.y <= 65535
   if (chunk < 1) chunk = 1;
   pl.chunk = chunk;
   pl.nchunks = (S + chunk - 1) / chunk;
@@ -124,14 +164,22 @@ size_t nw_partials_bytes(int64_t M, int64_t S) {
 }
 
 cudaError_t launch_nw_partial(const float* targets, int64_t M, const float* sources,
-                              const float* vals, int64_t S, float h, float* partials,
+                              const float* vals, int64_t S, int dims, float h, float* partials,
                               cudaStream_t s, int* launches) {
   const Plan pl = plan(M, S);
   const float c = sqrtf(kLog2e) / h;
   dim3 grid((unsigned)pl.mtiles, (unsigned)pl.nchunks);
-  const size_t smem = (size_t)pl.chunk * sizeof(float4);
-  nw_partial_kernel<<<grid, kThreads, smem, s>>>(targets, M, sources, vals, S, c, pl.chunk,
-                                                 reinterpret_cast<float2*>(partials));
+  const size_t smem = (size_t)imin64(pl.chunk, kStage) * sizeof(float4);
+  float2* part = reinterpret_cast<float2*>(partials);
+  if (dims == 1)
+    nw_partial_kernel<1><<<grid, kThreads, smem, s>>>(targets, M, sources, vals, S, c, pl.chunk,
+                                                      part);
+  else if (dims == 2)
+    nw_partial_kernel<2><<<grid, kThreads, smem, s>>>(targets, M, sources, vals, S, c, pl.chunk,
+                                                      part);
+  else
+    nw_partial_kernel<3><<<grid, kThreads, smem, s>>>(targets, M, sources, vals, S, c, pl.chunk,
+                                                      part);
   *launches += 1;
   return cudaGetLastError();
 }
@@ -139,7 +187,8 @@ cudaError_t launch_nw_partial(const float* targets, int64_t M, const float* sour
 cudaError_t launch_nw_finalize(int64_t M, int64_t S, const float* partials, float* out,
                                cudaStream_t s, int* launches) {
   const Plan pl = plan(M, S);
-  nw_finalize_kernel<<<(unsigned)((M + 255) / 256), 256, 0, s>>>(
+  nw_finalize_kernel<<<(unsigned)((M + kFinTargets - 1) / kFinTargets),
+                       kFinTargets * kFinGroups, 0, s>>>(
       reinterpret_cast<const float2*>(partials), (int)pl.nchunks, M, out);
   *launches += 1;
   return cudaGetLastError();

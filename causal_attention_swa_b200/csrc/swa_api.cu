@@ -93,23 +93,52 @@ swa_status check_attn_shape(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtyp
   return SWA_OK;
 }
 
+// Forward workspace (bf16): the per-head information of the scan of V.
 size_t fwd_ws(int64_t B, int64_t H, swa_dtype dt) {
-  return dt == SWA_BF16 ? round_up((size_t)(B * H) * sizeof(int), 256) : 0;
+  return dt == SWA_BF16 ? round_up((size_t)(B * H) * swa::kHeadInfoInts * sizeof(int), 256) : 0;
 }
 
-// Backward workspace: per-head flags | delta [BH][Npad] | -lse*log2e [BH][Npad];
-// Npad = N rounded up to 128.
+// Backward (and gradient) workspace, in this order:
+//   info   [BH][4] int32        per-head information
+//   delta  [BH][Npad] float32   dout . out per row (Npad = N rounded up to 128)
+//   nlse2  [BH][Npad] float32   -lse log2 e per row
+//   q16, k16, v16, do16  [BH][N][64] f16 each (bf16 only): the f16 operands
 struct BwdWs {
-  size_t flags, delta, nlse2, total;
+  size_t info, delta, nlse2, copy, total;
 };
 
 BwdWs bwd_ws(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtype dt) {
   BwdWs w;
-  w.flags = round_up((size_t)(B * H) * sizeof(int), 256);
+  w.info = round_up((size_t)(B * H) * swa::kHeadInfoInts * sizeof(int), 256);
   w.delta = round_up((size_t)(B * H * swa::pad128(N)) * sizeof(float), 256);
   w.nlse2 = w.delta;
-  w.total = w.flags + w.delta + w.nlse2;
+  w.copy = dt == SWA_BF16 ? round_up((size_t)(B * H * N * D) * 2, 256) : 0;
+  w.total = w.info + w.delta + w.nlse2 + 4 * w.copy;
   return w;
+}
+
+struct BwdPtrs {
+  int* info;
+  float* delta;
+  float* nlse2;
+  void* q16;
+  void* k16;
+  void* v16;
+  void* do16;
+};
+
+BwdPtrs carve(void* workspace, const BwdWs& w) {
+  char* b = static_cast<char*>(workspace);
+  BwdPtrs p;
+  p.info = reinterpret_cast<int*>(b);
+  p.delta = reinterpret_cast<float*>(b + w.info);
+  p.nlse2 = reinterpret_cast<float*>(b + w.info + w.delta);
+  char* c = b + w.info + w.delta + w.nlse2;
+  p.q16 = c;
+  p.k16 = c + w.copy;
+  p.v16 = c + 2 * w.copy;
+  p.do16 = c + 3 * w.copy;
+  return p;
 }
 
 }  // namespace
@@ -159,26 +188,23 @@ swa_status swa_attn_fwd(const void* q, const void* k, const void* v, void* out, 
   int launches = 0;
   cudaError_t e;
   if (dt == SWA_F32) {
-    e = swa::launch_attn_fwd_simt(dt, q, k, v, out, lse, BH, N, causal ? 1 : 0, scale, nullptr,
-                                  0, s, &launches);
+    e = swa::launch_attn_fwd_simt(dt, q, k, v, out, lse, BH, N, causal ? 1 : 0, scale, s,
+                                  &launches);
     if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_simt");
   } else {
-    int* flags = static_cast<int*>(workspace);
-    e = cudaMemsetAsync(flags, 0, (size_t)BH * sizeof(int), s);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(flags)");
-    e = swa::launch_scan_nonfinite(dt, v, BH, N * D, flags, s, &launches);
-    if (e != cudaSuccess) return cuda_fail(e, "scan_nonfinite(v)");
-    // Heads whose V is all finite: tensor-core kernel.  Heads holding a
-    // non-finite value: the pair-by-pair kernel, so masked pairs stay absent.
+    // per-head V information (non-finite values, range), then the
+    // tensor-core kernel for every head
+    int* vinfo = static_cast<int*>(workspace);
+    e = cudaMemsetAsync(vinfo, 0, (size_t)BH * swa::kHeadInfoInts * sizeof(int), s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(vinfo)");
+    e = swa::launch_scan_v_info(v, BH, N * D, vinfo, s, &launches);
+    if (e != cudaSuccess) return cuda_fail(e, "scan_v_info");
     {
       ProfScope ps(SWA_KERNEL_ATTN_FWD, s);
-      e = swa::launch_attn_fwd_tc(q, k, v, out, lse, B, H, N, causal ? 1 : 0, scale, flags, err,
-                                  s, &launches);
+      e = swa::launch_attn_fwd_tc(q, k, v, out, lse, B, H, N, causal ? 1 : 0, scale, vinfo,
+                                  swa::FwdSaved{}, err, s, &launches);
     }
     if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_tc");
-    e = swa::launch_attn_fwd_simt(dt, q, k, v, out, lse, BH, N, causal ? 1 : 0, scale, flags,
-                                  1, s, &launches);
-    if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_simt(non-finite heads)");
   }
   t_launches = launches;
   return SWA_OK;
@@ -210,38 +236,105 @@ swa_status swa_attn_bwd(const void* q, const void* k, const void* v, const void*
   const float scale = 1.0f / sqrtf((float)D);
   unsigned* err = device_error_word(&st);
   if (!err) return st;
-  char* base = static_cast<char*>(workspace);
-  int* flags = reinterpret_cast<int*>(base);
-  float* delta = reinterpret_cast<float*>(base + ws.flags);
-  float* nlse2 = reinterpret_cast<float*>(base + ws.flags + ws.delta);
+  const BwdPtrs w = carve(workspace, ws);
   const int64_t Npad = swa::pad128(N);
   const int c = causal ? 1 : 0;
   int launches = 0;
-  cudaError_t e = swa::launch_attn_bwd_prep(dt, out, dout, lse, delta, nlse2, BH, N, Npad, s,
-                                            &launches);
-  if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_prep");
+  cudaError_t e;
   if (dt == SWA_F32) {
-    e = swa::launch_attn_bwd_simt(dt, q, k, v, dout, lse, delta, Npad, dq, dk, dv, BH, N, c,
-                                  scale, nullptr, 0, s, &launches);
+    e = swa::launch_attn_bwd_prep(dt, out, dout, lse, w.delta, w.nlse2, BH, N, Npad, s,
+                                  &launches);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_prep");
+    e = swa::launch_attn_bwd_simt(dt, q, k, v, dout, lse, w.delta, Npad, dq, dk, dv, BH, N, c,
+                                  scale, s, &launches);
     if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_simt");
   } else {
-    e = cudaMemsetAsync(flags, 0, (size_t)BH * sizeof(int), s);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(flags)");
-    e = swa::launch_scan_nonfinite(dt, v, BH, N * D, flags, s, &launches);
-    if (e != cudaSuccess) return cuda_fail(e, "scan_nonfinite(v)");
-    e = swa::launch_scan_nonfinite(dt, dout, BH, N * D, flags, s, &launches);
-    if (e != cudaSuccess) return cuda_fail(e, "scan_nonfinite(dout)");
-    // Heads with all-finite V and dout: tensor-core kernels (dk and dv
-    // key-major, dq query-major); the others: pair-by-pair kernels.
+    // prep: f16 operand copies, delta, -lse log2 e, per-head information;
+    // then the tensor-core kernels for every head (f16 or bf16 operands per
+    // head; the information switches on their non-finite handling)
+    e = cudaMemsetAsync(w.info, 0, (size_t)BH * swa::kHeadInfoInts * sizeof(int), s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(info)");
+    e = swa::launch_attn_convert(q, k, v, dout, out, lse, w.q16, w.k16, w.v16, w.do16, w.delta,
+                                 w.nlse2, w.info, BH, N, s, &launches);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_convert");
     {
       ProfScope ps(SWA_KERNEL_ATTN_BWD, s);
-      e = swa::launch_attn_bwd_tc(q, k, v, dout, nlse2, delta, dq, dk, dv, B, H, N, c, scale,
-                                  flags, err, s, &launches);
+      e = swa::launch_attn_bwd_tc(swa::BwdOperands{w.q16, w.k16, w.v16, w.do16},
+                                  swa::BwdOperands{q, k, v, dout}, w.nlse2, w.delta, dq, dk, dv,
+                                  B, H, N, c, scale, w.info, err, s, &launches);
     }
     if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_tc");
-    e = swa::launch_attn_bwd_simt(dt, q, k, v, dout, lse, delta, Npad, dq, dk, dv, BH, N, c,
-                                  scale, flags, 1, s, &launches);
-    if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_simt(non-finite heads)");
+  }
+  t_launches = launches;
+  return SWA_OK;
+}
+
+size_t swa_attn_grad_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtype dt) {
+  if (B < 1 || H < 1 || N < 1 || D < 1) return 0;
+  return bwd_ws(B, H, N, D, dt).total;
+}
+
+swa_status swa_attn_grad(const void* q, const void* k, const void* v, void* out, float* lse,
+                         void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N,
+                         int64_t D, int causal, swa_dtype dt, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  t_msg[0] = 0;
+  t_launches = 0;
+  swa_status st = check_attn_shape(B, H, N, D, dt);
+  if (st != SWA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return fail(SWA_ERR_INVALID_ARGUMENT,
+                "q, k, v, out, lse, dq, dk, dv must be non-null and 16-byte aligned");
+  const BwdWs ws = bwd_ws(B, H, N, D, dt);
+  if (!aligned16(workspace) || workspace_bytes < ws.total)
+    return fail(SWA_ERR_INVALID_ARGUMENT, "workspace must be 16-byte aligned and >= %zu bytes",
+                ws.total);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t BH = B * H;
+  const float scale = 1.0f / sqrtf((float)D);
+  unsigned* err = device_error_word(&st);
+  if (!err) return st;
+  const BwdPtrs w = carve(workspace, ws);
+  const int64_t Npad = swa::pad128(N);
+  const int c = causal ? 1 : 0;
+  int launches = 0;
+  cudaError_t e;
+  if (dt == SWA_F32) {
+    e = swa::launch_attn_fwd_simt(dt, q, k, v, out, lse, BH, N, c, scale, s, &launches);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_simt");
+    e = swa::launch_attn_bwd_prep(dt, out, out, lse, w.delta, w.nlse2, BH, N, Npad, s,
+                                  &launches);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_prep");
+    e = swa::launch_attn_bwd_simt(dt, q, k, v, out, lse, w.delta, Npad, dq, dk, dv, BH, N, c,
+                                  scale, s, &launches);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_simt");
+  } else {
+    // prep (f16 copies of q, k, v; per-head information), the forward --
+    // which also saves an f16 copy of out, delta = |out_i|^2 and -lse log2 e
+    // from its float32 accumulator -- and the backward with dout = out
+    e = cudaMemsetAsync(w.info, 0, (size_t)BH * swa::kHeadInfoInts * sizeof(int), s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(info)");
+    e = swa::launch_attn_convert(q, k, v, nullptr, nullptr, nullptr, w.q16, w.k16, w.v16,
+                                 nullptr, nullptr, nullptr, w.info, BH, N, s, &launches);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_convert");
+    swa::FwdSaved saved;
+    saved.do16 = w.do16;
+    saved.delta = w.delta;
+    saved.nlse2 = w.nlse2;
+    {
+      ProfScope ps(SWA_KERNEL_ATTN_FWD, s);
+      e = swa::launch_attn_fwd_tc(q, k, v, out, lse, B, H, N, c, scale, w.info, saved, err, s,
+                                  &launches);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_tc");
+    {
+      ProfScope ps(SWA_KERNEL_ATTN_BWD, s);
+      e = swa::launch_attn_bwd_tc(swa::BwdOperands{w.q16, w.k16, w.v16, w.do16},
+                                  swa::BwdOperands{q, k, v, out}, w.nlse2, w.delta, dq, dk, dv,
+                                  B, H, N, c, scale, w.info, err, s, &launches);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_tc");
   }
   t_launches = launches;
   return SWA_OK;
@@ -252,21 +345,33 @@ size_t swa_nw_workspace_size(int64_t M, int64_t S) {
   return round_up(swa::nw_partials_bytes(M, S), 256);
 }
 
-swa_status swa_nw_regrid(const float* targets, int64_t M, const float* sources,
-                         const float* vals, int64_t S, float h, float* out, void* workspace,
-                         size_t workspace_bytes, void* stream) {
-  t_msg[0] = 0;
-  t_launches = 0;
+namespace {
+
+swa_status check_nw(const float* targets, int64_t M, const float* sources, const float* vals,
+                    int64_t S, int dims, float h) {
   if (M < 1 || S < 1)
     return fail(SWA_ERR_INVALID_ARGUMENT, "M and S must be >= 1 (got %lld, %lld)", (long long)M,
                 (long long)S);
   if (M > ((int64_t)1 << 31) || S > ((int64_t)1 << 31))
     return fail(SWA_ERR_UNSUPPORTED, "M and S must be <= 2^31");
+  if (dims < 1 || dims > 3)
+    return fail(SWA_ERR_UNSUPPORTED, "points must have 1, 2 or 3 coordinates (got %d)", dims);
   if (!(h > 0.f) || !isfinite(h))
     return fail(SWA_ERR_INVALID_ARGUMENT, "bandwidth h must be finite and > 0");
-  if (!aligned16(targets) || !aligned16(sources) || !aligned16(vals) || !aligned16(out))
+  if (!aligned16(targets) || !aligned16(sources) || !aligned16(vals))
     return fail(SWA_ERR_INVALID_ARGUMENT,
-                "targets, sources, vals, out must be non-null and 16-byte aligned");
+                "targets, sources, vals must be non-null and 16-byte aligned");
+  return SWA_OK;
+}
+
+swa_status nw_forward(const float* targets, int64_t M, const float* sources, const float* vals,
+                      int64_t S, int dims, float h, float* out, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  t_msg[0] = 0;
+  t_launches = 0;
+  swa_status st = check_nw(targets, M, sources, vals, S, dims, h);
+  if (st != SWA_OK) return st;
+  if (!aligned16(out)) return fail(SWA_ERR_INVALID_ARGUMENT, "out must be non-null and 16-byte aligned");
   const size_t need = swa_nw_workspace_size(M, S);
   if (!aligned16(workspace) || workspace_bytes < need)
     return fail(SWA_ERR_INVALID_ARGUMENT, "workspace must be 16-byte aligned and >= %zu bytes",
@@ -275,13 +380,89 @@ swa_status swa_nw_regrid(const float* targets, int64_t M, const float* sources,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   {
-    ProfScope ps(SWA_KERNEL_NW, s);
-    e = swa::launch_nw_partial(targets, M, sources, vals, S, h, static_cast<float*>(workspace),
-                               s, &launches);
+    ProfScope ps(SWA_KERNEL_NW, s);  // the whole call: pair grid and final sum
+    e = swa::launch_nw_partial(targets, M, sources, vals, S, dims, h,
+                               static_cast<float*>(workspace), s, &launches);
+    if (e != cudaSuccess) return cuda_fail(e, "nw_partial");
+    e = swa::launch_nw_finalize(M, S, static_cast<const float*>(workspace), out, s, &launches);
   }
-  if (e != cudaSuccess) return cuda_fail(e, "nw_partial");
-  e = swa::launch_nw_finalize(M, S, static_cast<const float*>(workspace), out, s, &launches);
   if (e != cudaSuccess) return cuda_fail(e, "nw_finalize");
+  t_launches = launches;
+  return SWA_OK;
+}
+
+}  // namespace
+
+swa_status swa_nw_regrid(const float* targets, int64_t M, const float* sources,
+                         const float* vals, int64_t S, float h, float* out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  return nw_forward(targets, M, sources, vals, S, 2, h, out, workspace, workspace_bytes, stream);
+}
+
+swa_status swa_nw_regrid_nd(const float* targets, int64_t M, const float* sources,
+                            const float* vals, int64_t S, int dims, float h, float* out,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  return nw_forward(targets, M, sources, vals, S, dims, h, out, workspace, workspace_bytes,
+                    stream);
+}
+
+size_t swa_nw_regrid_bwd_workspace_size(int64_t M, int64_t S, int dims) {
+  if (M < 1 || S < 1 || dims < 1 || dims > 3) return 0;
+  return round_up(swa::nw_bwd_workspace_bytes(M, S), 256);
+}
+
+swa_status swa_nw_regrid_bwd(const float* targets, int64_t M, const float* sources,
+                             const float* vals, int64_t S, int dims, float h, const float* gout,
+                             float* dtargets, float* dsources, float* dvals, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  t_msg[0] = 0;
+  t_launches = 0;
+  swa_status st = check_nw(targets, M, sources, vals, S, dims, h);
+  if (st != SWA_OK) return st;
+  if (!aligned16(gout) || !aligned16(dtargets) || !aligned16(dsources) || !aligned16(dvals))
+    return fail(SWA_ERR_INVALID_ARGUMENT,
+                "gout, dtargets, dsources, dvals must be non-null and 16-byte aligned");
+  const size_t need = swa_nw_regrid_bwd_workspace_size(M, S, dims);
+  if (!aligned16(workspace) || workspace_bytes < need)
+    return fail(SWA_ERR_INVALID_ARGUMENT, "workspace must be 16-byte aligned and >= %zu bytes",
+                need);
+  int launches = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  {
+    ProfScope ps(SWA_KERNEL_NW_BWD, s);
+    e = swa::launch_nw_bwd(targets, M, sources, vals, S, dims, h, gout, dtargets, dsources, dvals,
+                           static_cast<float*>(workspace), s, &launches);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "nw_bwd");
+  t_launches = launches;
+  return SWA_OK;
+}
+
+swa_status swa_qkv_proj(const void* x, const void* w, void* q, void* k, void* v, int64_t B,
+                        int64_t N, int64_t C, int64_t H, int64_t D, swa_dtype dt, void* stream) {
+  t_msg[0] = 0;
+  t_launches = 0;
+  if (dt != SWA_BF16) return fail(SWA_ERR_UNSUPPORTED, "the projection takes bf16 only");
+  swa_status st = check_attn_shape(B, H, N, D, dt);
+  if (st != SWA_OK) return st;
+  if (C < 64 || C % 64 != 0)
+    return fail(SWA_ERR_UNSUPPORTED, "C must be a positive multiple of 64 (got %lld)",
+                (long long)C);
+  if (C > (1 << 20) || B * N > ((int64_t)1 << 31))
+    return fail(SWA_ERR_UNSUPPORTED, "C <= 2^20 and B*N <= 2^31 are supported");
+  if (!aligned16(x) || !aligned16(w) || !aligned16(q) || !aligned16(k) || !aligned16(v))
+    return fail(SWA_ERR_INVALID_ARGUMENT, "x, w, q, k, v must be non-null and 16-byte aligned");
+  unsigned* err = device_error_word(&st);
+  if (!err) return st;
+  int launches = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  {
+    ProfScope ps(SWA_KERNEL_QKV, s);
+    e = swa::launch_qkv_proj(x, w, q, k, v, B, N, C, H, err, s, &launches);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "qkv_proj");
   t_launches = launches;
   return SWA_OK;
 }

@@ -35,12 +35,6 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
   return __float2bfloat16_rn(x);
 }
 
-// Per-head selection: a kernel given `flags` handles head h only when
-// (flags[h] != 0) == select; with flags == nullptr it handles every head.
-__device__ __forceinline__ bool head_selected(const int* flags, int64_t head, int select) {
-  return flags == nullptr || ((flags[head] != 0) == (select != 0));
-}
-
 // ------------------------------------------------- shared C-ABI bookkeeping
 // (swa_api.cu): error message, argument checks, device error word and the
 // per-thread launch count, for entry points defined in other files.
@@ -59,10 +53,28 @@ cudaError_t launch_scan_nonfinite(swa_dtype dt, const void* x, int64_t heads,
                                   int64_t elems_per_head, int* flags, cudaStream_t s,
                                   int* launches);
 
+// Per-head information of a bf16 call: kHeadInfoInts int32 per head (zeroed
+// by the caller): [0] bit 0 = V holds an infinity or NaN, bit 1 = dout does;
+// [1], [2], [3] = the largest biased exponent of the finite values of V, of
+// Q and K, of dout.
+constexpr int kHeadInfoInts = 4;
+
+// Fills fields 0 (bit 0) and 1 from a scan of V (the forward's needs).
+cudaError_t launch_scan_v_info(const void* v, int64_t heads, int64_t elems_per_head,
+                               int* info, cudaStream_t s, int* launches);
+
+// The backward's prep pass over [BH][N][64] bf16 tensors: f16 copies of q,
+// k, v (and dout if non-null) into q16, k16, v16 (do16); with `out` non-null
+// (dout then too) delta = dout . out and nlse2 = -lse log2 e per row, [BH][Npad]
+// with padding rows 0 and -inf; the per-head info.
+cudaError_t launch_attn_convert(const void* q, const void* k, const void* v, const void* dout,
+                                const void* out, const float* lse, void* q16, void* k16,
+                                void* v16, void* do16, float* delta, float* nlse2, int* info,
+                                int64_t BH, int64_t N, cudaStream_t s, int* launches);
+
 cudaError_t launch_attn_fwd_simt(swa_dtype dt, const void* q, const void* k, const void* v,
                                  void* out, float* lse, int64_t BH, int64_t N, int causal,
-                                 float scale, const int* flags, int select, cudaStream_t s,
-                                 int* launches);
+                                 float scale, cudaStream_t s, int* launches);
 
 // delta[h][i] and nlse2[h][i] = -lse * log2 e, both [BH][Npad] (Npad = N
 // rounded up to 128; padding rows 0 and -inf).
@@ -73,14 +85,22 @@ cudaError_t launch_attn_bwd_prep(swa_dtype dt, const void* out, const void* dout
 cudaError_t launch_attn_bwd_simt(swa_dtype dt, const void* q, const void* k, const void* v,
                                  const void* dout, const float* lse, const float* delta,
                                  int64_t dstride, void* dq, void* dk, void* dv, int64_t BH,
-                                 int64_t N, int causal, float scale, const int* flags, int select,
-                                 cudaStream_t s, int* launches);
+                                 int64_t N, int causal, float scale, cudaStream_t s,
+                                 int* launches);
 
 size_t nw_partials_bytes(int64_t M, int64_t S);
+// targets [M, dims], sources [S, dims] (dims = 1, 2 or 3).
 cudaError_t launch_nw_partial(const float* targets, int64_t M, const float* sources,
-                              const float* vals, int64_t S, float h, float* partials,
+                              const float* vals, int64_t S, int dims, float h, float* partials,
                               cudaStream_t s, int* launches);
 cudaError_t launch_nw_finalize(int64_t M, int64_t S, const float* partials, float* out,
                                cudaStream_t s, int* launches);
+
+// Backward of the regrid (nw_grad.cu): workspace bytes and the four launches.
+size_t nw_bwd_workspace_bytes(int64_t M, int64_t S);
+cudaError_t launch_nw_bwd(const float* targets, int64_t M, const float* sources,
+                          const float* vals, int64_t S, int dims, float h, const float* gout,
+                          float* dtargets, float* dsources, float* dvals, float* ws,
+                          cudaStream_t s, int* launches);
 
 }  // namespace swa

@@ -5,18 +5,19 @@
 // host application owns every device allocation and hands it only the
 // input and output buffers, or a latency-critical path that must not pay
 // for cudaMalloc / cudaFree and their implicit device synchronisation.  For
-// them this entry point keeps the forward's only scratch memory -- one int32
-// flag per head, set when that head's V holds an infinity or NaN -- in a
-// file-scope device array instead of a caller workspace.
+// them this entry point keeps the forward's only scratch memory -- four
+// int32 per head from the scan of V (whether it holds an infinity or NaN,
+// and the largest exponent of its finite values) -- in a file-scope device
+// array instead of a caller workspace.
 //
-// The array is kSwaNoallocMaxHeads = 4096 int32 (16 KB).  Every GPU that loads
-// the library holds it until the process exits.  Host code may not use the
+// The array holds kSwaNoallocMaxHeads = 4096 heads (4 x 4096 int32, 64 KB).
+// Every GPU that loads the library holds it until the process exits.  Host code may not use the
 // array's name as a device address (on the host it names a stand-in), so on
 // the first call on each device, with that device current, the entry point
 // looks the address up with cudaGetSymbolAddress and caches it; that first
 // call should therefore come before any stream capture.  All calls share
 // the array and it keeps the last call's contents: each call clears the
-// flags it uses before the scan, and calls that overlap on the GPU (other
+// entries it uses before the scan, and calls that overlap on the GPU (other
 // streams, other host threads) race on it.
 #include <mutex>
 
@@ -27,7 +28,8 @@ namespace {
 
 constexpr int64_t kSwaNoallocMaxHeads = 4096;
 
-static __device__ __align__(256) int g_noalloc_head_flags[kSwaNoallocMaxHeads];
+static __device__ __align__(256) int g_noalloc_head_flags[swa::kHeadInfoInts *
+                                                          kSwaNoallocMaxHeads];
 
 // Device address of g_noalloc_head_flags for the current device.
 int* noalloc_flags(swa_status* st) {
@@ -80,21 +82,18 @@ extern "C" swa_status swa_attn_fwd_noalloc(const void* q, const void* k, const v
   int launches = 0;
   cudaError_t e;
   if (dt == SWA_F32) {
-    e = swa::launch_attn_fwd_simt(dt, q, k, v, out, lse, BH, N, c, scale, nullptr, 0, s,
-                                  &launches);
+    e = swa::launch_attn_fwd_simt(dt, q, k, v, out, lse, BH, N, c, scale, s, &launches);
     if (e != cudaSuccess) return swa::api_cuda_fail(e, "attn_fwd_simt");
   } else {
-    int* flags = noalloc_flags(&st);
-    if (!flags) return st;
-    e = cudaMemsetAsync(flags, 0, (size_t)BH * sizeof(int), s);
-    if (e != cudaSuccess) return swa::api_cuda_fail(e, "cudaMemsetAsync(noalloc flags)");
-    e = swa::launch_scan_nonfinite(dt, v, BH, N * D, flags, s, &launches);
-    if (e != cudaSuccess) return swa::api_cuda_fail(e, "scan_nonfinite(v)");
-    e = swa::launch_attn_fwd_tc(q, k, v, out, lse, B, H, N, c, scale, flags, err, s, &launches);
+    int* vinfo = noalloc_flags(&st);
+    if (!vinfo) return st;
+    e = cudaMemsetAsync(vinfo, 0, (size_t)BH * swa::kHeadInfoInts * sizeof(int), s);
+    if (e != cudaSuccess) return swa::api_cuda_fail(e, "cudaMemsetAsync(noalloc scratch)");
+    e = swa::launch_scan_v_info(v, BH, N * D, vinfo, s, &launches);
+    if (e != cudaSuccess) return swa::api_cuda_fail(e, "scan_v_info");
+    e = swa::launch_attn_fwd_tc(q, k, v, out, lse, B, H, N, c, scale, vinfo, swa::FwdSaved{},
+                                 err, s, &launches);
     if (e != cudaSuccess) return swa::api_cuda_fail(e, "attn_fwd_tc");
-    e = swa::launch_attn_fwd_simt(dt, q, k, v, out, lse, BH, N, c, scale, flags, 1, s,
-                                  &launches);
-    if (e != cudaSuccess) return swa::api_cuda_fail(e, "attn_fwd_simt(non-finite heads)");
   }
   swa::api_end_call(launches);
   return SWA_OK;

@@ -35,6 +35,15 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// One arrival for the whole warp (the barrier counts warps): the lanes meet
+// at __syncwarp, which orders every lane's earlier memory and tcgen05
+// operations before lane 0's release.  One shared-memory atomic per warp
+// instead of 32 keeps the barrier traffic off the MIO queue.
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
                "r"(bytes)
@@ -123,6 +132,13 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
           smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Orders this thread's earlier generic-proxy shared-memory writes before
+// later async-proxy accesses (tcgen05.mma operand reads, TMA), once the
+// thread's release (an mbarrier arrive) is acquired by the issuing thread.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
@@ -353,16 +369,23 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo_byte
   return d;
 }
 
-// Instruction descriptor of tcgen05.mma kind::f16 with bf16 A and B and an
-// f32 accumulator:
-//   bits 4-5 D format (1 = f32); bits 7-9 A format (1 = bf16);
-//   bits 10-12 B format (1 = bf16); bit 15 A major (0 = K, 1 = MN);
-//   bit 16 B major; bits 17-22 N >> 3; bits 24-28 M >> 4.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_major,
-                                                      int b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn_major << 15) |
+// Instruction descriptor of tcgen05.mma kind::f16 with an f32 accumulator:
+//   bits 4-5 D format (1 = f32); bits 7-9 A format and bits 10-12 B format
+//   (0 = f16, 1 = bf16; A and B always of one type); bit 15 A major
+//   (0 = K, 1 = MN); bit 16 B major; bits 17-22 N >> 3; bits 24-28 M >> 4.
+__host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, int a_mn_major,
+                                                    int b_mn_major, uint32_t ab_format) {
+  return (1u << 4) | (ab_format << 7) | (ab_format << 10) | ((uint32_t)a_mn_major << 15) |
          ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_major,
+                                                      int b_mn_major) {
+  return idesc_f32acc(M, N, a_mn_major, b_mn_major, 1u);
+}
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int a_mn_major,
+                                                     int b_mn_major) {
+  return idesc_f32acc(M, N, a_mn_major, b_mn_major, 0u);
 }
 
 // ----------------------------------------------------------------- numerics
@@ -388,6 +411,42 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// Two floats -> packed f16x2 (lo in bits 0-15), round to nearest even.
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float f16lo(uint32_t v) {
+  float f;
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %1;\n\tcvt.f32.f16 %0, a;\n\t}" : "=f"(f) : "r"(v));
+  return f;
+}
+__device__ __forceinline__ float f16hi(uint32_t v) {
+  float f;
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %1;\n\tcvt.f32.f16 %0, b;\n\t}" : "=f"(f) : "r"(v));
+  return f;
+}
+
+// P (a softmax weight) as the 16-bit A operand of a kind::f16 MMA: f16 when
+// kF16 (10 fraction bits), else bf16.
+template <bool kF16>
+__device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
+  if constexpr (kF16) return pack_f16(lo, hi);
+  else return pack_bf16(lo, hi);
+}
+template <bool kF16>
+__device__ __forceinline__ float unpack_lo(uint32_t v) {
+  if constexpr (kF16) return f16lo(v);
+  else return bf16lo(v);
+}
+template <bool kF16>
+__device__ __forceinline__ float unpack_hi(uint32_t v) {
+  if constexpr (kF16) return f16hi(v);
+  else return bf16hi(v);
 }
 
 }  // namespace tc

@@ -2,9 +2,15 @@
 collective.
 
 The attention heads (b, h) and the regrid's targets are independent
-problems, so N ranks run N independent replicas of the workload, each on
-its own seeded batch (weak scaling).  The only collectives are a barrier
-around the timed region and a MAX reduction of each rank's elapsed time.
+problems, so one problem is split across ranks without any exchange: at
+world size W the problem is a batch of B*W sequences (and W blocks of
+regrid targets against one shared source set), and rank r computes
+sequences [r*B, (r+1)*B) -- the heads [r*B*H, (r+1)*B*H) of the flattened
+batch -- and target block r.  The per-rank work is fixed as W grows (weak
+scaling).  Every sequence is drawn from a seed of its own, so a rank draws
+its block alone and the global batch does not depend on W.  The only
+collectives are a barrier around the timed region and a MAX reduction of
+each rank's elapsed time.
 """
 from __future__ import annotations
 
@@ -50,9 +56,17 @@ def shutdown() -> None:
         dist.destroy_process_group()
 
 
-def replica_seed(base_seed: int, rank: int) -> int:
-    """Seed of rank r's batch: rank 0 keeps the workload's own seed."""
-    return base_seed + 1000 * rank
+def shard(units: int, world: int, rank: int) -> tuple[int, int]:
+    """Contiguous block (first, count) of `units` independent units for
+    `rank`; the blocks of ranks 0..world-1 partition [0, units) in order."""
+    base, extra = divmod(units, world)
+    first = rank * base + min(rank, extra)
+    return first, base + (1 if rank < extra else 0)
+
+
+def sequence_block(per_rank: int, rank: int) -> int:
+    """First sequence of rank r when every rank takes `per_rank` sequences."""
+    return per_rank * rank
 
 
 def barrier(device: torch.device | None = None) -> None:

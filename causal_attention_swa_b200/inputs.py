@@ -17,6 +17,18 @@ Recipes (numpy ``default_rng`` = PCG64, one generator per workload):
 * ``nw_grid``: 16384 sources uniform in [0,10]^2 with values
   sin(x) cos(y) + 0.1 N(0,1), 16384 targets uniform in [0,10]^2, seed 2,
   stored as float32.
+* ``nw_grid_nd``: the regrid workload with points of 1, 2 or 3 coordinates
+  uniform in [0,10]^d, values sin(x) cos(y) cos(z) (the factors that exist)
+  + 0.1 N(0,1), seed 2, stored as float32; d = 2 is ``nw_grid``.
+* ``qkv_inputs``: the projection's input x ~ N(0,1) [B, N, C] and weight
+  w ~ N(0, 1/C) [3 H 64, C] (so q, k, v come out ~ N(0,1)), drawn as float32
+  in that order and rounded to bfloat16.
+* ``attn_bf16_batch``: the same per sequence: sequence b of a batch draws
+  its q, k, v [H, N, D] from ``default_rng([seed, b])``, so any block of
+  sequences is drawn without the others (the multi-GPU split of one batch).
+* ``nw_targets_block``: block r of a regrid's target set -- block 0 is
+  ``nw_grid``'s targets, block r > 0 is drawn from ``default_rng([seed, r])``
+  uniform in [0,10]^2.
 * ``attn_bf16``: Q, K, V iid normal (std per tensor) drawn as float32 in the
   order q, k, v, rounded to bfloat16 (round to nearest even), layout
   [B, H, N, D]; optionally a number of V entries set to +inf at positions
@@ -100,6 +112,29 @@ def nw_grid(M: int = 16384, S: int = 16384, seed: int = 2):
     return (targets.astype(np.float32), sources.astype(np.float32), vals.astype(np.float32))
 
 
+def nw_grid_nd(M: int = 16384, S: int = 16384, dims: int = 2, seed: int = 2):
+    """Regrid workload with points of `dims` coordinates, float32:
+    targets [M, dims], sources [S, dims], vals [S]."""
+    if dims == 2:
+        return nw_grid(M, S, seed)
+    rng = np.random.default_rng(seed)
+    sources = rng.uniform(0.0, 10.0, size=(S, dims))
+    noise = rng.normal(size=S)
+    targets = rng.uniform(0.0, 10.0, size=(M, dims))
+    vals = np.sin(sources[:, 0]) + 0.1 * noise
+    if dims == 3:
+        vals = np.sin(sources[:, 0]) * np.cos(sources[:, 1]) * np.cos(sources[:, 2]) + 0.1 * noise
+    return (targets.astype(np.float32), sources.astype(np.float32), vals.astype(np.float32))
+
+
+def qkv_inputs(B: int, N: int, C: int, H: int, seed: int):
+    """(x, w) as uint16 bfloat16 bit patterns: x [B, N, C], w [3*H*64, C]."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal(size=(B, N, C), dtype=np.float32)
+    w = rng.standard_normal(size=(3 * H * D, C), dtype=np.float32) * np.float32(C ** -0.5)
+    return bf16_bits(x), bf16_bits(w)
+
+
 def attn_bf16(B: int, H: int, N: int, seed: int, qk_std: float = 1.0, v_std: float = 1.0,
               n_inf: int = 0):
     """(q, k, v) as uint16 bfloat16 bit patterns [B, H, N, 64], and the flat
@@ -121,9 +156,35 @@ def attn_bf16(B: int, H: int, N: int, seed: int, qk_std: float = 1.0, v_std: flo
     return bf16_bits(q), bf16_bits(k), bf16_bits(v), pos
 
 
+def attn_bf16_batch(B: int, H: int, N: int, seed: int, first: int = 0, qk_std: float = 1.0,
+                    v_std: float = 1.0):
+    """Sequences first .. first+B-1 of a batch whose sequence b draws q, k, v
+    ~ N(0, std^2) [H, N, 64] (float32, then bf16) from default_rng([seed, b]).
+    Returns uint16 bf16 patterns q, k, v [B, H, N, 64]."""
+    out = [np.empty((B, H, N, D), dtype=np.uint16) for _ in range(3)]
+    for i in range(B):
+        rng = np.random.default_rng([seed, first + i])
+        for t, std in zip(out, (qk_std, qk_std, v_std)):
+            x = rng.standard_normal(size=(H, N, D), dtype=np.float32)
+            if std != 1.0:
+                x *= np.float32(std)
+            t[i] = bf16_bits(x)
+    return tuple(out)
+
+
+def nw_targets_block(M: int, block: int, seed: int = 2):
+    """Block `block` of M regrid targets (float32 [M, 2])."""
+    if block == 0:
+        return nw_grid(M, M, seed)[0]
+    rng = np.random.default_rng([seed, block])
+    return rng.uniform(0.0, 10.0, size=(M, 2)).astype(np.float32)
+
+
 # Named workloads: shapes and seeds.
 WORKLOADS = {
     "attn_fwd_b4h16n4096": dict(B=4, H=16, N=4096, seed=3),
+    # drawn per sequence (attn_bf16_batch): the benchmark's batch, split
+    # across GPUs by sequences
     "attn_fwdbwd_b2h16n16384": dict(B=2, H=16, N=16384, seed=4),
     "attn_fwdbwd_b1h8n65536": dict(B=1, H=8, N=65536, seed=5, qk_std=0.5),
 }

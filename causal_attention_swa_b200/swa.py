@@ -27,8 +27,11 @@ EXPORTS = (
     "swa_attn_bwd", "swa_nw_workspace_size", "swa_nw_regrid", "swa_get_device_error",
     "swa_status_string", "swa_last_error_message", "swa_last_launch_count",
     "swa_profile_kernel", "swa_attn_fwd_noalloc", "swa_selftest_wait_timeout",
+    "swa_attn_grad_workspace_size", "swa_attn_grad", "swa_nw_regrid_nd",
+    "swa_nw_regrid_bwd_workspace_size", "swa_nw_regrid_bwd", "swa_qkv_proj",
 )
-SWA_KERNEL_NONE, SWA_KERNEL_ATTN_FWD, SWA_KERNEL_ATTN_BWD, SWA_KERNEL_NW = range(4)
+(SWA_KERNEL_NONE, SWA_KERNEL_ATTN_FWD, SWA_KERNEL_ATTN_BWD, SWA_KERNEL_NW, SWA_KERNEL_NW_BWD,
+ SWA_KERNEL_QKV) = range(6)
 
 
 class SwaError(RuntimeError):
@@ -65,10 +68,22 @@ def load_library():
     lib.swa_attn_bwd_workspace_size.restype = SZ
     lib.swa_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I64, I64, I64, I64, I, I, P, SZ, P]
     lib.swa_attn_bwd.restype = I
+    lib.swa_attn_grad_workspace_size.argtypes = [I64, I64, I64, I64, I]
+    lib.swa_attn_grad_workspace_size.restype = SZ
+    lib.swa_attn_grad.argtypes = [P, P, P, P, P, P, P, P, I64, I64, I64, I64, I, I, P, SZ, P]
+    lib.swa_attn_grad.restype = I
     lib.swa_nw_workspace_size.argtypes = [I64, I64]
     lib.swa_nw_workspace_size.restype = SZ
     lib.swa_nw_regrid.argtypes = [P, I64, P, P, I64, F, P, P, SZ, P]
     lib.swa_nw_regrid.restype = I
+    lib.swa_nw_regrid_nd.argtypes = [P, I64, P, P, I64, I, F, P, P, SZ, P]
+    lib.swa_nw_regrid_nd.restype = I
+    lib.swa_nw_regrid_bwd_workspace_size.argtypes = [I64, I64, I]
+    lib.swa_nw_regrid_bwd_workspace_size.restype = SZ
+    lib.swa_nw_regrid_bwd.argtypes = [P, I64, P, P, I64, I, F, P, P, P, P, P, SZ, P]
+    lib.swa_nw_regrid_bwd.restype = I
+    lib.swa_qkv_proj.argtypes = [P, P, P, P, P, I64, I64, I64, I64, I64, I, P]
+    lib.swa_qkv_proj.restype = I
     lib.swa_get_device_error.argtypes = [P]
     lib.swa_get_device_error.restype = I
     lib.swa_selftest_wait_timeout.argtypes = [P]
@@ -149,6 +164,10 @@ def attn_bwd_workspace_size(B, H, N, D, dtype_code) -> int:
     return int(load_library().swa_attn_bwd_workspace_size(B, H, N, D, dtype_code))
 
 
+def attn_grad_workspace_size(B, H, N, D, dtype_code) -> int:
+    return int(load_library().swa_attn_grad_workspace_size(B, H, N, D, dtype_code))
+
+
 def nw_workspace_size(M, S) -> int:
     return int(load_library().swa_nw_workspace_size(M, S))
 
@@ -208,6 +227,32 @@ def attn_bwd(q, k, v, out, dout, lse, causal: bool = True, dq=None, dk=None, dv=
     return dq, dk, dv
 
 
+def attn_grad(q, k, v, causal: bool = True, out=None, lse=None, dq=None, dk=None, dv=None,
+              workspace=None):
+    """swa_attn_grad: forward and the gradient of 1/2 sum out^2 in one call ->
+    (out, lse, dq, dk, dv)."""
+    if not isinstance(q, torch.Tensor) or q.dim() != 4:
+        raise ValueError("q must be a [B, H, N, D] tensor")
+    B, H, N, D = q.shape
+    dt = _dtype_code(q)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    _require_like(q, {"k": k, "v": v, "out": out, "lse": lse, "dq": dq, "dk": dk, "dv": dv},
+                  lambda n: ((B, H, N), torch.float32) if n == "lse" else (q.shape, q.dtype))
+    lib = load_library()
+    _require_cuda(q, k, v, out, lse, dq, dk, dv)
+    nbytes = attn_grad_workspace_size(B, H, N, D, dt)
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib.swa_attn_grad(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dq), _ptr(dk),
+                           _ptr(dv), B, H, N, D, int(bool(causal)), dt, _ptr(ws), nbytes,
+                           _stream_ptr(q.device))
+    _check(st, "swa_attn_grad")
+    return out, lse, dq, dk, dv
+
+
 def nw_regrid(targets, sources, vals, h: float = 0.5, out=None, workspace=None):
     """swa_nw_regrid: targets [M,2], sources [S,2], vals [S] fp32 -> out [M] fp32."""
     if not isinstance(targets, torch.Tensor) or targets.dim() != 2 or \
@@ -226,6 +271,71 @@ def nw_regrid(targets, sources, vals, h: float = 0.5, out=None, workspace=None):
                            _ptr(ws), nbytes, _stream_ptr(targets.device))
     _check(st, "swa_nw_regrid")
     return out
+
+
+def _nw_points(targets, sources):
+    if not isinstance(targets, torch.Tensor) or targets.dim() != 2 or \
+            not isinstance(sources, torch.Tensor) or sources.dim() != 2:
+        raise ValueError("targets and sources must be [M, d] and [S, d] tensors")
+    return targets.shape[0], sources.shape[0], targets.shape[1]
+
+
+def nw_regrid_nd(targets, sources, vals, h: float = 0.5, out=None, workspace=None):
+    """swa_nw_regrid_nd: targets [M,d], sources [S,d] (d = 1, 2, 3), vals [S]
+    fp32 -> out [M] fp32."""
+    M, S, d = _nw_points(targets, sources)
+    out = torch.empty((M,), dtype=torch.float32, device=targets.device) if out is None else out
+    shapes = {"targets": (M, d), "sources": (S, d), "vals": (S,), "out": (M,)}
+    _require_like(targets, {"targets": targets, "sources": sources, "vals": vals, "out": out},
+                  lambda n: (shapes[n], torch.float32))
+    lib = load_library()
+    _require_cuda(targets, sources, vals, out)
+    nbytes = nw_workspace_size(M, S)
+    ws = _workspace(nbytes, targets.device, workspace)
+    st = lib.swa_nw_regrid_nd(_ptr(targets), M, _ptr(sources), _ptr(vals), S, d, float(h),
+                              _ptr(out), _ptr(ws), nbytes, _stream_ptr(targets.device))
+    _check(st, "swa_nw_regrid_nd")
+    return out
+
+
+def nw_regrid_bwd(targets, sources, vals, gout, h: float = 0.5, workspace=None):
+    """swa_nw_regrid_bwd -> (dtargets [M,d], dsources [S,d], dvals [S])."""
+    M, S, d = _nw_points(targets, sources)
+    dt = torch.empty_like(targets)
+    ds = torch.empty_like(sources)
+    dv = torch.empty((S,), dtype=torch.float32, device=targets.device)
+    shapes = {"targets": (M, d), "sources": (S, d), "vals": (S,), "gout": (M,)}
+    _require_like(targets, {"targets": targets, "sources": sources, "vals": vals, "gout": gout},
+                  lambda n: (shapes[n], torch.float32))
+    lib = load_library()
+    _require_cuda(targets, sources, vals, gout, dt, ds, dv)
+    nbytes = int(lib.swa_nw_regrid_bwd_workspace_size(M, S, d))
+    ws = _workspace(nbytes, targets.device, workspace)
+    st = lib.swa_nw_regrid_bwd(_ptr(targets), M, _ptr(sources), _ptr(vals), S, d, float(h),
+                               _ptr(gout), _ptr(dt), _ptr(ds), _ptr(dv), _ptr(ws), nbytes,
+                               _stream_ptr(targets.device))
+    _check(st, "swa_nw_regrid_bwd")
+    return dt, ds, dv
+
+
+def qkv_proj(x, w, H: int, q=None, k=None, v=None):
+    """swa_qkv_proj: x [B, N, C] bf16, w [3*H*64, C] bf16 -> q, k, v
+    [B, H, N, 64] bf16."""
+    if not isinstance(x, torch.Tensor) or x.dim() != 3:
+        raise ValueError("x must be a [B, N, C] tensor")
+    B, N, C = x.shape
+    shape = (B, H, N, 64)
+    q = torch.empty(shape, dtype=x.dtype, device=x.device) if q is None else q
+    k = torch.empty(shape, dtype=x.dtype, device=x.device) if k is None else k
+    v = torch.empty(shape, dtype=x.dtype, device=x.device) if v is None else v
+    shapes = {"x": (B, N, C), "w": (3 * H * 64, C), "q": shape, "k": shape, "v": shape}
+    _require_like(x, {"x": x, "w": w, "q": q, "k": k, "v": v}, lambda n: (shapes[n], x.dtype))
+    lib = load_library()
+    _require_cuda(x, w, q, k, v)
+    st = lib.swa_qkv_proj(_ptr(x), _ptr(w), _ptr(q), _ptr(k), _ptr(v), B, N, C, H, 64,
+                          _dtype_code(x), _stream_ptr(x.device))
+    _check(st, "swa_qkv_proj")
+    return q, k, v
 
 
 def selftest_wait_timeout(device=None) -> None:

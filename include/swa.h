@@ -62,8 +62,8 @@ typedef enum {
 } swa_dtype;
 
 /*
- * Bytes of workspace swa_attn_fwd needs (one int32 flag per head for the
- * bf16 path, 0 for float32).
+ * Bytes of workspace swa_attn_fwd needs (four int32 of per-head information
+ * for the bf16 path, 0 for float32).
  */
 size_t swa_attn_fwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D,
                                    swa_dtype dtype);
@@ -77,9 +77,13 @@ size_t swa_attn_fwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D,
  *   out      [B,H,N,D] of `dtype`         (out)  out_i = sum_j P_ij v_j
  *   lse      [B,H,N] float32              (out)  m_i + ln z_i (natural log)
  *   B, H >= 1; N >= 1; D == 64.
- * The bf16 path scans V for non-finite values; heads that hold one are
- * computed by the exact pair-by-pair kernel so that masked pairs stay
- * absent, the others by the tensor-core kernel.
+ * The bf16 path runs every head on the tensor cores.  A scan of V finds the
+ * heads that hold an infinity or NaN: for those the kernel replaces every
+ * non-finite V entry by 0 before its products and gives each output entry
+ * the IEEE class of the sum over its existing pairs (every weight > 0), so
+ * a masked pair never multiplies a value.  The same scan decides the
+ * operand type of P V: f16 (P and V) when every finite |V| < 2^15, else bf16.
+ * float32 inputs run on CUDA cores in float32.
  */
 swa_status swa_attn_fwd(const void* q, const void* k, const void* v, void* out,
                         float* lse, int64_t B, int64_t H, int64_t N, int64_t D,
@@ -87,8 +91,9 @@ swa_status swa_attn_fwd(const void* q, const void* k, const void* v, void* out,
                         size_t workspace_bytes, void* stream);
 
 /*
- * Bytes of workspace swa_attn_bwd needs: per-head flags, and delta and
- * lse * log2(e) as float32 [B,H,Npad] each (Npad = N rounded up to 128).
+ * Bytes of workspace swa_attn_bwd needs: per-head information (four int32),
+ * delta and lse * log2(e) as float32 [B,H,Npad] each (Npad = N rounded up to
+ * 128) and, for bf16, f16 copies of q, k, v and dout ([B,H,N,D] each).
  */
 size_t swa_attn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D,
                                    swa_dtype dtype);
@@ -103,14 +108,43 @@ size_t swa_attn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D,
  * P_ij = exp(s_ij - lse_i); delta_i = sum_d dout_id out_id;
  * dS_ij = P_ij (dout_i . v_j - delta_i); dq_i = scale sum_j dS_ij k_j;
  * dk_j = scale sum_i dS_ij q_i; dv_j = sum_i P_ij dout_i (existing pairs only).
- * V and dout may hold non-finite values (heads with one take the exact
- * pair-by-pair kernel).
+ * bf16: tensor cores for every head, with f16 operands (copies made by a prep
+ * pass) when every finite |q|, |k|, |v|, |dout| < 2^15, else bf16.  V and
+ * dout may hold infinities or NaN: every product over existing pairs is the
+ * IEEE one, and no masked pair multiplies a value (dV of a diagonal block
+ * reads a copy of dout with its non-finite entries replaced by 0, and those
+ * entries' classes are merged back).  float32: CUDA cores, float32.
  */
 swa_status swa_attn_bwd(const void* q, const void* k, const void* v, const void* out,
                         const void* dout, const float* lse, void* dq, void* dk, void* dv,
                         int64_t B, int64_t H, int64_t N, int64_t D, int causal,
                         swa_dtype dtype, void* workspace, size_t workspace_bytes,
                         void* stream);
+
+/* Bytes of workspace swa_attn_grad needs (as swa_attn_bwd_workspace_size). */
+size_t swa_attn_grad_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D,
+                                    swa_dtype dtype);
+
+/*
+ * Forward and gradient in one call: the query GRADIENT of "Show HN: Automatic
+ * deduction of FlashAttention kernel from ~25 lines of SQL" (page 2) --
+ * loss = 1/2 sum out^2 over the attention view, and its gradient with
+ * respect to every value of q, k and v in one backward pass.
+ *   q, k, v     [B,H,N,D] of `dtype`   (in)
+ *   out         [B,H,N,D] of `dtype`   (out)  as swa_attn_fwd
+ *   lse         [B,H,N] float32        (out)  as swa_attn_fwd
+ *   dq, dk, dv  [B,H,N,D] of `dtype`   (out)  gradient of 1/2 sum out^2
+ * Same as swa_attn_fwd followed by swa_attn_bwd with dout = out, except that
+ * for bf16 the backward's upstream gradient is the forward's float32 output
+ * (kept as an f16 copy in the workspace; delta_i = |out_i|^2 in float32), not
+ * the bf16 `out`: the gradient of rows whose dq nearly cancels (rows that see
+ * few keys) is then not limited by the bf16 rounding of out.
+ * Workspace: swa_attn_grad_workspace_size() bytes.  Errors as swa_attn_bwd.
+ */
+swa_status swa_attn_grad(const void* q, const void* k, const void* v, void* out, float* lse,
+                         void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N,
+                         int64_t D, int causal, swa_dtype dtype, void* workspace,
+                         size_t workspace_bytes, void* stream);
 
 /*
  * swa_attn_fwd without a workspace, for callers that cannot allocate device
@@ -119,9 +153,9 @@ swa_status swa_attn_bwd(const void* q, const void* k, const void* v, const void*
  * pay for cudaMalloc/cudaFree and their implicit synchronisation).  The
  * pages have no counterpart: this is an interface convenience.
  * Same arguments, results and errors as swa_attn_fwd minus the workspace.
- * The forward's scratch (one int32 flag per head) lives in a static device
- * array of 4096 entries (16 KB, held by every GPU that loads the library
- * until exit); B*H > 4096 returns SWA_ERR_UNSUPPORTED.  The first call on
+ * The forward's scratch (four int32 of information per head) lives in a
+ * static device array for 4096 heads (64 KB, held by every GPU that loads
+ * the library until exit); B*H > 4096 returns SWA_ERR_UNSUPPORTED.  The first call on
  * each device looks up the array's device address (make it before any
  * stream capture).  All calls share the array: calls that overlap on the
  * GPU race.  Allocates nothing.
@@ -144,6 +178,55 @@ size_t swa_nw_workspace_size(int64_t M, int64_t S);
 swa_status swa_nw_regrid(const float* targets, int64_t M, const float* sources,
                          const float* vals, int64_t S, float h, float* out,
                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The regrid with points of `dims` coordinates (1, 2 or 3; dims = 2 is
+ * swa_nw_regrid): the NADARAYA_WATSON view with the squared distance summed
+ * over every coordinate column of the point tables.
+ *   targets [M,dims] float32   sources [S,dims] float32   vals [S] float32
+ *   out     [M] float32        out_p = sum_q w_pq v_q / sum_q w_pq,
+ *   w_pq = exp(-sum_c (t_pc - s_qc)^2 / h^2).  Workspace: swa_nw_workspace_size.
+ * Other dims return SWA_ERR_UNSUPPORTED.
+ */
+swa_status swa_nw_regrid_nd(const float* targets, int64_t M, const float* sources,
+                            const float* vals, int64_t S, int dims, float h, float* out,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace swa_nw_regrid_bwd needs. */
+size_t swa_nw_regrid_bwd_workspace_size(int64_t M, int64_t S, int dims);
+
+/*
+ * Gradient of the regrid (the GRADIENT query's backward pass applied to the
+ * NADARAYA_WATSON view: the same softmax-weighted average over a join, with
+ * weights P_pq = w_pq / sum_q w_pq) for an upstream gradient gout = dL/dout:
+ *   gout      [M] float32        (in)
+ *   dtargets  [M,dims] float32   (out)  dL/dt_p = (-2/h^2) sum_q (gout_p / Z_p)
+ *                                        w_pq (v_q - out_p) (t_p - s_q)
+ *   dsources  [S,dims] float32   (out)  dL/ds_q = (+2/h^2) sum_p (same terms)
+ *   dvals     [S] float32        (out)  dL/dv_q = sum_p gout_p P_pq
+ * with Z_p = sum_q w_pq and out_p recomputed (the forward's output is not an
+ * input).  Two passes over the pair grid (per target, then per source) with
+ * deterministic partial sums.  Arguments and errors as swa_nw_regrid_nd.
+ */
+swa_status swa_nw_regrid_bwd(const float* targets, int64_t M, const float* sources,
+                             const float* vals, int64_t S, int dims, float h, const float* gout,
+                             float* dtargets, float* dsources, float* dvals, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/*
+ * The projection in front of attention ("Wiki notes", page 5, mini_attention:
+ * Q = x Wq, K = x Wk, V = x Wv), written straight into attention's layout.
+ *   x        [B*N, C] bf16 (token rows, b major)      (in)
+ *   w        [3*H*D, C] bf16: one row per output feature -- q's features
+ *            h*D + d, then k's, then v's (a linear layer's weight layout)
+ *   q, k, v  [B,H,N,D] bf16                             (out)
+ * q[b,h,n,d] = sum_c x[b*N+n, c] w[h*D+d, c] (k, v: rows H*D.., 2*H*D..),
+ * float32 accumulation on the tensor cores, one rounding to bf16.
+ * D == 64, C a positive multiple of 64 (else SWA_ERR_UNSUPPORTED); bf16 only.
+ */
+swa_status swa_qkv_proj(const void* x, const void* w, void* q, void* k, void* v, int64_t B,
+                        int64_t N, int64_t C, int64_t H, int64_t D, swa_dtype dtype,
+                        void* stream);
 
 /*
  * Synchronises `stream`, then reads and clears this device's error word.
@@ -175,9 +258,11 @@ int swa_last_launch_count(void);
 /* Main kernels that swa_profile_kernel can bracket with events. */
 typedef enum {
     SWA_KERNEL_NONE = 0,
-    SWA_KERNEL_ATTN_FWD = 1, /* swa_attn_fwd: the kernel of the heads with finite V */
-    SWA_KERNEL_ATTN_BWD = 2, /* swa_attn_bwd: the main kernel(s) of the finite heads */
-    SWA_KERNEL_NW = 3        /* swa_nw_regrid: the pair-grid kernel (not the final sum) */
+    SWA_KERNEL_ATTN_FWD = 1, /* swa_attn_fwd, swa_attn_grad: the tensor-core forward */
+    SWA_KERNEL_ATTN_BWD = 2, /* swa_attn_bwd, swa_attn_grad: the tensor-core backward */
+    SWA_KERNEL_NW = 3,       /* swa_nw_regrid(_nd): both kernels (pair grid and final sum) */
+    SWA_KERNEL_NW_BWD = 4,   /* swa_nw_regrid_bwd: its four kernels */
+    SWA_KERNEL_QKV = 5       /* swa_qkv_proj */
 } swa_kernel;
 
 /*

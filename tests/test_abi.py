@@ -39,13 +39,15 @@ def test_status_strings(lib):
 
 
 def test_workspace_sizes(lib):
-    # bf16 forward: one int32 flag per head, rounded to 256 bytes
-    assert lib.swa_attn_fwd_workspace_size(2, 16, 16384, 64, swa.SWA_BF16) == 256
+    # bf16 forward: four int32 of per-head information, rounded to 256 bytes
+    assert lib.swa_attn_fwd_workspace_size(2, 16, 16384, 64, swa.SWA_BF16) == 512
     assert lib.swa_attn_fwd_workspace_size(1, 1, 256, 64, swa.SWA_F32) == 0
-    # backward: flags + delta and lse*log2(e) padded to 128-row blocks
+    # backward: information + delta and lse*log2(e) padded to 128-row blocks,
+    # and for bf16 four f16 operand copies
     B, H, N, D = 2, 16, 16384, 64
-    want = 256 + 2 * B * H * N * 4
+    want = 512 + 2 * B * H * N * 4 + 4 * B * H * N * D * 2
     assert lib.swa_attn_bwd_workspace_size(B, H, N, D, swa.SWA_BF16) == want
+    assert lib.swa_attn_grad_workspace_size(B, H, N, D, swa.SWA_BF16) == want
     assert lib.swa_attn_bwd_workspace_size(1, 1, 256, 64, swa.SWA_F32) == 256 + 2 * 1024
     assert lib.swa_attn_bwd_workspace_size(1, 1, 300, 64, swa.SWA_F32) == 256 + 2 * 1536
     assert lib.swa_nw_workspace_size(16384, 16384) > 0
@@ -87,6 +89,19 @@ def test_bwd_argument_errors(lib):
     assert st == swa.SWA_ERR_INVALID_ARGUMENT
 
 
+def test_grad_argument_errors(lib):
+    good = [FAKE] * 8
+    st = lib.swa_attn_grad(*good, 1, 1, 16, 64, 1, swa.SWA_BF16, FAKE, 16, None)
+    assert st == swa.SWA_ERR_INVALID_ARGUMENT  # workspace too small
+    assert b"workspace" in lib.swa_last_error_message()
+    bad = list(good)
+    bad[7] = None  # dv
+    st = lib.swa_attn_grad(*bad, 1, 1, 16, 64, 1, swa.SWA_BF16, FAKE, 1 << 30, None)
+    assert st == swa.SWA_ERR_INVALID_ARGUMENT
+    st = lib.swa_attn_grad(*good, 1, 1, 16, 128, 1, swa.SWA_BF16, FAKE, 1 << 30, None)
+    assert st == swa.SWA_ERR_UNSUPPORTED
+
+
 def test_nw_argument_errors(lib):
     F = ctypes.c_float
     assert lib.swa_nw_regrid(FAKE, 0, FAKE, FAKE, 4, F(0.5), FAKE, FAKE, 1 << 20, None) == \
@@ -99,6 +114,23 @@ def test_nw_argument_errors(lib):
         swa.SWA_ERR_INVALID_ARGUMENT
     assert lib.swa_nw_regrid(FAKE, 4, FAKE, FAKE, 4, F(0.5), FAKE, FAKE, 8, None) == \
         swa.SWA_ERR_INVALID_ARGUMENT
+
+
+def test_nw_nd_and_gradient_argument_errors(lib):
+    F = ctypes.c_float
+    for dims, code in ((0, swa.SWA_ERR_UNSUPPORTED), (4, swa.SWA_ERR_UNSUPPORTED)):
+        assert lib.swa_nw_regrid_nd(FAKE, 4, FAKE, FAKE, 4, dims, F(0.5), FAKE, FAKE, 1 << 20,
+                                    None) == code
+        assert lib.swa_nw_regrid_bwd(FAKE, 4, FAKE, FAKE, 4, dims, F(0.5), FAKE, FAKE, FAKE,
+                                     FAKE, FAKE, 1 << 30, None) == code
+    assert lib.swa_nw_regrid_bwd(FAKE, 4, FAKE, FAKE, 4, 3, F(0.5), None, FAKE, FAKE, FAKE,
+                                 FAKE, 1 << 30, None) == swa.SWA_ERR_INVALID_ARGUMENT
+    assert lib.swa_nw_regrid_bwd(FAKE, 4, FAKE, FAKE, 4, 3, F(0.5), FAKE, FAKE, FAKE, FAKE,
+                                 FAKE, 8, None) == swa.SWA_ERR_INVALID_ARGUMENT
+    assert lib.swa_nw_regrid_bwd_workspace_size(16384, 16384, 2) > 0
+    # the largest S the API accepts plans at most 65535 source chunks (grid.y):
+    # one target's partials then take at most 65535 x 8 bytes
+    assert 0 < lib.swa_nw_workspace_size(1, 1 << 31) <= (65535 * 8 + 255) // 256 * 256
 
 
 def test_product_path_does_not_import_the_oracle():
@@ -133,6 +165,9 @@ def test_binding_rejects_mismatched_tensors_before_any_launch(bad):
         swa.attn_fwd(q, k, v, out=out, lse=lse)
     with pytest.raises(ValueError, match="expected shape"):
         swa.attn_bwd(q, k, v, out, out, lse)
+    if bad != "lse_dtype":
+        with pytest.raises(ValueError, match="expected shape"):
+            swa.attn_grad(q, k, v, out=out)
 
 
 def test_binding_rejects_mismatched_regrid_tensors():

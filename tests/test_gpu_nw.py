@@ -11,7 +11,7 @@ import torch
 
 import oracle
 from causal_attention_swa_b200 import inputs, swa
-from _compare import check_f32
+from _compare import check_f32, check_f32_scaled
 
 pytestmark = pytest.mark.gpu
 
@@ -65,3 +65,79 @@ def test_nw_degenerate_cases():
     s2 = rng.uniform(0, 2, size=(500, 2)).astype(np.float32)
     v2 = rng.normal(size=500).astype(np.float32)
     check_f32(run(t, s2, v2, h=0.25), oracle.nw_regrid(t, s2, v2, h=0.25), "nw h=0.25")
+
+
+# ------------------------------------------ points of 1, 2 or 3 coordinates
+
+def run_nd(t, s, v, h=0.5):
+    out = swa.nw_regrid_nd(dev(t), dev(s), dev(v), h=h)
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("dims", [1, 2, 3])
+@pytest.mark.parametrize("M,S", [(1, 1), (1023, 17), (3000, 4097)])
+def test_nw_nd_ragged_sizes(dims, M, S):
+    rng = np.random.default_rng(M * 11 + S + dims)
+    t = rng.uniform(0, 3, size=(M, dims)).astype(np.float32)
+    s = rng.uniform(0, 3, size=(S, dims)).astype(np.float32)
+    v = rng.normal(size=S).astype(np.float32)
+    check_f32(run_nd(t, s, v), oracle.nw_regrid_nd(t, s, v, h=0.5), f"nw {dims}-d {M}x{S}")
+
+
+@pytest.mark.parametrize("dims", [1, 3])
+def test_nw_nd_grid_16384(dims):
+    t, s, v = inputs.nw_grid_nd(16384, 16384, dims)
+    check_f32(run_nd(t, s, v), oracle.nw_regrid_nd(t, s, v, h=0.5), f"nw {dims}-d 16384x16384")
+
+
+def test_nw_nd_two_dims_is_swa_nw_regrid():
+    t, s, v = inputs.nw_grid(3000, 5000)
+    a = run_nd(t, s, v)
+    b = run(t, s, v)
+    assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------- regrid gradient
+
+def run_bwd(t, s, v, g, h=0.5):
+    res = swa.nw_regrid_bwd(dev(t), dev(s), dev(v), dev(g), h=h)
+    torch.cuda.synchronize()
+    assert swa.get_device_error() == swa.SWA_OK
+    return res
+
+
+def check_bwd(t, s, v, g, h, what):
+    dt, ds, dv = run_bwd(t, s, v, g, h)
+    w_dt, w_ds, w_dv = oracle.nw_regrid_bwd(t, s, v, g, h=h)
+    check_f32_scaled(dt, w_dt, f"dtargets {what}")
+    check_f32_scaled(ds, w_ds, f"dsources {what}")
+    check_f32_scaled(dv, w_dv, f"dvals {what}")
+
+
+@pytest.mark.parametrize("dims", [1, 2, 3])
+@pytest.mark.parametrize("M,S", [(1, 1), (5, 3000), (2500, 1), (1023, 2049), (3000, 4097)])
+def test_nw_gradient_ragged_sizes(dims, M, S):
+    rng = np.random.default_rng(M * 13 + S + dims)
+    t = rng.uniform(0, 3, size=(M, dims)).astype(np.float32)
+    s = rng.uniform(0, 3, size=(S, dims)).astype(np.float32)
+    v = rng.normal(size=S).astype(np.float32)
+    g = rng.normal(size=M).astype(np.float32)
+    check_bwd(t, s, v, g, 0.5, f"{dims}-d {M}x{S}")
+
+
+@pytest.mark.parametrize("dims", [2, 3])
+def test_nw_gradient_grid_16384(dims):
+    """The regrid workload (16384 targets and sources in [0,10]^d) with
+    loss = 1/2 sum out^2: gout = out (the oracle's)."""
+    t, s, v = inputs.nw_grid_nd(16384, 16384, dims)
+    g = oracle.nw_regrid_nd(t, s, v, h=0.5).astype(np.float32)
+    check_bwd(t, s, v, g, 0.5, f"{dims}-d 16384x16384")
+
+
+def test_nw_gradient_demo_inputs_and_another_bandwidth():
+    t, s, y = inputs.pages_nw()
+    t32, s32, y32 = (a.astype(np.float32) for a in (t, s, y))
+    g = np.ones(64, np.float32)
+    check_bwd(t32, s32, y32, g, 0.5, "demo inputs")
+    check_bwd(t32, s32, y32, g, 0.25, "demo inputs h=0.25")

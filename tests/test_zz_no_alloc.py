@@ -13,6 +13,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from causal_attention_swa_b200 import inputs, swa
 from _compare import check_bf16, check_f32, check_lse
 
@@ -61,8 +62,38 @@ def test_noalloc_forward_matches_the_workspace_forward_twice_in_a_row():
         assert swa.get_device_error() == swa.SWA_OK
         check_bf16(got_out, want_out, "out (noalloc vs workspace forward)")
         check_lse(got_lse, want_lse, "lse (noalloc vs workspace forward)")
+        # and against the float64 oracle itself (classes of the +inf head included)
+        w_out, w_lse = oracle.attn_fwd(*(inputs.bf16_to_f64(b) for b in bits))
+        check_bf16(got_out, w_out, "out (noalloc vs oracle)")
+        check_lse(got_lse, w_lse, "lse (noalloc vs oracle)")
     o = got_out.float().cpu().numpy()
     assert np.isfinite(o).all()                # second call: no stale flag, no inf
+
+
+def test_noalloc_forward_allocates_no_device_memory():
+    """After a first call (which looks up the static array's address), more
+    calls change neither the device's free memory nor torch's allocations."""
+    rng = np.random.default_rng(5)
+    bits = [inputs.bf16_bits(rng.standard_normal((1, 4, 512, 64), dtype=np.float32))
+            for _ in range(3)]
+    q, k, v = (_bf16_dev(b) for b in bits)
+    out = torch.empty_like(q)
+    lse = torch.empty((1, 4, 512), dtype=torch.float32, device=q.device)
+    lib, f = _noalloc_fn()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    args = (ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+            ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+            ctypes.c_void_p(lse.data_ptr()), 1, 4, 512, 64, 1, swa.SWA_BF16, stream)
+    assert f(*args) == swa.SWA_OK
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    for _ in range(5):
+        assert f(*args) == swa.SWA_OK
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert torch.cuda.memory_allocated() == alloc0
 
 
 def test_noalloc_forward_float32_path():
