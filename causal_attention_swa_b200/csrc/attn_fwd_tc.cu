@@ -17,15 +17,15 @@
 //   warp  16    TMA producer: Q0, Q1 once, then K_j, V_j into 4 stages
 //   warp  17    MMA issuer for query tile 0 (one elected lane), TMEM owner
 //   warp  18    MMA issuer for query tile 1
-//   warp  19    V converter: rewrites each staged V tile in place (bf16 ->
-//               f16, and a non-finite entry -> 0 with its row recorded), then
-//               releases it to the issuers; it also gives its registers to
-//               the softmax warps of its scheduler
+//   warp  19    V cleaner (heads whose V holds an infinity or NaN): rewrites
+//               each staged V tile in place (a non-finite entry -> 0, its row
+//               recorded), then releases it to the issuers; it also gives its
+//               registers to the softmax warps of its scheduler
 // Each query tile has an issuer of its own, so neither tile's MMAs queue
 // behind the other tile's barriers; each issuer releases a K/V stage on a
 // barrier of its own and the producer waits for the issuers that read it.
 // Registers: launched at 96 per thread (640 x 96); the softmax warps take
-// 104 and warps 16-19 give up to 40, one of them on each scheduler (the
+// 112 and warps 16-19 give up to 32, one of them on each scheduler (the
 // registers of a warp stay in its scheduler's file).  The launcher checks
 // that the kernel was built with exactly 96: a larger claim than the
 // scheduler holds would stall setmaxnreg.inc.
@@ -51,10 +51,10 @@
 // of a row moves (and O, l are rescaled) only when the new row max exceeds
 // it by more than 8, so P <= 2^8 (exact after the final division by l).
 // Precision of O += P V: P enters the MMA as f16 (10 fraction bits) with V
-// converted to f16 in shared memory, for every head whose finite V values
-// lie below 2^15 in magnitude (f16 holds them exactly, up to f16's
-// subnormal spacing of 2^-24); a head with larger values keeps both in
-// bf16.  A bf16 P (7 fraction bits) is exact enough for the output itself,
+// read from an f16 copy of V (the caller's prep pass writes it), for every
+// head whose finite V values lie below 2^15 in magnitude (f16 holds them
+// exactly, up to f16's subnormal spacing of 2^-24); a head with larger
+// values keeps both in bf16 (V as given).  A bf16 P (7 fraction bits) is exact enough for the output itself,
 // but the output is what the gradient of loss = 1/2 sum out^2 feeds back
 // as dout, and the rounding of few-key rows (early rows) reaches the
 // gradient amplified by the cancellation in sum_j dS_ij k_j; with the f16 P
@@ -76,7 +76,7 @@
 // Non-finite V (absent rows: a masked pair must never enter a product,
 // "check_masks_are_absent_rows"): a masked weight of a diagonal tile meets
 // the V rows of keys after the query, and 0 * inf would be NaN.  For a head
-// whose V holds an infinity or NaN (the scan's flag) the converter warp
+// whose V holds an infinity or NaN (the scan's flag) the cleaner warp
 // replaces every non-finite V entry by 0 before the MMA reads the tile and
 // records, per column d, the first key row holding +inf, -inf and NaN; the
 // epilogue then sets out[i, d] to the IEEE class that the sum over the
@@ -106,8 +106,12 @@ constexpr int kSoftmaxWarps = 16;
 constexpr int kThreads = (kSoftmaxWarps + 4) * 32;  // 640: five warps per scheduler
 // 16384 registers per scheduler / (5 warps * 32 threads), rounded down to 8
 constexpr int kLaunchRegs = 96;
-constexpr int kSoftmaxRegs = 104;
-constexpr int kOtherRegs = 40;
+// The softmax warps hold 64 scores per thread plus the loop's state; at 104
+// registers their loop reloaded spilled values every tile (and how many
+// depended on the code around it).  The other warps (TMA, MMA issue, the V
+// cleaner) fit in 32.
+constexpr int kSoftmaxRegs = 112;
+constexpr int kOtherRegs = 32;
 // Warp w runs on scheduler w % 4 and setmaxnreg moves registers only
 // between the warps of one scheduler: each scheduler holds four softmax
 // warps and one of warps 16-19, which gives up what the four take.
@@ -120,7 +124,7 @@ constexpr float kRescaleThreshold = 8.0f;
 // A P computed against a stale reference max must still fit the operand
 // type before it is moved to the new max: < 2^15 in f16, < 2^64 in bf16.
 template <bool kF16> constexpr float kFastRange = kF16 ? 15.0f : 64.0f;
-constexpr int kConvWarp = kSoftmaxWarps + 3;  // warp 19
+constexpr int kCleanWarp = kSoftmaxWarps + 3;  // warp 19
 // Per-head information (kHeadInfoInts int32 per head): bit 0 of [0] is set if
 // V holds an infinity or NaN, [1] is the largest biased exponent of its
 // finite values.  f16 operands are used when that exponent is below 2^15's.
@@ -139,8 +143,8 @@ struct __align__(1024) Smem {
   uint64_t s_free[2];
   uint64_t p_full[2];
   uint64_t pv_done[2];
-  uint64_t v_ready[kStages];    // the converter has rewritten the stage's V tile
-  uint64_t cls_done;            // the converter has recorded every tile's classes
+  uint64_t v_ready[kStages];    // the cleaner has rewritten the stage's V tile
+  uint64_t cls_done;            // the cleaner has recorded every tile's classes
   int first_cls[3][HD];         // per column: first key row with +inf, -inf, NaN
   uint64_t pair[2][4];          // the two threads of a row: tile t, lanes 32w..
   float part[2][2][2][BM];      // [tile][parity][half][row]: partial row max / sum
@@ -163,36 +167,38 @@ __device__ __forceinline__ bool wait_unbounded_by_abort(uint64_t* bar, uint32_t 
   return true;
 }
 
-// Rewrites one staged V tile (128 rows of 128 bytes, 128-byte swizzle) in
-// place: a non-finite entry becomes 0 with its row recorded in first_cls
-// (when `nonfinite`), and every entry is converted to f16 (when kF16).
+// Rewrites one staged V tile of a head whose V holds an infinity or NaN
+// (128 rows of 128 bytes, 128-byte swizzle) in place: a non-finite 16-bit
+// entry (f16 in the f16 instance, bf16 in the other) becomes 0 and its row
+// goes into first_cls.  16-byte chunks without one are left untouched.
 template <bool kF16>
-__device__ __forceinline__ void convert_v_tile(uint8_t* tile, int lane, int key0, bool nonfinite,
-                                               int (*first_cls)[HD]) {
+__device__ __forceinline__ void clean_v_tile(uint8_t* tile, int lane, int key0,
+                                             int (*first_cls)[HD]) {
+  constexpr uint32_t kExp = kF16 ? 0x7C00u : 0x7F80u;   // exponent field all ones
+  constexpr uint32_t kMan = kF16 ? 0x03FFu : 0x007Fu;   // fraction: non-zero = NaN
   uint4* base = reinterpret_cast<uint4*>(tile);
-#pragma unroll 4
+#pragma unroll 2
   for (int c = lane; c < kTileBytes / 16; c += 32) {
     const uint4 x = base[c];
     uint32_t w[4] = {x.x, x.y, x.z, x.w};
-    if (nonfinite) {
-      const int r = c >> 3;                      // row of the tile
-      const int d0 = ((c & 7) ^ (r & 7)) * 8;    // its first column (swizzle undone)
+    bool any = false;
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
+    for (int e = 0; e < 4; ++e)
+      any |= ((w[e] & kExp) == kExp) | (((w[e] >> 16) & kExp) == kExp);
+    if (!any) continue;
+    const int r = c >> 3;                      // row of the tile
+    const int d0 = ((c & 7) ^ (r & 7)) * 8;    // its first column (swizzle undone)
 #pragma unroll
-        for (int p = 0; p < 2; ++p) {
-          const uint32_t b = (w[e] >> (16 * p)) & 0xFFFFu;
-          if ((b & 0x7F80u) == 0x7F80u) {
-            const int cls = (b & 0x7Fu) ? 2 : ((b & 0x8000u) ? 1 : 0);
-            atomicMin(&first_cls[cls][d0 + 2 * e + p], key0 + r);
-            w[e] &= ~(0xFFFFu << (16 * p));
-          }
+    for (int e = 0; e < 4; ++e)
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        const uint32_t b = (w[e] >> (16 * p)) & 0xFFFFu;
+        if ((b & kExp) == kExp) {
+          const int cls = (b & kMan) ? 2 : ((b & 0x8000u) ? 1 : 0);
+          atomicMin(&first_cls[cls][d0 + 2 * e + p], key0 + r);
+          w[e] &= ~(0xFFFFu << (16 * p));
         }
-    }
-    if constexpr (kF16) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) w[e] = pack_f16(bf16lo(w[e]), bf16hi(w[e]));
-    }
+      }
     base[c] = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
@@ -203,16 +209,17 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
                    float* __restrict__ lse, int N, int BH, int n_ctiles, int causal,
-                   float scale_log2, const int* __restrict__ vinfo, uint16_t* __restrict__ do16,
-                   float* __restrict__ delta, float* __restrict__ nlse2,
-                   unsigned* __restrict__ err) {
+                   float scale_log2, const int* __restrict__ vinfo, int all_bf16,
+                   uint16_t* __restrict__ do16, float* __restrict__ delta,
+                   float* __restrict__ nlse2, unsigned* __restrict__ err) {
   // Longest first: every head's latest (heaviest) query tiles, then the next.
   const int head = blockIdx.x % BH;
   const int c = n_ctiles - 1 - blockIdx.x / BH;
   const bool nonfinite = (vinfo[kHeadInfoInts * head] & 1) != 0;
-  if ((vinfo[kHeadInfoInts * head + 1] < kF16ExpLimit) != kF16) return;  // the other instance's head
-  // the converter rewrites V tiles for f16 operands or to remove non-finite values
-  const bool convert = kF16 || nonfinite;
+  const bool f16_head = !all_bf16 && vinfo[kHeadInfoInts * head + 1] < kF16ExpLimit;
+  if (f16_head != kF16) return;  // the other instance's head
+  // the cleaner rewrites the V tiles of a head with non-finite values
+  const bool convert = nonfinite;
 
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -348,14 +355,14 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       wait_unbounded_by_abort(&sm.drain[t], 0);
     }
     __syncwarp();
-  } else if (warp == kConvWarp) {
-    // ---------------------------------------------------------- converter
+  } else if (warp == kCleanWarp) {
+    // ------------------------------------------------------------ cleaner
     if (convert) {
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % kStages;
         if (!mbar_wait_parked(&sm.v_full[s], (j / kStages) & 1, abort, err, kDevTimeoutFull))
           break;
-        convert_v_tile<kF16>(sm.v[s], lane, j * BN, nonfinite, sm.first_cls);
+        clean_v_tile<kF16>(sm.v[s], lane, j * BN, sm.first_cls);
         fence_proxy_async_smem();  // the MMA (async proxy) reads what was written
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.v_ready[s]);
@@ -661,7 +668,8 @@ template <bool kF16>
 cudaError_t launch_fwd_instance(const CUtensorMap& tq, const CUtensorMap& tk,
                                 const CUtensorMap& tv, void* out, float* lse, int64_t BH,
                                 int64_t N, int causal, float scale, const int* vinfo,
-                                const FwdSaved& saved, unsigned* err, cudaStream_t s) {
+                                int all_bf16, const FwdSaved& saved, unsigned* err,
+                                cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<kF16>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
@@ -674,28 +682,33 @@ cudaError_t launch_fwd_instance(const CUtensorMap& tq, const CUtensorMap& tk,
   const int64_t grid = (int64_t)n_ctiles * BH;
   attn_fwd_tc_kernel<kF16><<<(unsigned)grid, kThreads, kSmemBytes, s>>>(
       tq, tk, tv, static_cast<__nv_bfloat16*>(out), lse, (int)N, (int)BH, n_ctiles, causal,
-      scale * kLog2e, vinfo, static_cast<uint16_t*>(saved.do16), saved.delta, saved.nlse2, err);
+      scale * kLog2e, vinfo, all_bf16, static_cast<uint16_t*>(saved.do16), saved.delta,
+      saved.nlse2, err);
   return cudaGetLastError();
 }
 
-cudaError_t launch_attn_fwd_tc(const void* q, const void* k, const void* v, void* out,
-                               float* lse, int64_t B, int64_t H, int64_t N, int causal,
-                               float scale, const int* vinfo, const FwdSaved& saved,
+cudaError_t launch_attn_fwd_tc(const void* q, const void* k, const void* v, const void* v16,
+                               void* out, float* lse, int64_t B, int64_t H, int64_t N,
+                               int causal, float scale, const int* vinfo, const FwdSaved& saved,
                                unsigned* err, cudaStream_t s, int* launches) {
   const int64_t BH = B * H;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, tv16;
   cudaError_t e;
   if ((e = make_tmap_bf16_rows(&tq, q, BH, N, BM)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_rows(&tk, k, BH, N, BN)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_rows(&tv, v, BH, N, BN)) != cudaSuccess) return e;
-  // f16-operand heads (the usual case) first; the bf16 instance's blocks of
-  // those heads exit at once, and the other way round
-  if ((e = launch_fwd_instance<true>(tq, tk, tv, out, lse, BH, N, causal, scale, vinfo, saved,
-                                     err, s)) != cudaSuccess)
-    return e;
-  *launches += 1;
-  if ((e = launch_fwd_instance<false>(tq, tk, tv, out, lse, BH, N, causal, scale, vinfo, saved,
-                                      err, s)) != cudaSuccess)
+  const int all_bf16 = v16 == nullptr ? 1 : 0;
+  if (!all_bf16) {
+    // f16-operand heads (the usual case) first; the bf16 instance's blocks of
+    // those heads exit at once, and the other way round
+    if ((e = make_tmap_bf16_rows(&tv16, v16, BH, N, BN)) != cudaSuccess) return e;
+    if ((e = launch_fwd_instance<true>(tq, tk, tv16, out, lse, BH, N, causal, scale, vinfo, 0,
+                                       saved, err, s)) != cudaSuccess)
+      return e;
+    *launches += 1;
+  }
+  if ((e = launch_fwd_instance<false>(tq, tk, tv, out, lse, BH, N, causal, scale, vinfo,
+                                      all_bf16, saved, err, s)) != cudaSuccess)
     return e;
   *launches += 1;
   return cudaSuccess;

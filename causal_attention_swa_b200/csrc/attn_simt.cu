@@ -469,7 +469,8 @@ scan_v_info_kernel(const uint4* __restrict__ v, int64_t vec_per_head, int* __res
 // tensor per thread) over the padded rows [BH][Npad] (Npad = N rounded up to
 // 128), 128 rows per block, so a block never spans two heads:
 //   * f16 copies (round to nearest even; exact below 2^15 in magnitude) of
-//     q, k, v and, when given, dout -- the operands of the f16 instance;
+//     v and, when given, q and k, and dout -- the operands of the f16
+//     instances (the forward reads only v's);
 //   * when `out` is given: delta = sum_d dout_d out_d and nlse2 = -lse log2 e
 //     (padding rows: 0 and -inf);
 //   * the per-head info (all four fields; dout's only when dout is given).
@@ -496,12 +497,15 @@ attn_convert_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
     float acc = 0.f;
     if (real) {
       const int64_t vec = (head * N + i) * 8 + part;
-      uint4 x = q[vec];
-      q16[vec] = to_f16x8(x);
-      qke = max(qke, maxexp8(x));
-      x = k[vec];
-      k16[vec] = to_f16x8(x);
-      qke = max(qke, maxexp8(x));
+      uint4 x;
+      if (q != nullptr) {
+        x = q[vec];
+        q16[vec] = to_f16x8(x);
+        qke = max(qke, maxexp8(x));
+        x = k[vec];
+        k16[vec] = to_f16x8(x);
+        qke = max(qke, maxexp8(x));
+      }
       x = v[vec];
       v16[vec] = to_f16x8(x);
       ve = max(ve, maxexp8(x));

@@ -25,11 +25,13 @@ struct FwdSaved {
   float* nlse2 = nullptr;
 };
 
-// vinfo: the per-head V information of launch_scan_v_info.  Two launches
-// (f16-operand and bf16-operand instances; each takes the heads of its type).
-cudaError_t launch_attn_fwd_tc(const void* q, const void* k, const void* v, void* out,
-                               float* lse, int64_t B, int64_t H, int64_t N, int causal,
-                               float scale, const int* vinfo, const FwdSaved& saved,
+// vinfo: the per-head information of the prep pass.  v16: an f16 copy of v
+// (launch_attn_convert); with v16 the f16-operand instance takes the heads
+// within f16's range and the bf16 instance the others (two launches);
+// without it every head takes bf16 operands (one launch).
+cudaError_t launch_attn_fwd_tc(const void* q, const void* k, const void* v, const void* v16,
+                               void* out, float* lse, int64_t B, int64_t H, int64_t N,
+                               int causal, float scale, const int* vinfo, const FwdSaved& saved,
                                unsigned* err, cudaStream_t s, int* launches);
 
 // The four 16-bit operand tensors of a backward instance, [BH][N][64] each.

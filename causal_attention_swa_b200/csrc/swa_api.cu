@@ -93,9 +93,19 @@ swa_status check_attn_shape(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtyp
   return SWA_OK;
 }
 
-// Forward workspace (bf16): the per-head information of the scan of V.
-size_t fwd_ws(int64_t B, int64_t H, swa_dtype dt) {
-  return dt == SWA_BF16 ? round_up((size_t)(B * H) * swa::kHeadInfoInts * sizeof(int), 256) : 0;
+// Forward workspace (bf16 only), in this order:
+//   info  [BH][4] int32       per-head information of the prep pass
+//   v16   [BH][N][64] f16     the f16 copy of V (the f16 instance's operand)
+struct FwdWs {
+  size_t info, total;
+};
+
+FwdWs fwd_ws(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtype dt) {
+  FwdWs w{0, 0};
+  if (dt != SWA_BF16) return w;
+  w.info = round_up((size_t)(B * H) * swa::kHeadInfoInts * sizeof(int), 256);
+  w.total = w.info + round_up((size_t)(B * H * N * D) * 2, 256);
+  return w;
 }
 
 // Backward (and gradient) workspace, in this order:
@@ -162,10 +172,8 @@ void api_end_call(int launches) { t_launches = launches; }
 extern "C" {
 
 size_t swa_attn_fwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtype dt) {
-  (void)N;
-  (void)D;
-  if (B < 1 || H < 1) return 0;
-  return fwd_ws(B, H, dt);
+  if (B < 1 || H < 1 || N < 1 || D < 1) return 0;
+  return fwd_ws(B, H, N, D, dt).total;
 }
 
 swa_status swa_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
@@ -177,7 +185,8 @@ swa_status swa_attn_fwd(const void* q, const void* k, const void* v, void* out, 
   if (st != SWA_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
     return fail(SWA_ERR_INVALID_ARGUMENT, "q, k, v, out, lse must be non-null and 16-byte aligned");
-  const size_t need = fwd_ws(B, H, dt);
+  const FwdWs ws = fwd_ws(B, H, N, D, dt);
+  const size_t need = ws.total;
   if (need && (!aligned16(workspace) || workspace_bytes < need))
     return fail(SWA_ERR_INVALID_ARGUMENT, "workspace must be 16-byte aligned and >= %zu bytes", need);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -192,17 +201,20 @@ swa_status swa_attn_fwd(const void* q, const void* k, const void* v, void* out, 
                                   &launches);
     if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_simt");
   } else {
-    // per-head V information (non-finite values, range), then the
-    // tensor-core kernel for every head
+    // prep: the f16 copy of V and the per-head V information (non-finite
+    // values, range); then the tensor-core kernels for every head
     int* vinfo = static_cast<int*>(workspace);
+    void* v16 = static_cast<char*>(workspace) + ws.info;
     e = cudaMemsetAsync(vinfo, 0, (size_t)BH * swa::kHeadInfoInts * sizeof(int), s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(vinfo)");
-    e = swa::launch_scan_v_info(v, BH, N * D, vinfo, s, &launches);
-    if (e != cudaSuccess) return cuda_fail(e, "scan_v_info");
+    e = swa::launch_attn_convert(nullptr, nullptr, v, nullptr, nullptr, nullptr, nullptr,
+                                 nullptr, v16, nullptr, nullptr, nullptr, vinfo, BH, N, s,
+                                 &launches);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_convert");
     {
       ProfScope ps(SWA_KERNEL_ATTN_FWD, s);
-      e = swa::launch_attn_fwd_tc(q, k, v, out, lse, B, H, N, causal ? 1 : 0, scale, vinfo,
-                                  swa::FwdSaved{}, err, s, &launches);
+      e = swa::launch_attn_fwd_tc(q, k, v, v16, out, lse, B, H, N, causal ? 1 : 0, scale,
+                                  vinfo, swa::FwdSaved{}, err, s, &launches);
     }
     if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_tc");
   }
@@ -324,8 +336,8 @@ swa_status swa_attn_grad(const void* q, const void* k, const void* v, void* out,
     saved.nlse2 = w.nlse2;
     {
       ProfScope ps(SWA_KERNEL_ATTN_FWD, s);
-      e = swa::launch_attn_fwd_tc(q, k, v, out, lse, B, H, N, c, scale, w.info, saved, err, s,
-                                  &launches);
+      e = swa::launch_attn_fwd_tc(q, k, v, w.v16, out, lse, B, H, N, c, scale, w.info, saved,
+                                  err, s, &launches);
     }
     if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_tc");
     {

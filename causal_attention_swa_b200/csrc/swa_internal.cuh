@@ -63,10 +63,10 @@ constexpr int kHeadInfoInts = 4;
 cudaError_t launch_scan_v_info(const void* v, int64_t heads, int64_t elems_per_head,
                                int* info, cudaStream_t s, int* launches);
 
-// The backward's prep pass over [BH][N][64] bf16 tensors: f16 copies of q,
-// k, v (and dout if non-null) into q16, k16, v16 (do16); with `out` non-null
-// (dout then too) delta = dout . out and nlse2 = -lse log2 e per row, [BH][Npad]
-// with padding rows 0 and -inf; the per-head info.
+// The prep pass over [BH][N][64] bf16 tensors: f16 copies of v (and of q and
+// k if q is non-null, of dout if non-null) into v16 (q16, k16, do16); with
+// `out` non-null (dout then too) delta = dout . out and nlse2 = -lse log2 e
+// per row, [BH][Npad] with padding rows 0 and -inf; the per-head info.
 cudaError_t launch_attn_convert(const void* q, const void* k, const void* v, const void* dout,
                                 const void* out, const float* lse, void* q16, void* k16,
                                 void* v16, void* do16, float* delta, float* nlse2, int* info,

@@ -62,8 +62,9 @@ typedef enum {
 } swa_dtype;
 
 /*
- * Bytes of workspace swa_attn_fwd needs (four int32 of per-head information
- * for the bf16 path, 0 for float32).
+ * Bytes of workspace swa_attn_fwd needs: for bf16, four int32 of per-head
+ * information (rounded up to 256 bytes) and an f16 copy of V ([B,H,N,D],
+ * rounded up to 256 bytes); 0 for float32.
  */
 size_t swa_attn_fwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D,
                                    swa_dtype dtype);
@@ -77,12 +78,13 @@ size_t swa_attn_fwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D,
  *   out      [B,H,N,D] of `dtype`         (out)  out_i = sum_j P_ij v_j
  *   lse      [B,H,N] float32              (out)  m_i + ln z_i (natural log)
  *   B, H >= 1; N >= 1; D == 64.
- * The bf16 path runs every head on the tensor cores.  A scan of V finds the
- * heads that hold an infinity or NaN: for those the kernel replaces every
- * non-finite V entry by 0 before its products and gives each output entry
- * the IEEE class of the sum over its existing pairs (every weight > 0), so
- * a masked pair never multiplies a value.  The same scan decides the
- * operand type of P V: f16 (P and V) when every finite |V| < 2^15, else bf16.
+ * The bf16 path runs every head on the tensor cores.  A prep pass over V
+ * writes its f16 copy into the workspace and finds the heads that hold an
+ * infinity or NaN: for those the kernel replaces every non-finite V entry by
+ * 0 before its products and gives each output entry the IEEE class of the
+ * sum over its existing pairs (every weight > 0), so a masked pair never
+ * multiplies a value.  The same pass decides the operand type of P V: f16
+ * (P and the f16 copy of V) when every finite |V| < 2^15, else bf16.
  * float32 inputs run on CUDA cores in float32.
  */
 swa_status swa_attn_fwd(const void* q, const void* k, const void* v, void* out,
@@ -153,7 +155,10 @@ swa_status swa_attn_grad(const void* q, const void* k, const void* v, void* out,
  * pay for cudaMalloc/cudaFree and their implicit synchronisation).  The
  * pages have no counterpart: this is an interface convenience.
  * Same arguments, results and errors as swa_attn_fwd minus the workspace.
- * The forward's scratch (four int32 of information per head) lives in a
+ * With no room for an f16 copy of V, P V takes bf16 operands for every
+ * head (out within the same tolerance, but not bitwise equal to
+ * swa_attn_fwd's).  The forward's scratch (four int32 of information per
+ * head) lives in a
  * static device array for 4096 heads (64 KB, held by every GPU that loads
  * the library until exit); B*H > 4096 returns SWA_ERR_UNSUPPORTED.  The first call on
  * each device looks up the array's device address (make it before any

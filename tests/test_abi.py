@@ -40,7 +40,8 @@ def test_status_strings(lib):
 
 def test_workspace_sizes(lib):
     # bf16 forward: four int32 of per-head information, rounded to 256 bytes
-    assert lib.swa_attn_fwd_workspace_size(2, 16, 16384, 64, swa.SWA_BF16) == 512
+    assert lib.swa_attn_fwd_workspace_size(2, 16, 16384, 64, swa.SWA_BF16) == 512 + 2 * 16 * 16384 * 64 * 2
+    assert lib.swa_attn_fwd_workspace_size(1, 1, 3, 64, swa.SWA_BF16) == 256 + 512
     assert lib.swa_attn_fwd_workspace_size(1, 1, 256, 64, swa.SWA_F32) == 0
     # backward: information + delta and lse*log2(e) padded to 128-row blocks,
     # and for bf16 four f16 operand copies

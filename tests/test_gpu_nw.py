@@ -116,7 +116,7 @@ def check_bwd(t, s, v, g, h, what):
 
 
 @pytest.mark.parametrize("dims", [1, 2, 3])
-@pytest.mark.parametrize("M,S", [(1, 1), (5, 3000), (2500, 1), (1023, 2049), (3000, 4097)])
+@pytest.mark.parametrize("M,S", [(1, 1), (5, 3000), (2500, 2), (1023, 2049), (3000, 4097)])
 def test_nw_gradient_ragged_sizes(dims, M, S):
     rng = np.random.default_rng(M * 13 + S + dims)
     t = rng.uniform(0, 3, size=(M, dims)).astype(np.float32)
@@ -124,6 +124,29 @@ def test_nw_gradient_ragged_sizes(dims, M, S):
     v = rng.normal(size=S).astype(np.float32)
     g = rng.normal(size=M).astype(np.float32)
     check_bwd(t, s, v, g, 0.5, f"{dims}-d {M}x{S}")
+
+
+@pytest.mark.parametrize("dims", [1, 2, 3])
+def test_nw_gradient_single_source(dims):
+    """One source: out_p = (w v) / w = v, so dsources is 0 in exact
+    arithmetic.  float32 leaves out_p within two roundings of v, and each
+    term (2/h^2) g_p (v - out_p) (t_p - s) keeps that rounding: with random
+    roundings the sum stays within 4 standard deviations of
+    (2/h^2) 2^-23 |v| sqrt(sum_p g_p^2 (t_p - s)^2).  dtargets and dvals
+    (= sum_p g_p) are compared as usual."""
+    M, h = 2500, 0.5
+    rng = np.random.default_rng(77 + dims)
+    t = rng.uniform(0, 3, size=(M, dims)).astype(np.float32)
+    s = rng.uniform(0, 3, size=(1, dims)).astype(np.float32)
+    v = rng.normal(size=1).astype(np.float32)
+    g = rng.normal(size=M).astype(np.float32)
+    dt, ds, dv = run_bwd(t, s, v, g, h)
+    w_dt, _, w_dv = oracle.nw_regrid_bwd(t, s, v, g, h=h)
+    check_f32_scaled(dt, w_dt, f"dtargets {dims}-d one source")
+    check_f32_scaled(dv, w_dv, f"dvals {dims}-d one source")
+    sigma = (2.0 / h ** 2) * 2.0 ** -23 * abs(float(v[0])) * \
+        float(np.sqrt((g[:, None].astype(np.float64) ** 2 * (t - s) ** 2).sum(axis=0)).max())
+    assert float(np.abs(ds.cpu().numpy()).max()) <= 4 * sigma, (ds, sigma)
 
 
 @pytest.mark.parametrize("dims", [2, 3])

@@ -4,9 +4,12 @@ or their latency budget rules out cudaMalloc and its synchronisation).  Its
 per-head scratch lives in a static device array shared by every call, so
 this test makes two calls in a row -- the first with a head whose V holds
 +inf (its flag gets set), the second with all heads finite (the flag must
-have been cleared) -- and checks each against swa_attn_fwd on the same
-inputs, through the C ABI, with the parity tests' tolerances.  It is
-collected last so a failure here cannot hide the other tests' results."""
+have been cleared) -- and checks each against the float64 oracle with the
+parity tests' tolerances, through the C ABI.  Without room for an f16 copy
+of V its P V products take bf16 operands, so it is not bitwise equal to
+swa_attn_fwd: each is within the per-row bound of the exact result, so the
+two lie within twice that bound of each other.  It is collected last so a
+failure here cannot hide the other tests' results."""
 import ctypes
 
 import numpy as np
@@ -15,7 +18,7 @@ import torch
 
 import oracle
 from causal_attention_swa_b200 import inputs, swa
-from _compare import check_bf16, check_f32, check_lse
+from _compare import BF16_REL, check_bf16, check_f32, check_lse
 
 pytestmark = pytest.mark.gpu
 
@@ -47,7 +50,7 @@ def _bf16_dev(bits):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-def test_noalloc_forward_matches_the_workspace_forward_twice_in_a_row():
+def test_noalloc_forward_matches_the_oracle_twice_in_a_row():
     torch.cuda.init()
     rng = np.random.default_rng(77)
     shape = (2, 3, 300, 64)
@@ -60,12 +63,13 @@ def test_noalloc_forward_matches_the_workspace_forward_twice_in_a_row():
         want_out, want_lse = swa.attn_fwd(q, k, v, causal=True)
         torch.cuda.synchronize()
         assert swa.get_device_error() == swa.SWA_OK
-        check_bf16(got_out, want_out, "out (noalloc vs workspace forward)")
-        check_lse(got_lse, want_lse, "lse (noalloc vs workspace forward)")
-        # and against the float64 oracle itself (classes of the +inf head included)
+        # the float64 oracle (classes of the +inf head included)
         w_out, w_lse = oracle.attn_fwd(*(inputs.bf16_to_f64(b) for b in bits))
         check_bf16(got_out, w_out, "out (noalloc vs oracle)")
         check_lse(got_lse, w_lse, "lse (noalloc vs oracle)")
+        # the workspace forward: both within BF16_REL of the exact rows
+        check_bf16(got_out, want_out, "out (noalloc vs workspace forward)", rel=2 * BF16_REL)
+        check_lse(got_lse, want_lse, "lse (noalloc vs workspace forward)")
     o = got_out.float().cpu().numpy()
     assert np.isfinite(o).all()                # second call: no stale flag, no inf
 
