@@ -54,9 +54,9 @@
 // read from an f16 copy of V (the caller's prep pass writes it), for every
 // head whose finite V values lie below 2^15 in magnitude (f16 holds them
 // exactly, up to f16's subnormal spacing of 2^-24); a head with larger
-// values keeps both in bf16 (V as given).  A bf16 P (7 fraction bits) is exact enough for the output itself,
-// but the output is what the gradient of loss = 1/2 sum out^2 feeds back
-// as dout, and the rounding of few-key rows (early rows) reaches the
+// values keeps both in bf16 (V as given).  A bf16 P (7 fraction bits) is
+// exact enough for the output itself, but the output is what the gradient
+// of loss = 1/2 sum out^2 feeds back as dout, and the rounding of few-key rows (early rows) reaches the
 // gradient amplified by the cancellation in sum_j dS_ij k_j; with the f16 P
 // the end-to-end gradient stays inside the bf16 path's tolerance.  Rows
 // that see few keys (the first rows of a causal head) average no rounding
@@ -120,6 +120,7 @@ constexpr int kTmaWarp = kSoftmaxWarps;
 constexpr int kMmaWarp = kSoftmaxWarps + 1;  // issuer of tile 0; kMmaWarp + 1 issues tile 1
 constexpr int kHalf = BN / 2;                // score columns per softmax thread
 constexpr uint32_t kTmemCols = 512;
+constexpr int kHeadGroup = 4;                // heads scheduled together (K, V share L2)
 constexpr float kRescaleThreshold = 8.0f;
 // A P computed against a stale reference max must still fit the operand
 // type before it is moved to the new max: < 2^15 in f16, < 2^64 in bf16.
@@ -167,40 +168,59 @@ __device__ __forceinline__ bool wait_unbounded_by_abort(uint64_t* bar, uint32_t 
   return true;
 }
 
-// Rewrites one staged V tile of a head whose V holds an infinity or NaN
-// (128 rows of 128 bytes, 128-byte swizzle) in place: a non-finite 16-bit
-// entry (f16 in the f16 instance, bf16 in the other) becomes 0 and its row
-// goes into first_cls.  16-byte chunks without one are left untouched.
+// The V cleaner's unit: one 16-byte chunk c (row c / 8 of the staged tile,
+// 128-byte swizzle) of a head whose V holds an infinity or NaN.  A
+// non-finite 16-bit entry (f16 in the f16 instance, bf16 in the other)
+// becomes 0 and its key row goes into first_cls (per column: first row with
+// +inf, -inf, NaN).
 template <bool kF16>
-__device__ __forceinline__ void clean_v_tile(uint8_t* tile, int lane, int key0,
-                                             int (*first_cls)[HD]) {
+__device__ __forceinline__ void clean_v_chunk(uint4* base, int c, int key0,
+                                              int (*first_cls)[HD]) {
   constexpr uint32_t kExp = kF16 ? 0x7C00u : 0x7F80u;   // exponent field all ones
   constexpr uint32_t kMan = kF16 ? 0x03FFu : 0x007Fu;   // fraction: non-zero = NaN
-  uint4* base = reinterpret_cast<uint4*>(tile);
-#pragma unroll 2
-  for (int c = lane; c < kTileBytes / 16; c += 32) {
-    const uint4 x = base[c];
-    uint32_t w[4] = {x.x, x.y, x.z, x.w};
-    bool any = false;
+  const uint4 x = base[c];
+  uint32_t w[4] = {x.x, x.y, x.z, x.w};
+  bool any = false;
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
-      any |= ((w[e] & kExp) == kExp) | (((w[e] >> 16) & kExp) == kExp);
-    if (!any) continue;
-    const int r = c >> 3;                      // row of the tile
-    const int d0 = ((c & 7) ^ (r & 7)) * 8;    // its first column (swizzle undone)
+  for (int e = 0; e < 4; ++e)
+    any |= ((w[e] & kExp) == kExp) | (((w[e] >> 16) & kExp) == kExp);
+  if (!any) return;
+  const int r = c >> 3;                      // row of the tile
+  const int d0 = ((c & 7) ^ (r & 7)) * 8;    // its first column (swizzle undone)
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
+  for (int e = 0; e < 4; ++e)
 #pragma unroll
-      for (int p = 0; p < 2; ++p) {
-        const uint32_t b = (w[e] >> (16 * p)) & 0xFFFFu;
-        if ((b & kExp) == kExp) {
-          const int cls = (b & kMan) ? 2 : ((b & 0x8000u) ? 1 : 0);
-          atomicMin(&first_cls[cls][d0 + 2 * e + p], key0 + r);
-          w[e] &= ~(0xFFFFu << (16 * p));
-        }
+    for (int p = 0; p < 2; ++p) {
+      const uint32_t b = (w[e] >> (16 * p)) & 0xFFFFu;
+      if ((b & kExp) == kExp) {
+        const int cls = (b & kMan) ? 2 : ((b & 0x8000u) ? 1 : 0);
+        atomicMin(&first_cls[cls][d0 + 2 * e + p], key0 + r);
+        w[e] &= ~(0xFFFFu << (16 * p));
       }
-    base[c] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  base[c] = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Cleans one staged V tile (128 rows of 128 bytes).  With the prep pass's
+// row mask of the tile (rows holding a non-finite entry) only those rows are
+// read, 8 lanes per row; without it, every chunk.
+template <bool kF16>
+__device__ __forceinline__ void clean_v_tile(uint8_t* tile, int lane, int key0,
+                                             const uint4* rowmask, int (*first_cls)[HD]) {
+  uint4* base = reinterpret_cast<uint4*>(tile);
+  if (rowmask != nullptr) {
+    const uint4 m4 = *rowmask;
+    const uint32_t words[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll 1
+    for (int wd = 0; wd < 4; ++wd)
+      for (uint32_t m = words[wd]; m != 0u; m &= m - 1u) {  // warp-uniform
+        const int r = 32 * wd + (__ffs(m) - 1);
+        if (lane < 8) clean_v_chunk<kF16>(base, r * 8 + lane, key0, first_cls);
+      }
+    return;
   }
+#pragma unroll 2
+  for (int c = lane; c < kTileBytes / 16; c += 32) clean_v_chunk<kF16>(base, c, key0, first_cls);
 }
 
 template <bool kF16>
@@ -209,12 +229,18 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
                    float* __restrict__ lse, int N, int BH, int n_ctiles, int causal,
-                   float scale_log2, const int* __restrict__ vinfo, int all_bf16,
+                   float scale_log2, const int* __restrict__ vinfo,
+                   const uint4* __restrict__ vrows, int all_bf16,
                    uint16_t* __restrict__ do16, float* __restrict__ delta,
                    float* __restrict__ nlse2, unsigned* __restrict__ err) {
-  // Longest first: every head's latest (heaviest) query tiles, then the next.
-  const int head = blockIdx.x % BH;
-  const int c = n_ctiles - 1 - blockIdx.x / BH;
+  // Heads in groups of kHeadGroup, whose K and V (4 MB per head at N = 16384)
+  // stay in L2 while the group's blocks run; inside a group the heaviest
+  // (latest) query tiles first, heads interleaved.
+  const int group = blockIdx.x / (kHeadGroup * n_ctiles);
+  const int g_heads = min(kHeadGroup, BH - group * kHeadGroup);
+  const int rr = blockIdx.x - group * kHeadGroup * n_ctiles;
+  const int head = group * kHeadGroup + rr % g_heads;
+  const int c = n_ctiles - 1 - rr / g_heads;
   const bool nonfinite = (vinfo[kHeadInfoInts * head] & 1) != 0;
   const bool f16_head = !all_bf16 && vinfo[kHeadInfoInts * head + 1] < kF16ExpLimit;
   if (f16_head != kF16) return;  // the other instance's head
@@ -362,7 +388,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int s = j % kStages;
         if (!mbar_wait_parked(&sm.v_full[s], (j / kStages) & 1, abort, err, kDevTimeoutFull))
           break;
-        clean_v_tile<kF16>(sm.v[s], lane, j * BN, sm.first_cls);
+        const uint4* rowmask =
+            vrows != nullptr ? vrows + (size_t)head * ((N + BN - 1) / BN) + j : nullptr;
+        clean_v_tile<kF16>(sm.v[s], lane, j * BN, rowmask, sm.first_cls);
         fence_proxy_async_smem();  // the MMA (async proxy) reads what was written
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.v_ready[s]);
@@ -668,8 +696,8 @@ template <bool kF16>
 cudaError_t launch_fwd_instance(const CUtensorMap& tq, const CUtensorMap& tk,
                                 const CUtensorMap& tv, void* out, float* lse, int64_t BH,
                                 int64_t N, int causal, float scale, const int* vinfo,
-                                int all_bf16, const FwdSaved& saved, unsigned* err,
-                                cudaStream_t s) {
+                                const unsigned* vrows, int all_bf16, const FwdSaved& saved,
+                                unsigned* err, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<kF16>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
@@ -682,15 +710,17 @@ cudaError_t launch_fwd_instance(const CUtensorMap& tq, const CUtensorMap& tk,
   const int64_t grid = (int64_t)n_ctiles * BH;
   attn_fwd_tc_kernel<kF16><<<(unsigned)grid, kThreads, kSmemBytes, s>>>(
       tq, tk, tv, static_cast<__nv_bfloat16*>(out), lse, (int)N, (int)BH, n_ctiles, causal,
-      scale * kLog2e, vinfo, all_bf16, static_cast<uint16_t*>(saved.do16), saved.delta,
+      scale * kLog2e, vinfo, reinterpret_cast<const uint4*>(vrows), all_bf16,
+      static_cast<uint16_t*>(saved.do16), saved.delta,
       saved.nlse2, err);
   return cudaGetLastError();
 }
 
 cudaError_t launch_attn_fwd_tc(const void* q, const void* k, const void* v, const void* v16,
                                void* out, float* lse, int64_t B, int64_t H, int64_t N,
-                               int causal, float scale, const int* vinfo, const FwdSaved& saved,
-                               unsigned* err, cudaStream_t s, int* launches) {
+                               int causal, float scale, const int* vinfo, const unsigned* vrows,
+                               const FwdSaved& saved, unsigned* err, cudaStream_t s,
+                               int* launches) {
   const int64_t BH = B * H;
   CUtensorMap tq, tk, tv, tv16;
   cudaError_t e;
@@ -702,13 +732,13 @@ cudaError_t launch_attn_fwd_tc(const void* q, const void* k, const void* v, cons
     // f16-operand heads (the usual case) first; the bf16 instance's blocks of
     // those heads exit at once, and the other way round
     if ((e = make_tmap_bf16_rows(&tv16, v16, BH, N, BN)) != cudaSuccess) return e;
-    if ((e = launch_fwd_instance<true>(tq, tk, tv16, out, lse, BH, N, causal, scale, vinfo, 0,
-                                       saved, err, s)) != cudaSuccess)
+    if ((e = launch_fwd_instance<true>(tq, tk, tv16, out, lse, BH, N, causal, scale, vinfo,
+                                       vrows, 0, saved, err, s)) != cudaSuccess)
       return e;
     *launches += 1;
   }
   if ((e = launch_fwd_instance<false>(tq, tk, tv, out, lse, BH, N, causal, scale, vinfo,
-                                      all_bf16, saved, err, s)) != cudaSuccess)
+                                      vrows, all_bf16, saved, err, s)) != cudaSuccess)
     return e;
   *launches += 1;
   return cudaSuccess;

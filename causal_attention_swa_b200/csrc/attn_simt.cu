@@ -473,7 +473,10 @@ scan_v_info_kernel(const uint4* __restrict__ v, int64_t vec_per_head, int* __res
 //     instances (the forward reads only v's);
 //   * when `out` is given: delta = sum_d dout_d out_d and nlse2 = -lse log2 e
 //     (padding rows: 0 and -inf);
-//   * the per-head info (all four fields; dout's only when dout is given).
+//   * the per-head info (all four fields; dout's only when dout is given);
+//   * when `vrows` is given: per 128-row tile of V, a 128-bit mask of its
+//     rows that hold an infinity or NaN ([BH][Npad / 128][4] uint32; bit
+//     r % 32 of word r / 32 for row r of the tile), every word written.
 constexpr int kConvRows = 128;
 __global__ void __launch_bounds__(256)
 attn_convert_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
@@ -481,9 +484,12 @@ attn_convert_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
                     const uint4* __restrict__ out, const float* __restrict__ lse,
                     uint4* __restrict__ q16, uint4* __restrict__ k16, uint4* __restrict__ v16,
                     uint4* __restrict__ do16, float* __restrict__ delta,
-                    float* __restrict__ nlse2, int* __restrict__ info, int64_t N, int64_t Npad) {
+                    float* __restrict__ nlse2, int* __restrict__ info,
+                    unsigned* __restrict__ vrows, int64_t N, int64_t Npad) {
   __shared__ unsigned sh[4];
+  __shared__ unsigned rows_nf[kConvRows / 32];  // this tile's rows with a non-finite V entry
   if (threadIdx.x < 4) sh[threadIdx.x] = 0u;
+  if (threadIdx.x < kConvRows / 32) rows_nf[threadIdx.x] = 0u;
   __syncthreads();
   const int64_t rp0 = (int64_t)blockIdx.x * kConvRows;
   const int64_t head = rp0 / Npad;
@@ -509,7 +515,11 @@ attn_convert_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
       x = v[vec];
       v16[vec] = to_f16x8(x);
       ve = max(ve, maxexp8(x));
-      fl |= nonfinite8(x) ? 1u : 0u;
+      if (nonfinite8(x)) {
+        fl |= 1u;
+        const int r = it * 32 + (threadIdx.x >> 3);  // row within the tile
+        atomicOr(&rows_nf[r >> 5], 1u << (r & 31));
+      }
       if (dout != nullptr) {
         x = dout[vec];
         do16[vec] = to_f16x8(x);
@@ -528,7 +538,9 @@ attn_convert_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
       }
     }
   }
-  flush_info(fl, ve, qke, de, info + 4 * head, sh);
+  flush_info(fl, ve, qke, de, info + 4 * head, sh);  // (its __syncthreads covers rows_nf)
+  if (vrows != nullptr && threadIdx.x < kConvRows / 32)
+    vrows[(int64_t)blockIdx.x * (kConvRows / 32) + threadIdx.x] = rows_nf[threadIdx.x];
 }
 
 template <typename T>
@@ -592,12 +604,14 @@ cudaError_t launch_scan_v_info(const void* v, int64_t heads, int64_t elems_per_h
 cudaError_t launch_attn_convert(const void* q, const void* k, const void* v, const void* dout,
                                 const void* out, const float* lse, void* q16, void* k16,
                                 void* v16, void* do16, float* delta, float* nlse2, int* info,
-                                int64_t BH, int64_t N, cudaStream_t s, int* launches) {
+                                unsigned* vrows, int64_t BH, int64_t N, cudaStream_t s,
+                                int* launches) {
   const int64_t Npad = pad128(N);
   const int64_t blocks = BH * Npad / kConvRows;
   attn_convert_kernel<<<(unsigned)blocks, 256, 0, s>>>(
       (const uint4*)q, (const uint4*)k, (const uint4*)v, (const uint4*)dout, (const uint4*)out,
-      lse, (uint4*)q16, (uint4*)k16, (uint4*)v16, (uint4*)do16, delta, nlse2, info, N, Npad);
+      lse, (uint4*)q16, (uint4*)k16, (uint4*)v16, (uint4*)do16, delta, nlse2, info, vrows, N,
+      Npad);
   *launches += 1;
   return cudaGetLastError();
 }

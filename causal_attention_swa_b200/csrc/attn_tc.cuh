@@ -28,11 +28,14 @@ struct FwdSaved {
 // vinfo: the per-head information of the prep pass.  v16: an f16 copy of v
 // (launch_attn_convert); with v16 the f16-operand instance takes the heads
 // within f16's range and the bf16 instance the others (two launches);
-// without it every head takes bf16 operands (one launch).
+// without it every head takes bf16 operands (one launch).  vrows (nullable):
+// the prep pass's per-tile masks of V rows with a non-finite entry, which
+// let the V cleaner of a flagged head skip clean rows.
 cudaError_t launch_attn_fwd_tc(const void* q, const void* k, const void* v, const void* v16,
                                void* out, float* lse, int64_t B, int64_t H, int64_t N,
-                               int causal, float scale, const int* vinfo, const FwdSaved& saved,
-                               unsigned* err, cudaStream_t s, int* launches);
+                               int causal, float scale, const int* vinfo, const unsigned* vrows,
+                               const FwdSaved& saved, unsigned* err, cudaStream_t s,
+                               int* launches);
 
 // The four 16-bit operand tensors of a backward instance, [BH][N][64] each.
 struct BwdOperands {

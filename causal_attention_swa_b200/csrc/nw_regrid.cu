@@ -104,36 +104,50 @@ nw_partial_kernel(const float* __restrict__ targets, int64_t M,
   }
 }
 
-// Block = 32 targets x 8 chunk groups: thread (g, t) adds chunks g, g + 8,
-// ... of target t (32 consecutive targets per chunk: coalesced 256-byte
-// reads), then thread (0, t) adds the eight group sums in order.
-constexpr int kFinTargets = 32;
+// Block = 32 lanes x 8 chunk groups; lane t holds kFinVec consecutive
+// targets (2: one 16-byte load of two (sum w, sum w v) pairs, when M is
+// even; else 1).  Thread (g, t) adds chunks g, g + 8, ... (each chunk's 32
+// lanes read 256 or 512 contiguous bytes), then thread (0, t) adds the eight
+// group sums in order: the result does not depend on timing.
+constexpr int kFinLanes = 32;
 constexpr int kFinGroups = 8;
-__global__ void __launch_bounds__(kFinTargets * kFinGroups)
+template <int kFinVec>
+__global__ void __launch_bounds__(kFinLanes * kFinGroups)
 nw_finalize_kernel(const float2* __restrict__ partials, int nchunks, int64_t M,
                    float* __restrict__ out) {
-  __shared__ float2 part[kFinGroups][kFinTargets];
-  const int t = threadIdx.x % kFinTargets, g = threadIdx.x / kFinTargets;
-  const int64_t p = (int64_t)blockIdx.x * kFinTargets + t;
-  float2 acc = make_float2(0.f, 0.f);
+  __shared__ float4 part[kFinGroups][kFinLanes];
+  const int t = threadIdx.x % kFinLanes, g = threadIdx.x / kFinLanes;
+  const int64_t p = ((int64_t)blockIdx.x * kFinLanes + t) * kFinVec;  // first target
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);  // (sw, swv) of targets p, p + 1
   if (p < M) {
-#pragma unroll 4
+#pragma unroll 8
     for (int ch = g; ch < nchunks; ch += kFinGroups) {
-      const float2 a = partials[(int64_t)ch * M + p];
-      acc.x += a.x;
-      acc.y += a.y;
+      if constexpr (kFinVec == 2) {
+        const float4 a = *reinterpret_cast<const float4*>(partials + (int64_t)ch * M + p);
+        acc.x += a.x;
+        acc.y += a.y;
+        acc.z += a.z;
+        acc.w += a.w;
+      } else {
+        const float2 a = partials[(int64_t)ch * M + p];
+        acc.x += a.x;
+        acc.y += a.y;
+      }
     }
   }
   part[g][t] = acc;
   __syncthreads();
   if (g == 0 && p < M) {
-    float sw = 0.f, swv = 0.f;
+    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < kFinGroups; ++i) {
-      sw += part[i][t].x;
-      swv += part[i][t].y;
+      sum.x += part[i][t].x;
+      sum.y += part[i][t].y;
+      sum.z += part[i][t].z;
+      sum.w += part[i][t].w;
     }
-    out[p] = swv / sw;
+    out[p] = sum.y / sum.x;
+    if (kFinVec == 2) out[p + 1] = sum.w / sum.z;  // M even: p + 1 < M
   }
 }
 
@@ -187,9 +201,14 @@ cudaError_t launch_nw_partial(const float* targets, int64_t M, const float* sour
 cudaError_t launch_nw_finalize(int64_t M, int64_t S, const float* partials, float* out,
                                cudaStream_t s, int* launches) {
   const Plan pl = plan(M, S);
-  nw_finalize_kernel<<<(unsigned)((M + kFinTargets - 1) / kFinTargets),
-                       kFinTargets * kFinGroups, 0, s>>>(
-      reinterpret_cast<const float2*>(partials), (int)pl.nchunks, M, out);
+  const auto* part = reinterpret_cast<const float2*>(partials);
+  constexpr unsigned kBlock = kFinLanes * kFinGroups;
+  if (M % 2 == 0)  // every chunk row starts on a 16-byte boundary
+    nw_finalize_kernel<2><<<(unsigned)((M / 2 + kFinLanes - 1) / kFinLanes), kBlock, 0, s>>>(
+        part, (int)pl.nchunks, M, out);
+  else
+    nw_finalize_kernel<1><<<(unsigned)((M + kFinLanes - 1) / kFinLanes), kBlock, 0, s>>>(
+        part, (int)pl.nchunks, M, out);
   *launches += 1;
   return cudaGetLastError();
 }

@@ -93,42 +93,54 @@ swa_status check_attn_shape(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtyp
   return SWA_OK;
 }
 
+// Per 128-row tile of V, the mask of its rows that hold an infinity or NaN:
+// [BH][Npad / 128][4] uint32 (written whole by the prep pass).
+size_t vrows_bytes(int64_t B, int64_t H, int64_t N) {
+  return round_up((size_t)(B * H) * (size_t)(swa::pad128(N) / 128) * 16, 256);
+}
+
 // Forward workspace (bf16 only), in this order:
-//   info  [BH][4] int32       per-head information of the prep pass
-//   v16   [BH][N][64] f16     the f16 copy of V (the f16 instance's operand)
+//   info   [BH][4] int32            per-head information of the prep pass
+//   vrows  [BH][Npad/128][4] uint32 non-finite row masks of V's tiles
+//   v16    [BH][N][64] f16          the f16 copy of V (the f16 instance's operand)
 struct FwdWs {
-  size_t info, total;
+  size_t info, vrows, total;
 };
 
 FwdWs fwd_ws(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtype dt) {
-  FwdWs w{0, 0};
+  FwdWs w{0, 0, 0};
   if (dt != SWA_BF16) return w;
   w.info = round_up((size_t)(B * H) * swa::kHeadInfoInts * sizeof(int), 256);
-  w.total = w.info + round_up((size_t)(B * H * N * D) * 2, 256);
+  w.vrows = vrows_bytes(B, H, N);
+  w.total = w.info + w.vrows + round_up((size_t)(B * H * N * D) * 2, 256);
   return w;
 }
 
 // Backward (and gradient) workspace, in this order:
 //   info   [BH][4] int32        per-head information
+//   vrows  [BH][Npad/128][4] uint32  non-finite row masks of V's tiles (the
+//                               gradient's forward reads them)
 //   delta  [BH][Npad] float32   dout . out per row (Npad = N rounded up to 128)
 //   nlse2  [BH][Npad] float32   -lse log2 e per row
 //   q16, k16, v16, do16  [BH][N][64] f16 each (bf16 only): the f16 operands
 struct BwdWs {
-  size_t info, delta, nlse2, copy, total;
+  size_t info, vrows, delta, nlse2, copy, total;
 };
 
 BwdWs bwd_ws(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtype dt) {
   BwdWs w;
   w.info = round_up((size_t)(B * H) * swa::kHeadInfoInts * sizeof(int), 256);
+  w.vrows = dt == SWA_BF16 ? vrows_bytes(B, H, N) : 0;
   w.delta = round_up((size_t)(B * H * swa::pad128(N)) * sizeof(float), 256);
   w.nlse2 = w.delta;
   w.copy = dt == SWA_BF16 ? round_up((size_t)(B * H * N * D) * 2, 256) : 0;
-  w.total = w.info + w.delta + w.nlse2 + 4 * w.copy;
+  w.total = w.info + w.vrows + w.delta + w.nlse2 + 4 * w.copy;
   return w;
 }
 
 struct BwdPtrs {
   int* info;
+  unsigned* vrows;
   float* delta;
   float* nlse2;
   void* q16;
@@ -141,9 +153,10 @@ BwdPtrs carve(void* workspace, const BwdWs& w) {
   char* b = static_cast<char*>(workspace);
   BwdPtrs p;
   p.info = reinterpret_cast<int*>(b);
-  p.delta = reinterpret_cast<float*>(b + w.info);
-  p.nlse2 = reinterpret_cast<float*>(b + w.info + w.delta);
-  char* c = b + w.info + w.delta + w.nlse2;
+  p.vrows = reinterpret_cast<unsigned*>(b + w.info);
+  p.delta = reinterpret_cast<float*>(b + w.info + w.vrows);
+  p.nlse2 = reinterpret_cast<float*>(b + w.info + w.vrows + w.delta);
+  char* c = b + w.info + w.vrows + w.delta + w.nlse2;
   p.q16 = c;
   p.k16 = c + w.copy;
   p.v16 = c + 2 * w.copy;
@@ -204,17 +217,18 @@ swa_status swa_attn_fwd(const void* q, const void* k, const void* v, void* out, 
     // prep: the f16 copy of V and the per-head V information (non-finite
     // values, range); then the tensor-core kernels for every head
     int* vinfo = static_cast<int*>(workspace);
-    void* v16 = static_cast<char*>(workspace) + ws.info;
+    unsigned* vrows = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + ws.info);
+    void* v16 = static_cast<char*>(workspace) + ws.info + ws.vrows;
     e = cudaMemsetAsync(vinfo, 0, (size_t)BH * swa::kHeadInfoInts * sizeof(int), s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(vinfo)");
     e = swa::launch_attn_convert(nullptr, nullptr, v, nullptr, nullptr, nullptr, nullptr,
-                                 nullptr, v16, nullptr, nullptr, nullptr, vinfo, BH, N, s,
+                                 nullptr, v16, nullptr, nullptr, nullptr, vinfo, vrows, BH, N, s,
                                  &launches);
     if (e != cudaSuccess) return cuda_fail(e, "attn_convert");
     {
       ProfScope ps(SWA_KERNEL_ATTN_FWD, s);
       e = swa::launch_attn_fwd_tc(q, k, v, v16, out, lse, B, H, N, causal ? 1 : 0, scale,
-                                  vinfo, swa::FwdSaved{}, err, s, &launches);
+                                  vinfo, vrows, swa::FwdSaved{}, err, s, &launches);
     }
     if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_tc");
   }
@@ -267,7 +281,7 @@ swa_status swa_attn_bwd(const void* q, const void* k, const void* v, const void*
     e = cudaMemsetAsync(w.info, 0, (size_t)BH * swa::kHeadInfoInts * sizeof(int), s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(info)");
     e = swa::launch_attn_convert(q, k, v, dout, out, lse, w.q16, w.k16, w.v16, w.do16, w.delta,
-                                 w.nlse2, w.info, BH, N, s, &launches);
+                                 w.nlse2, w.info, nullptr, BH, N, s, &launches);
     if (e != cudaSuccess) return cuda_fail(e, "attn_convert");
     {
       ProfScope ps(SWA_KERNEL_ATTN_BWD, s);
@@ -328,7 +342,7 @@ swa_status swa_attn_grad(const void* q, const void* k, const void* v, void* out,
     e = cudaMemsetAsync(w.info, 0, (size_t)BH * swa::kHeadInfoInts * sizeof(int), s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(info)");
     e = swa::launch_attn_convert(q, k, v, nullptr, nullptr, nullptr, w.q16, w.k16, w.v16,
-                                 nullptr, nullptr, nullptr, w.info, BH, N, s, &launches);
+                                 nullptr, nullptr, nullptr, w.info, w.vrows, BH, N, s, &launches);
     if (e != cudaSuccess) return cuda_fail(e, "attn_convert");
     swa::FwdSaved saved;
     saved.do16 = w.do16;
@@ -336,8 +350,8 @@ swa_status swa_attn_grad(const void* q, const void* k, const void* v, void* out,
     saved.nlse2 = w.nlse2;
     {
       ProfScope ps(SWA_KERNEL_ATTN_FWD, s);
-      e = swa::launch_attn_fwd_tc(q, k, v, w.v16, out, lse, B, H, N, c, scale, w.info, saved,
-                                  err, s, &launches);
+      e = swa::launch_attn_fwd_tc(q, k, v, w.v16, out, lse, B, H, N, c, scale, w.info, w.vrows,
+                                  saved, err, s, &launches);
     }
     if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_tc");
     {

@@ -66,11 +66,14 @@ cudaError_t launch_scan_v_info(const void* v, int64_t heads, int64_t elems_per_h
 // The prep pass over [BH][N][64] bf16 tensors: f16 copies of v (and of q and
 // k if q is non-null, of dout if non-null) into v16 (q16, k16, do16); with
 // `out` non-null (dout then too) delta = dout . out and nlse2 = -lse log2 e
-// per row, [BH][Npad] with padding rows 0 and -inf; the per-head info.
+// per row, [BH][Npad] with padding rows 0 and -inf; the per-head info; if
+// vrows is non-null, per 128-row tile of V the mask of its rows that hold an
+// infinity or NaN ([BH][Npad / 128][4] uint32, every word written).
 cudaError_t launch_attn_convert(const void* q, const void* k, const void* v, const void* dout,
                                 const void* out, const float* lse, void* q16, void* k16,
                                 void* v16, void* do16, float* delta, float* nlse2, int* info,
-                                int64_t BH, int64_t N, cudaStream_t s, int* launches);
+                                unsigned* vrows, int64_t BH, int64_t N, cudaStream_t s,
+                                int* launches);
 
 cudaError_t launch_attn_fwd_simt(swa_dtype dt, const void* q, const void* k, const void* v,
                                  void* out, float* lse, int64_t BH, int64_t N, int causal,

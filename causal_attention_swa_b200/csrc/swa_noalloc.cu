@@ -91,8 +91,8 @@ extern "C" swa_status swa_attn_fwd_noalloc(const void* q, const void* k, const v
     if (e != cudaSuccess) return swa::api_cuda_fail(e, "cudaMemsetAsync(noalloc scratch)");
     e = swa::launch_scan_v_info(v, BH, N * D, vinfo, s, &launches);
     if (e != cudaSuccess) return swa::api_cuda_fail(e, "scan_v_info");
-    e = swa::launch_attn_fwd_tc(q, k, v, nullptr, out, lse, B, H, N, c, scale, vinfo, swa::FwdSaved{},
-                                 err, s, &launches);
+    e = swa::launch_attn_fwd_tc(q, k, v, nullptr, out, lse, B, H, N, c, scale, vinfo, nullptr,
+                                swa::FwdSaved{}, err, s, &launches);
     if (e != cudaSuccess) return swa::api_cuda_fail(e, "attn_fwd_tc");
   }
   swa::api_end_call(launches);

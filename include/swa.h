@@ -63,8 +63,9 @@ typedef enum {
 
 /*
  * Bytes of workspace swa_attn_fwd needs: for bf16, four int32 of per-head
- * information (rounded up to 256 bytes) and an f16 copy of V ([B,H,N,D],
- * rounded up to 256 bytes); 0 for float32.
+ * information, a 128-bit mask per 128-row tile of V (its rows that hold an
+ * infinity or NaN) and an f16 copy of V ([B,H,N,D]), each rounded up to 256
+ * bytes; 0 for float32.
  */
 size_t swa_attn_fwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D,
                                    swa_dtype dtype);
@@ -94,8 +95,11 @@ swa_status swa_attn_fwd(const void* q, const void* k, const void* v, void* out,
 
 /*
  * Bytes of workspace swa_attn_bwd needs: per-head information (four int32),
- * delta and lse * log2(e) as float32 [B,H,Npad] each (Npad = N rounded up to
- * 128) and, for bf16, f16 copies of q, k, v and dout ([B,H,N,D] each).
+ * for bf16 a 128-bit mask per 128-row tile of V (rows holding an infinity or
+ * NaN; the gradient call's forward reads it), delta and lse * log2(e) as
+ * float32 [B,H,Npad] each (Npad = N rounded up to 128) and, for bf16, f16
+ * copies of q, k, v and dout ([B,H,N,D] each); each part rounded up to 256
+ * bytes.
  */
 size_t swa_attn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D,
                                    swa_dtype dtype);

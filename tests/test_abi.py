@@ -39,14 +39,17 @@ def test_status_strings(lib):
 
 
 def test_workspace_sizes(lib):
-    # bf16 forward: four int32 of per-head information, rounded to 256 bytes
-    assert lib.swa_attn_fwd_workspace_size(2, 16, 16384, 64, swa.SWA_BF16) == 512 + 2 * 16 * 16384 * 64 * 2
-    assert lib.swa_attn_fwd_workspace_size(1, 1, 3, 64, swa.SWA_BF16) == 256 + 512
-    assert lib.swa_attn_fwd_workspace_size(1, 1, 256, 64, swa.SWA_F32) == 0
-    # backward: information + delta and lse*log2(e) padded to 128-row blocks,
-    # and for bf16 four f16 operand copies
+    # bf16 forward: four int32 of per-head information and the per-tile masks
+    # of V rows with a non-finite entry (16 bytes per 128-row tile), each
+    # rounded to 256 bytes, then the f16 copy of V
     B, H, N, D = 2, 16, 16384, 64
-    want = 512 + 2 * B * H * N * 4 + 4 * B * H * N * D * 2
+    rows = 2 * 16 * (16384 // 128) * 16
+    assert lib.swa_attn_fwd_workspace_size(B, H, N, D, swa.SWA_BF16) == 512 + rows + B * H * N * D * 2
+    assert lib.swa_attn_fwd_workspace_size(1, 1, 3, 64, swa.SWA_BF16) == 256 + 256 + 512
+    assert lib.swa_attn_fwd_workspace_size(1, 1, 256, 64, swa.SWA_F32) == 0
+    # backward: information, the masks (bf16), delta and lse*log2(e) padded to
+    # 128-row blocks, and for bf16 four f16 operand copies
+    want = 512 + rows + 2 * B * H * N * 4 + 4 * B * H * N * D * 2
     assert lib.swa_attn_bwd_workspace_size(B, H, N, D, swa.SWA_BF16) == want
     assert lib.swa_attn_grad_workspace_size(B, H, N, D, swa.SWA_BF16) == want
     assert lib.swa_attn_bwd_workspace_size(1, 1, 256, 64, swa.SWA_F32) == 256 + 2 * 1024
