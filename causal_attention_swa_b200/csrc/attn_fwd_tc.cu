@@ -9,25 +9,24 @@
 // (scores = q.k/8 over the pairs with q.t >= k.t, w = exp(s - row max),
 // out = sum w/z v).
 //
-// Block = two 128-row query tiles of one head (256 rows) and 640 threads:
-//   warps 0-7   softmax for query tile 0, warps 8-15 for query tile 1; in
-//               each group, warps 4h + w (w = 0..3) take TMEM lanes
-//               32w..32w+31 (rows) and score columns 64h..64h+63, so a row
-//               is shared by two threads that agree on its max each tile
-//   warp  16    TMA producer: Q0, Q1 once, then K_j, V_j into 4 stages
-//   warp  17    MMA issuer for query tile 0 (one elected lane), TMEM owner
-//   warp  18    MMA issuer for query tile 1
-//   warp  19    V cleaner (heads whose V holds an infinity or NaN): rewrites
+// Block = two 128-row query tiles of one head (256 rows) and 384 threads:
+//   warps 0-3   softmax for query tile 0, warps 4-7 for query tile 1; warp w
+//               takes TMEM lanes 32(w%4)..+31, one row per thread, all 128
+//               score columns of the key tile
+//   warp  8     TMA producer: Q0, Q1 once, then K_j, V_j into 4 stages
+//   warp  9     MMA issuer for query tile 0 (one elected lane), TMEM owner
+//   warp  10    MMA issuer for query tile 1
+//   warp  11    V cleaner (heads whose V holds an infinity or NaN): rewrites
 //               each staged V tile in place (a non-finite entry -> 0, its row
 //               recorded), then releases it to the issuers; it also gives its
 //               registers to the softmax warps of its scheduler
 // Each query tile has an issuer of its own, so neither tile's MMAs queue
 // behind the other tile's barriers; each issuer releases a K/V stage on a
 // barrier of its own and the producer waits for the issuers that read it.
-// Registers: launched at 96 per thread (640 x 96); the softmax warps take
-// 112 and warps 16-19 give up to 32, one of them on each scheduler (the
+// Registers: launched at 168 per thread (384 x 168); the softmax warps take
+// 232 and warps 8-11 give up to 40, one of them on each scheduler (the
 // registers of a warp stay in its scheduler's file).  The launcher checks
-// that the kernel was built with exactly 96: a larger claim than the
+// that the kernel was built with exactly 168: a larger claim than the
 // scheduler holds would stall setmaxnreg.inc.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384)
 // O0 [384,448) O1 [448,512).  P_t (16-bit, two per column) has columns of
@@ -44,9 +43,10 @@
 // roles take no issue slots from the softmax warps that share a scheduler.
 // At D = 64 the exponentials bound the kernel: a score costs one MUFU ex2
 // (16 per clock per SM) and 4 * 64 MMA flops (about 8000 per clock per SM),
-// so ex2 time is about twice the MMA time.  A single warp cannot keep its
-// scheduler's MUFU busy (the FMA -> ex2 -> convert chains are too short),
-// so every scheduler runs four softmax warps.
+// so ex2 time is about twice the MMA time.  A warp whose ex2 loop runs over
+// 128 independent scores keeps its scheduler's MUFU ~88% busy alone (~99%
+// with the second softmax warp), so one thread per row suffices; it also
+// needs no exchange of partial row maxima between threads.
 // Online softmax in the log2 domain with a lazy rescale: the reference max
 // of a row moves (and O, l are rescaled) only when the new row max exceeds
 // it by more than 8, so P <= 2^8 (exact after the final division by l).
@@ -56,9 +56,10 @@
 // exactly, up to f16's subnormal spacing of 2^-24); a head with larger
 // values keeps both in bf16 (V as given).  A bf16 P (7 fraction bits) is
 // exact enough for the output itself, but the output is what the gradient
-// of loss = 1/2 sum out^2 feeds back as dout, and the rounding of few-key rows (early rows) reaches the
-// gradient amplified by the cancellation in sum_j dS_ij k_j; with the f16 P
-// the end-to-end gradient stays inside the bf16 path's tolerance.  Rows
+// of loss = 1/2 sum out^2 feeds back as dout, and the rounding of few-key
+// rows (early rows) reaches the gradient amplified by the cancellation in
+// sum_j dS_ij k_j; with the f16 P the end-to-end gradient stays inside the
+// bf16 path's tolerance.  Rows
 // that see few keys (the first rows of a causal head) average no rounding
 // away, so on the diagonal tile -- the last key tile of every causal query
 // tile -- P also enters as the sum of two 16-bit words: its rounding
@@ -102,30 +103,25 @@ constexpr int BN = 128;                 // keys per K/V tile
 constexpr int HD = 64;                  // head dimension
 constexpr int kStages = 4;              // K/V pipeline depth
 constexpr int kTileBytes = BM * HD * 2; // 16 KB per bf16 tile
-constexpr int kSoftmaxWarps = 16;
-constexpr int kThreads = (kSoftmaxWarps + 4) * 32;  // 640: five warps per scheduler
-// 16384 registers per scheduler / (5 warps * 32 threads), rounded down to 8
-constexpr int kLaunchRegs = 96;
-// The softmax warps hold 64 scores per thread plus the loop's state; at 104
-// registers their loop reloaded spilled values every tile (and how many
-// depended on the code around it).  The other warps (TMA, MMA issue, the V
-// cleaner) fit in 32.
-constexpr int kSoftmaxRegs = 112;
-constexpr int kOtherRegs = 32;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kThreads = (kSoftmaxWarps + 4) * 32;  // 384: three warps per scheduler
+// 16384 registers per scheduler / (3 warps * 32 threads), rounded down to 8
+constexpr int kLaunchRegs = 168;
+// A softmax thread holds its row's 128 scores plus the loop's state.  The
+// other warps (TMA, MMA issue, the V cleaner) fit in 40.
+constexpr int kSoftmaxRegs = 232;
+constexpr int kOtherRegs = 40;
 // Warp w runs on scheduler w % 4 and setmaxnreg moves registers only
-// between the warps of one scheduler: each scheduler holds four softmax
-// warps and one of warps 16-19, which gives up what the four take.
-static_assert(4 * kSoftmaxRegs + kOtherRegs <= 5 * kLaunchRegs, "register split per scheduler");
+// between the warps of one scheduler: each scheduler holds two softmax
+// warps (one per query tile) and one of warps 8-11, which gives up what the
+// two take.
+static_assert(2 * kSoftmaxRegs + kOtherRegs <= 3 * kLaunchRegs, "register split per scheduler");
 constexpr int kTmaWarp = kSoftmaxWarps;
 constexpr int kMmaWarp = kSoftmaxWarps + 1;  // issuer of tile 0; kMmaWarp + 1 issues tile 1
-constexpr int kHalf = BN / 2;                // score columns per softmax thread
 constexpr uint32_t kTmemCols = 512;
 constexpr int kHeadGroup = 4;                // heads scheduled together (K, V share L2)
 constexpr float kRescaleThreshold = 8.0f;
-// A P computed against a stale reference max must still fit the operand
-// type before it is moved to the new max: < 2^15 in f16, < 2^64 in bf16.
-template <bool kF16> constexpr float kFastRange = kF16 ? 15.0f : 64.0f;
-constexpr int kCleanWarp = kSoftmaxWarps + 3;  // warp 19
+constexpr int kCleanWarp = kSoftmaxWarps + 3;  // warp 11
 // Per-head information (kHeadInfoInts int32 per head): bit 0 of [0] is set if
 // V holds an infinity or NaN, [1] is the largest biased exponent of its
 // finite values.  f16 operands are used when that exponent is below 2^15's.
@@ -147,8 +143,6 @@ struct __align__(1024) Smem {
   uint64_t v_ready[kStages];    // the cleaner has rewritten the stage's V tile
   uint64_t cls_done;            // the cleaner has recorded every tile's classes
   int first_cls[3][HD];         // per column: first key row with +inf, -inf, NaN
-  uint64_t pair[2][4];          // the two threads of a row: tile t, lanes 32w..
-  float part[2][2][2][BM];      // [tile][parity][half][row]: partial row max / sum
   uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
@@ -277,7 +271,6 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(&sm.s_free[t], kSoftmaxWarps / 2);  // one arrival per softmax warp of tile t
       mbar_init(&sm.p_full[t], kSoftmaxWarps / 2);
       mbar_init(&sm.pv_done[t], 1);
-      for (int w = 0; w < 4; ++w) mbar_init(&sm.pair[t][w], 2);  // the row's two warps
     }
     mbar_init(&sm.drain[0], 1);
     mbar_init(&sm.drain[1], 1);
@@ -345,7 +338,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         mma_ts_run8<128, 8, 16, 24, 32, 40, 48, 56>(tmem + col_o(t), tmem + col_p(t), v_desc,
                                                     idesc_o, j > 0 ? 1u : 0u);
         if (causal && j == n_t[t] - 1)  // the diagonal tile: + P's residual (in S's columns)
-          mma_ts_run8<128, 8, 16, 24, 64, 72, 80, 88>(tmem + col_o(t), tmem + col_s(t), v_desc,
+          mma_ts_run8<128, 8, 16, 24, 32, 40, 48, 56>(tmem + col_o(t), tmem + col_s(t), v_desc,
                                                       idesc_o, 1u);
         mma_commit_elect(&sm.pv_done[t]);
         mma_commit_elect(&sm.kv_empty[t][j % kStages]);
@@ -402,47 +395,34 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   } else if (warp < kSoftmaxWarps) {
     // ------------------------------------------------------------ softmax
     regs_increase<kSoftmaxRegs>();
-    const int t = warp >> 3;        // query tile
-    const int h = (warp >> 2) & 1;  // score columns 64h..64h+63
-    const int wt = warp & 3;        // TMEM lanes 32wt..32wt+31
+    const int t = warp >> 2;   // query tile
+    const int wt = warp & 3;   // TMEM lanes 32wt..32wt+31 (the warp's subpartition)
     const int r = wt * 32 + lane;
     const int g = 2 * c + t;
     const int row = g * BM + r;
     const uint32_t lane_off = static_cast<uint32_t>(wt * 32) << 16;
-    const uint32_t tS = tmem + lane_off + col_s(t) + kHalf * h;
-    const uint32_t tP = tmem + lane_off + col_p(t) + (kHalf / 2) * h;
-    const uint32_t tO = tmem + lane_off + col_o(t) + (HD / 2) * h;
-    uint64_t* pair = &sm.pair[t][wt];
-    int pair_phase = 0;
-    // publish v for the row, wait for the partner thread's value
-    auto exchange = [&](float v, float& other) -> bool {
-      const int slot = pair_phase & 1;
-      sm.part[t][slot][h][r] = v;
-      warp_arrive(pair);
-      if (!mbar_wait_parked(pair, pair_phase & 1, abort, err, kDevTimeoutOther)) return false;
-      other = sm.part[t][slot][h ^ 1][r];
-      ++pair_phase;
-      return true;
-    };
-    float m_used = -INFINITY;  // reference max (log2 domain), the same in both
-                               // threads of the row
-    float l = 0.f;             // this thread's share of the row sum
+    const uint32_t tS = tmem + lane_off + col_s(t);
+    const uint32_t tP = tmem + lane_off + col_p(t);
+    const uint32_t tO = tmem + lane_off + col_o(t);
+    float m_used = -INFINITY;  // reference max of the row (log2 domain)
+    float l = 0.f;             // row sum against m_used
     bool ok = true;
     bool s_ready = false;  // S_t,j already seen complete by the probe of tile j-1
+    const float2 sc2 = make_float2(scale_log2, scale_log2);
     for (int j = 0; j < n_t[t]; ++j) {
       if (!s_ready && !mbar_wait_parked(&sm.s_full[t], j & 1, abort, err, kDevTimeoutMma)) {
         ok = false;
         break;
       }
       fence_after_sync();
-      float x[kHalf];
+      float x[BN];
       {
-        uint32_t u[kHalf / 16][16];
+        uint32_t u[BN / 16][16];
 #pragma unroll
-        for (int i = 0; i < kHalf / 16; ++i) tmem_ld16(tS + i * 16, u[i]);
+        for (int i = 0; i < BN / 16; ++i) tmem_ld16(tS + i * 16, u[i]);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < kHalf / 16; ++i)
+        for (int i = 0; i < BN / 16; ++i)
 #pragma unroll
           for (int e = 0; e < 16; ++e) x[i * 16 + e] = __uint_as_float(u[i][e]);
       }
@@ -451,88 +431,42 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       const bool need_mask = (j * BN + BN > N) || (causal && j == g);
       if (need_mask) {
 #pragma unroll
-        for (int e = 0; e < kHalf; ++e) {
-          const int key = j * BN + kHalf * h + e;
+        for (int e = 0; e < BN; ++e) {
+          const int key = j * BN + e;
           if (key >= N || (causal && key > row)) x[e] = -INFINITY;
         }
       }
-      // 8 chains of three-input maxima over this thread's 64 scores
-      float mxp[8];
+      // 16 chains of three-input maxima over the row's 128 scores
+      float mxp[16];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) mxp[a] = fmax3(x[a], x[a + 8], x[a + 16]);
+      for (int a = 0; a < 16; ++a) mxp[a] = fmax3(x[a], x[a + 16], x[a + 32]);
 #pragma unroll
-      for (int a = 0; a < 8; ++a) mxp[a] = fmax3(mxp[a], x[a + 24], x[a + 32]);
+      for (int a = 0; a < 16; ++a) mxp[a] = fmax3(mxp[a], x[a + 48], x[a + 64]);
 #pragma unroll
-      for (int a = 0; a < 8; ++a) mxp[a] = fmax3(mxp[a], x[a + 40], x[a + 48]);
+      for (int a = 0; a < 16; ++a) mxp[a] = fmax3(mxp[a], x[a + 80], x[a + 96]);
 #pragma unroll
-      for (int a = 0; a < 8; ++a) mxp[a] = fmaxf(mxp[a], x[a + 56]);
-      const float mine = fmaxf(fmax3(mxp[0], mxp[1], mxp[2]),
-                               fmax3(fmax3(mxp[3], mxp[4], mxp[5]), mxp[6], mxp[7]));
-      // Publish this thread's max now, read the partner's when it is needed:
-      // before the ex2 loop only if a score of this thread could lie far
-      // above m_used (the first tile, a jump of more than kFastRange, a
-      // NaN); else after it, when the partner has long published.  Both
-      // threads derive the same m_new from (m_used, both maxima); a P
-      // computed against m_used is then moved to m_new (rare: the partner
-      // raised the max by more than the lazy threshold) by one rounding.
-      const float mine_l2 = mine * scale_log2;  // scale_log2 > 0 commutes with the max
-      const int slot = pair_phase & 1;
-      const uint32_t par = static_cast<uint32_t>(pair_phase & 1);
-      ++pair_phase;
-      sm.part[t][slot][h][r] = mine_l2;
-      warp_arrive(pair);
-      float m_new = m_used;
-      bool pair_seen = false;  // set by an earlier successful probe
-      auto fetch_and_decide = [&]() -> bool {
-        if (!pair_seen && !mbar_wait_parked(pair, par, abort, err, kDevTimeoutOther))
-          return false;
-        const float theirs = sm.part[t][slot][h ^ 1][r];
-        // the same operand order in both threads of the row
-        const float cand = h == 0 ? fmaxf(mine_l2, theirs) : fmaxf(theirs, mine_l2);
-        const float mc = fmaxf(m_used, cand);
-        if (j == 0 || mc > m_used + kRescaleThreshold) m_new = mc;
-        return true;
-      };
-      // the diagonal tile (last of a causal query tile) recomputes P below
-      // for its residual, against the final reference max: fetch it first
-      const bool diag_lo = causal && j == n_t[t] - 1;
-      const bool early = diag_lo ||
-          __any_sync(0xffffffffu, j == 0 || !(mine_l2 <= m_used + kFastRange<kF16>));
-      if (early && !fetch_and_decide()) { ok = false; break; }
-      const float m_exp = m_new;  // the reference the ex2 loop uses
-      // O_t += P_t,j-1 V_j-1 (issued at the end of the last tile) is probed
-      // now and waited for, if still needed, only after the ex2 loop
+      for (int a = 0; a < 16; ++a) mxp[a] = fmaxf(mxp[a], x[a + 112]);
+#pragma unroll
+      for (int a = 0; a < 5; ++a) mxp[a] = fmax3(mxp[3 * a], mxp[3 * a + 1], mxp[3 * a + 2]);
+      const float mine = fmax3(fmax3(mxp[0], mxp[1], mxp[2]), fmaxf(mxp[3], mxp[4]), mxp[15]);
+      // Lazy rescale: the reference moves only when the row max exceeds it
+      // by more than kRescaleThreshold (always on the first tile), so every
+      // P = 2^(s - m_used) <= 2^8.
+      const float mc = fmaxf(m_used, mine * scale_log2);  // scale_log2 > 0 commutes with max
+      const float m_new = (j == 0 || mc > m_used + kRescaleThreshold) ? mc : m_used;
+      // O_t += P_t,j-1 V_j-1 (issued at the end of the last tile) reads P_t:
+      // probed now, waited for (if still needed) after the ex2 loop
       const bool pv_ready = j == 0 || mbar_test_wait(&sm.pv_done[t], (j - 1) & 1);
+      const float2 nm2 = make_float2(-m_new, -m_new);
       float2 rsp[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      const float2 sc2 = make_float2(scale_log2, scale_log2);
-      const float2 nm2 = make_float2(-m_exp, -m_exp);
-      uint32_t pk[kHalf / 32][16];
-      auto exps = [&](int i) {
+      uint32_t pk[BN / 32][16];
 #pragma unroll
-        for (int e = 16 * i; e < 16 * i + 16; ++e) {
-          const float2 a = __ffma2_rn(make_float2(x[2 * e], x[2 * e + 1]), sc2, nm2);
-          const float2 pe = make_float2(ex2(a.x), ex2(a.y));
-          rsp[e & 1] = __fadd2_rn(rsp[e & 1], pe);
-          pk[i][e & 15] = pack_p<kF16>(pe.x, pe.y);
-        }
-      };
-      exps(0);
-      // the partner published with this thread: probe between the halves
-      if (!early) pair_seen = mbar_test_wait(pair, par);
-      exps(1);
-      if (!early && !fetch_and_decide()) { ok = false; break; }
-      if (__any_sync(0xffffffffu, m_exp != m_new)) {  // rare: the partner moved the max
-        const float beta = ex2(m_exp - m_new);
-#pragma unroll
-        for (int i = 0; i < kHalf / 32; ++i)
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[i][e] = pack_p<kF16>(unpack_lo<kF16>(pk[i][e]) * beta,
-                                    unpack_hi<kF16>(pk[i][e]) * beta);
-        rsp[0].x *= beta; rsp[0].y *= beta; rsp[1].x *= beta; rsp[1].y *= beta;
+      for (int e = 0; e < BN / 2; ++e) {
+        const float2 a = __ffma2_rn(make_float2(x[2 * e], x[2 * e + 1]), sc2, nm2);
+        const float2 pe = make_float2(ex2(a.x), ex2(a.y));
+        rsp[e & 1] = __fadd2_rn(rsp[e & 1], pe);
+        pk[e >> 4][e & 15] = pack_p<kF16>(pe.x, pe.y);
       }
-      // O_t += P_t,j-1 V_j-1 must finish before O_t is rescaled or P_t is
-      // overwritten: by now it normally has.
       if (j > 0) {
         if (!pv_ready &&
             !mbar_wait_parked(&sm.pv_done[t], (j - 1) & 1, abort, err, kDevTimeoutMma)) {
@@ -540,10 +474,11 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           break;
         }
         fence_after_sync();
+        // O_t is complete: move it to the new reference (rare)
         if (__any_sync(0xffffffffu, m_new != m_used)) {
-          const float alpha = ex2(m_used - m_new);
-#pragma unroll
-          for (int i = 0; i < HD / 32; ++i) {
+          const float alpha = ex2(m_used - m_new);  // 1 in rows whose reference stays
+#pragma unroll 1
+          for (int i = 0; i < HD / 16; ++i) {
             uint32_t u[16];
             tmem_ld16(tO + i * 16, u);
             tmem_wait_ld();
@@ -556,12 +491,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       m_used = m_new;
 #pragma unroll
-      for (int i = 0; i < kHalf / 32; ++i) tmem_st16(tP + i * 16, pk[i]);
-      if (diag_lo) {
-        // P's rounding residual P - hi(P), 16 keys per 8 columns, over this
-        // thread's own S columns (each chunk is read before it is written)
+      for (int i = 0; i < BN / 32; ++i) tmem_st16(tP + i * 16, pk[i]);
+      if (causal && j == n_t[t] - 1) {
+        // the diagonal tile: P's rounding residual P - hi(P), 16 keys per 8
+        // columns, over the row's own S columns (each chunk is read before
+        // it is written); a second P V product adds it
 #pragma unroll 1
-        for (int cidx = 0; cidx < kHalf / 16; ++cidx) {
+        for (int cidx = 0; cidx < BN / 16; ++cidx) {
           uint32_t u[16];
           tmem_ld16(tS + 16 * cidx, u);
           tmem_wait_ld();
@@ -569,7 +505,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
           for (int e2 = 0; e2 < 8; ++e2) {
             float2 sv = make_float2(__uint_as_float(u[2 * e2]), __uint_as_float(u[2 * e2 + 1]));
-            const int key = j * BN + kHalf * h + 16 * cidx + 2 * e2;
+            const int key = j * BN + 16 * cidx + 2 * e2;
             if (key >= N || key > row) sv.x = -INFINITY;
             if (key + 1 >= N || key + 1 > row) sv.y = -INFINITY;
             const float2 a = __ffma2_rn(sv, sc2, nm2);
@@ -587,15 +523,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       warp_arrive(&sm.p_full[t]);
       l += (rsp[0].x + rsp[0].y) + (rsp[1].x + rsp[1].y);
     }
-    float l_other = 0.f;
-    if (ok && n_t[t] > 0 && exchange(l, l_other) &&
+    if (ok && n_t[t] > 0 &&
         mbar_wait_parked(&sm.pv_done[t], (n_t[t] - 1) & 1, abort, err, kDevTimeoutMma)) {
       fence_after_sync();
-      const float l_row = h == 0 ? l + l_other : l_other + l;
-      const float inv = 1.f / l_row;
-      float o[HD / 2];  // this thread's 32 columns of out_row, float32
+      const float inv = 1.f / l;
+      float o[HD];  // out_row, float32
 #pragma unroll
-      for (int i = 0; i < HD / 32; ++i) {
+      for (int i = 0; i < HD / 16; ++i) {
         uint32_t u[16];
         tmem_ld16(tO + i * 16, u);
         tmem_wait_ld();
@@ -606,45 +540,42 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         // IEEE class of sum_{j in J(row)} P_ij v_jd with every P_ij > 0
         const int last = causal ? row : N - 1;
 #pragma unroll
-        for (int e = 0; e < HD / 2; ++e) {
-          const int d = (HD / 2) * h + e;
+        for (int d = 0; d < HD; ++d) {
           const bool pinf = sm.first_cls[0][d] <= last, ninf = sm.first_cls[1][d] <= last;
           const bool nan = sm.first_cls[2][d] <= last || (pinf && ninf);
-          if (nan) o[e] = __uint_as_float(0x7FC00000u);
-          else if (pinf) o[e] = INFINITY;
-          else if (ninf) o[e] = -INFINITY;
+          if (nan) o[d] = __uint_as_float(0x7FC00000u);
+          else if (pinf) o[d] = INFINITY;
+          else if (ninf) o[d] = -INFINITY;
         }
       }
-      const float lse2 = m_used + __log2f(l_row);  // lse * log2 e
+      const float lse2 = m_used + __log2f(l);  // lse * log2 e
       if (row < N) {
-        uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)head * N + row) * HD + (HD / 2) * h);
+        uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)head * N + row) * HD);
 #pragma unroll
-        for (int i = 0; i < HD / 16; ++i)
+        for (int i = 0; i < HD / 8; ++i)
           dst[i] = make_uint4(pack_bf16(o[8 * i], o[8 * i + 1]), pack_bf16(o[8 * i + 2], o[8 * i + 3]),
                               pack_bf16(o[8 * i + 4], o[8 * i + 5]),
                               pack_bf16(o[8 * i + 6], o[8 * i + 7]));
-        if (h == 0) lse[(size_t)head * N + row] = lse2 * kLn2;
+        lse[(size_t)head * N + row] = lse2 * kLn2;
       }
       if (do16 != nullptr) {
         // what the backward of loss = 1/2 sum out^2 reads: dout = out as f16,
         // delta = sum_d out_d^2, -lse log2 e (rows past N: 0 and -inf)
         float sq = 0.f;
 #pragma unroll
-        for (int e = 0; e < HD / 2; ++e) sq = fmaf(o[e], o[e], sq);
-        float sq_other = 0.f;
-        const bool got = exchange(sq, sq_other);
+        for (int d = 0; d < HD; ++d) sq = fmaf(o[d], o[d], sq);
         const int64_t Npad = pad128(N);
         if (row < N) {
-          uint4* dst = reinterpret_cast<uint4*>(do16 + ((size_t)head * N + row) * HD + (HD / 2) * h);
+          uint4* dst = reinterpret_cast<uint4*>(do16 + ((size_t)head * N + row) * HD);
 #pragma unroll
-          for (int i = 0; i < HD / 16; ++i)
+          for (int i = 0; i < HD / 8; ++i)
             dst[i] = make_uint4(pack_f16(o[8 * i], o[8 * i + 1]), pack_f16(o[8 * i + 2], o[8 * i + 3]),
                                 pack_f16(o[8 * i + 4], o[8 * i + 5]),
                                 pack_f16(o[8 * i + 6], o[8 * i + 7]));
         }
-        if (got && h == 0 && row < Npad) {
+        if (row < Npad) {
           const bool real = row < N;
-          delta[(size_t)head * Npad + row] = real ? sq + sq_other : 0.f;
+          delta[(size_t)head * Npad + row] = real ? sq : 0.f;
           nlse2[(size_t)head * Npad + row] = real ? -lse2 : -INFINITY;
         }
       }
