@@ -180,6 +180,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const float* __restrict__ delta, __nv_bfloat16* __restrict__ dk,
                      __nv_bfloat16* __restrict__ dv, int N, int BH, int causal, float scale,
                      float scale_log2, const int* __restrict__ info, unsigned* __restrict__ err) {
+  pdl_prologue();  // the next launch (independent outputs) overlaps this one's tail
   const int n_blocks = (N + BQ - 1) / BQ;
   const int Npad = n_blocks * BQ;
   int head, jb;
@@ -515,6 +516,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
                    const float* __restrict__ delta, __nv_bfloat16* __restrict__ dq, int N, int BH,
                    int causal, float scale, float scale_log2, const int* __restrict__ info,
                    unsigned* __restrict__ err) {
+  pdl_prologue();  // the next launch (independent outputs) overlaps this one's tail
   const int n_blocks = (N + BQ - 1) / BQ;
   const int Npad = n_blocks * BQ;
   int head, ib;
@@ -777,7 +779,8 @@ template <bool kF16>
 cudaError_t launch_bwd_instance(const void* q, const void* k, const void* v, const void* dout,
                                 const float* nlse2, const float* delta, void* dq, void* dk,
                                 void* dv, int64_t BH, int64_t N, int causal, float scale,
-                                const int* info, unsigned* err, cudaStream_t s, int* launches) {
+                                const int* info, unsigned* err, cudaStream_t s, bool after,
+                                int* launches) {
   CUtensorMap tq, tk, tv, tdo;
   cudaError_t e;
   if ((e = make_tmap_bf16_rows(&tq, q, BH, N, BQ)) != cudaSuccess) return e;
@@ -791,16 +794,22 @@ cudaError_t launch_bwd_instance(const void* q, const void* k, const void* v, con
                            (int)kSmemQ);
   if (e != cudaSuccess) return e;
   const int64_t n_blocks = (N + BK - 1) / BK;
-  attn_bwd_dkdv_kernel<kF16><<<(unsigned)(n_blocks * BH), kThreads, kSmemKV, s>>>(
-      tq, tk, tv, tdo, nlse2, delta, static_cast<__nv_bfloat16*>(dk),
-      static_cast<__nv_bfloat16*>(dv), (int)N, (int)BH, causal, scale, scale * kLog2e, info,
-      err);
+  // dkdv, dq and the other instance's pair write disjoint outputs and read
+  // only what was complete before the first of them: each after the first
+  // may start in the tail of the one before
+  const dim3 grid((unsigned)(n_blocks * BH));
+  e = launch_after(after, attn_bwd_dkdv_kernel<kF16>, grid, dim3(kThreads), kSmemKV, s, tq, tk,
+                   tv, tdo, nlse2, delta, static_cast<__nv_bfloat16*>(dk),
+                   static_cast<__nv_bfloat16*>(dv), (int)N, (int)BH, causal, scale,
+                   scale * kLog2e, info, err);
+  if (e != cudaSuccess) return e;
   *launches += 1;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  attn_bwd_dq_kernel<kF16><<<(unsigned)(n_blocks * BH), kThreads, kSmemQ, s>>>(
-      tk, tv, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(dout), nlse2, delta,
-      static_cast<__nv_bfloat16*>(dq), (int)N, (int)BH, causal, scale, scale * kLog2e, info,
-      err);
+  e = launch_after(true, attn_bwd_dq_kernel<kF16>, grid, dim3(kThreads), kSmemQ, s, tk, tv,
+                   static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(dout), nlse2,
+                   delta, static_cast<__nv_bfloat16*>(dq), (int)N, (int)BH, causal, scale,
+                   scale * kLog2e, info, err);
+  if (e != cudaSuccess) return e;
   *launches += 1;
   return cudaGetLastError();
 }
@@ -814,10 +823,11 @@ cudaError_t launch_attn_bwd_tc(const BwdOperands& f16, const BwdOperands& bf16,
                                int* launches) {
   const int64_t BH = B * H;
   cudaError_t e = launch_bwd_instance<true>(f16.q, f16.k, f16.v, f16.dout, nlse2, delta, dq, dk,
-                                            dv, BH, N, causal, scale, info, err, s, launches);
+                                            dv, BH, N, causal, scale, info, err, s, false,
+                                            launches);
   if (e != cudaSuccess) return e;
   return launch_bwd_instance<false>(bf16.q, bf16.k, bf16.v, bf16.dout, nlse2, delta, dq, dk, dv,
-                                    BH, N, causal, scale, info, err, s, launches);
+                                    BH, N, causal, scale, info, err, s, true, launches);
 }
 
 }  // namespace swa

@@ -227,6 +227,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const uint4* __restrict__ vrows, int all_bf16,
                    uint16_t* __restrict__ do16, float* __restrict__ delta,
                    float* __restrict__ nlse2, unsigned* __restrict__ err) {
+  pdl_prologue();  // the other instance's launch overlaps this one's tail
   // Heads in groups of kHeadGroup, whose K and V (4 MB per head at N = 16384)
   // stay in L2 while the group's blocks run; inside a group the heaviest
   // (latest) query tiles first, heads interleaved.
@@ -628,7 +629,7 @@ cudaError_t launch_fwd_instance(const CUtensorMap& tq, const CUtensorMap& tk,
                                 const CUtensorMap& tv, void* out, float* lse, int64_t BH,
                                 int64_t N, int causal, float scale, const int* vinfo,
                                 const unsigned* vrows, int all_bf16, const FwdSaved& saved,
-                                unsigned* err, cudaStream_t s) {
+                                unsigned* err, cudaStream_t s, bool after) {
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<kF16>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
@@ -639,11 +640,12 @@ cudaError_t launch_fwd_instance(const CUtensorMap& tq, const CUtensorMap& tk,
   if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;  // register split unsafe
   const int n_ctiles = (int)((N + 2 * BM - 1) / (2 * BM));
   const int64_t grid = (int64_t)n_ctiles * BH;
-  attn_fwd_tc_kernel<kF16><<<(unsigned)grid, kThreads, kSmemBytes, s>>>(
-      tq, tk, tv, static_cast<__nv_bfloat16*>(out), lse, (int)N, (int)BH, n_ctiles, causal,
-      scale * kLog2e, vinfo, reinterpret_cast<const uint4*>(vrows), all_bf16,
-      static_cast<uint16_t*>(saved.do16), saved.delta,
-      saved.nlse2, err);
+  e = launch_after(after, attn_fwd_tc_kernel<kF16>, dim3((unsigned)grid), dim3(kThreads),
+                   kSmemBytes, s, tq, tk, tv, static_cast<__nv_bfloat16*>(out), lse, (int)N,
+                   (int)BH, n_ctiles, causal, scale * kLog2e, vinfo,
+                   reinterpret_cast<const uint4*>(vrows), all_bf16,
+                   static_cast<uint16_t*>(saved.do16), saved.delta, saved.nlse2, err);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -664,12 +666,14 @@ cudaError_t launch_attn_fwd_tc(const void* q, const void* k, const void* v, cons
     // those heads exit at once, and the other way round
     if ((e = make_tmap_bf16_rows(&tv16, v16, BH, N, BN)) != cudaSuccess) return e;
     if ((e = launch_fwd_instance<true>(tq, tk, tv16, out, lse, BH, N, causal, scale, vinfo,
-                                       vrows, 0, saved, err, s)) != cudaSuccess)
+                                       vrows, 0, saved, err, s, false)) != cudaSuccess)
       return e;
     *launches += 1;
   }
+  // behind the f16 instance (disjoint heads, no data between them) it may
+  // start in that launch's tail; alone it follows the prep pass as usual
   if ((e = launch_fwd_instance<false>(tq, tk, tv, out, lse, BH, N, causal, scale, vinfo,
-                                      vrows, all_bf16, saved, err, s)) != cudaSuccess)
+                                      vrows, all_bf16, saved, err, s, !all_bf16)) != cudaSuccess)
     return e;
   *launches += 1;
   return cudaSuccess;

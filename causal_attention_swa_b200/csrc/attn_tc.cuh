@@ -5,9 +5,31 @@
 
 #include <cuda.h>
 
+#include <utility>
+
 #include "swa_internal.cuh"
 
 namespace swa {
+
+// Launches `kernel` on stream s, with programmatic stream serialisation when
+// `after` is set: it may start once every block of the previous grid has
+// begun (the kernels call pdl_prologue()), instead of after that grid ends.
+// Only for a grid that reads nothing the previous grid writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_after(bool after, void (*kernel)(KArgs...), dim3 grid, dim3 block,
+                         size_t smem, cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = after ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // [BH][N][64] of a 16-bit type (bf16 or f16: the copy does not convert) as
 // a 3-D TMA tensor map (64, N, BH) with 64 x box_rows x 1 boxes and 128-byte

@@ -349,6 +349,32 @@ __device__ __forceinline__ void regs_decrease() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
 }
 
+// ---------------------------------------------- programmatic dependent launch
+
+// A grid launched with programmatic stream serialisation (launch_after) may
+// start while the grid before it still runs, once every block of that grid
+// has executed pdl_allow_next() or exited.
+__device__ __forceinline__ void pdl_allow_next() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Waits until the grid this one was launched behind has completed and its
+// memory operations are visible; returns at once in a grid launched without
+// programmatic serialisation.
+__device__ __forceinline__ void pdl_wait_prior() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Kernel prologue of a grid that may run behind (or ahead of) a
+// programmatically serialised neighbour: let the next grid start, and keep
+// this grid's completion behind the previous grid's -- its last block waits
+// for it -- so that a later ordinary launch still follows both.
+__device__ __forceinline__ void pdl_prologue() {
+  pdl_allow_next();
+  if (blockIdx.x == gridDim.x - 1 && blockIdx.y == gridDim.y - 1 && blockIdx.z == gridDim.z - 1)
+    pdl_wait_prior();
+}
+
 // ---------------------------------------------------------------- descriptors
 
 // Shared-memory matrix descriptor, 128-byte swizzle (TMA SWIZZLE_128B
