@@ -493,6 +493,30 @@ swa_status swa_qkv_proj(const void* x, const void* w, void* q, void* k, void* v,
   return SWA_OK;
 }
 
+swa_status swa_attn_merge(const void* out_part, const float* lse_part, float* out_acc,
+                          float* lse_acc, void* out_final, int64_t rows, int64_t D, int first,
+                          swa_dtype dt, void* stream) {
+  t_msg[0] = 0;
+  t_launches = 0;
+  if (dt != SWA_BF16 && dt != SWA_F32) return fail(SWA_ERR_INVALID_ARGUMENT, "unknown dtype");
+  if (D != 64) return fail(SWA_ERR_UNSUPPORTED, "D must be 64 (got %lld)", (long long)D);
+  if (rows < 1 || rows > ((int64_t)1 << 31))
+    return fail(SWA_ERR_INVALID_ARGUMENT, "rows must be in [1, 2^31] (got %lld)",
+                (long long)rows);
+  if (!aligned16(out_part) || !aligned16(lse_part) || !aligned16(out_acc) ||
+      !aligned16(lse_acc) || (out_final != nullptr && !aligned16(out_final)))
+    return fail(SWA_ERR_INVALID_ARGUMENT,
+                "out_part, lse_part, out_acc, lse_acc must be non-null and 16-byte aligned "
+                "(out_final too, when given)");
+  int launches = 0;
+  cudaError_t e = swa::launch_attn_merge(dt, out_part, lse_part, out_acc, lse_acc, out_final,
+                                         rows, first ? 1 : 0, static_cast<cudaStream_t>(stream),
+                                         &launches);
+  if (e != cudaSuccess) return cuda_fail(e, "attn_merge");
+  t_launches = launches;
+  return SWA_OK;
+}
+
 swa_status swa_get_device_error(void* stream) {
   t_msg[0] = 0;
   swa_status st;

@@ -63,6 +63,14 @@ constexpr int kHeadInfoInts = 4;
 cudaError_t launch_scan_v_info(const void* v, int64_t heads, int64_t elems_per_head,
                                int* info, cudaStream_t s, int* launches);
 
+// Merge of a partial attention result over a disjoint key set into a
+// float32 accumulator (attn_merge.cu): out_part [rows][64] of dt, lse_part
+// [rows]; out_acc [rows][64] float32, lse_acc [rows] (in/out; ignored on
+// input when `first`); out_final (nullable) receives the merged rows in dt.
+cudaError_t launch_attn_merge(swa_dtype dt, const void* out_part, const float* lse_part,
+                              float* out_acc, float* lse_acc, void* out_final, int64_t rows,
+                              int first, cudaStream_t s, int* launches);
+
 // The prep pass over [BH][N][64] bf16 tensors: f16 copies of v (and of q and
 // k if q is non-null, of dout if non-null) into v16 (q16, k16, do16); with
 // `out` non-null (dout then too) delta = dout . out and nlse2 = -lse log2 e

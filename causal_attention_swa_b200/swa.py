@@ -29,6 +29,7 @@ EXPORTS = (
     "swa_profile_kernel", "swa_attn_fwd_noalloc", "swa_selftest_wait_timeout",
     "swa_attn_grad_workspace_size", "swa_attn_grad", "swa_nw_regrid_nd",
     "swa_nw_regrid_bwd_workspace_size", "swa_nw_regrid_bwd", "swa_qkv_proj",
+    "swa_attn_merge",
 )
 (SWA_KERNEL_NONE, SWA_KERNEL_ATTN_FWD, SWA_KERNEL_ATTN_BWD, SWA_KERNEL_NW, SWA_KERNEL_NW_BWD,
  SWA_KERNEL_QKV) = range(6)
@@ -84,6 +85,8 @@ def load_library():
     lib.swa_nw_regrid_bwd.restype = I
     lib.swa_qkv_proj.argtypes = [P, P, P, P, P, I64, I64, I64, I64, I64, I, P]
     lib.swa_qkv_proj.restype = I
+    lib.swa_attn_merge.argtypes = [P, P, P, P, P, I64, I64, I, I, P]
+    lib.swa_attn_merge.restype = I
     lib.swa_get_device_error.argtypes = [P]
     lib.swa_get_device_error.restype = I
     lib.swa_selftest_wait_timeout.argtypes = [P]
@@ -336,6 +339,29 @@ def qkv_proj(x, w, H: int, q=None, k=None, v=None):
                           _dtype_code(x), _stream_ptr(x.device))
     _check(st, "swa_qkv_proj")
     return q, k, v
+
+
+def attn_merge(out_part, lse_part, out_acc, lse_acc, first: bool, out_final=None):
+    """swa_attn_merge: merge a partial result (out_part [B,H,N,64] bf16 or
+    fp32, lse_part [B,H,N] fp32) over one key set into the float32
+    accumulator (out_acc [B,H,N,64], lse_acc [B,H,N]) over a disjoint set;
+    with out_final, also write the merged rows in out_part's dtype."""
+    if not isinstance(out_part, torch.Tensor) or out_part.dim() != 4:
+        raise ValueError("out_part must be a [B, H, N, D] tensor")
+    B, H, N, D = out_part.shape
+    named = {"lse_part": lse_part, "out_acc": out_acc, "lse_acc": lse_acc}
+    shapes = {"lse_part": ((B, H, N), torch.float32), "out_acc": ((B, H, N, D), torch.float32),
+              "lse_acc": ((B, H, N), torch.float32), "out_final": (out_part.shape, out_part.dtype)}
+    if out_final is not None:
+        named["out_final"] = out_final
+    _require_like(out_part, named, lambda n: shapes[n])
+    lib = load_library()
+    _require_cuda(out_part, *named.values())
+    st = lib.swa_attn_merge(_ptr(out_part), _ptr(lse_part), _ptr(out_acc), _ptr(lse_acc),
+                            _ptr(out_final), B * H * N, D, int(bool(first)),
+                            _dtype_code(out_part), _stream_ptr(out_part.device))
+    _check(st, "swa_attn_merge")
+    return out_acc, lse_acc
 
 
 def selftest_wait_timeout(device=None) -> None:

@@ -238,6 +238,28 @@ swa_status swa_qkv_proj(const void* x, const void* w, void* q, void* k, void* v,
                         void* stream);
 
 /*
+ * Merges a partial attention result over a set of keys into an accumulator
+ * over a disjoint set (sequence sharding: a rank's queries meet the other
+ * ranks' key blocks one at a time).  The view ATTENTION_WINDOW's average
+ * splits exactly ("Show HN ...", page 2): with lse = max + ln z of each set,
+ *   lse = ln(e^lse_acc + e^lse_part)
+ *   out = e^(lse_acc - lse) out_acc + e^(lse_part - lse) out_part
+ * (a set with lse = -inf contributes nothing).
+ *   out_part   [rows][D] of `dtype`    (in)   partial output (swa_attn_fwd's out)
+ *   lse_part   [rows] float32          (in)   its lse (natural log)
+ *   out_acc    [rows][D] float32       (in/out; input ignored when `first`)
+ *   lse_acc    [rows] float32          (in/out; input ignored when `first`)
+ *   out_final  [rows][D] of `dtype` or NULL   (out) the merged rows, rounded
+ * rows = B*H*N of the row-major [B,H,N,D] tensors; D == 64.  One kernel,
+ * asynchronous on `stream`; out_final may be out_part.
+ * Errors: SWA_ERR_INVALID_ARGUMENT (null or misaligned pointer, rows outside
+ * [1, 2^31], unknown dtype), SWA_ERR_UNSUPPORTED (D != 64).
+ */
+swa_status swa_attn_merge(const void* out_part, const float* lse_part, float* out_acc,
+                          float* lse_acc, void* out_final, int64_t rows, int64_t D, int first,
+                          swa_dtype dtype, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears this device's error word.
  * Returns SWA_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait since
  * the last call, SWA_ERR_CUDA if the synchronisation failed, else SWA_OK.

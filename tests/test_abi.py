@@ -137,6 +137,23 @@ def test_nw_nd_and_gradient_argument_errors(lib):
     assert 0 < lib.swa_nw_workspace_size(1, 1 << 31) <= (65535 * 8 + 255) // 256 * 256
 
 
+def test_merge_argument_errors(lib):
+    ok = (FAKE, FAKE, FAKE, FAKE, None, 128, 64, 1, swa.SWA_BF16, None)
+
+    def call(**kw):
+        names = ("op", "lp", "oa", "la", "of", "rows", "D", "first", "dt", "s")
+        args = dict(zip(names, ok))
+        args.update(kw)
+        return lib.swa_attn_merge(*(args[n] for n in names))
+    assert call(D=32) == swa.SWA_ERR_UNSUPPORTED
+    assert call(rows=0) == swa.SWA_ERR_INVALID_ARGUMENT
+    assert call(rows=(1 << 31) + 1) == swa.SWA_ERR_INVALID_ARGUMENT
+    assert call(op=None) == swa.SWA_ERR_INVALID_ARGUMENT
+    assert call(la=FAKE + 4) == swa.SWA_ERR_INVALID_ARGUMENT
+    assert call(of=FAKE + 8) == swa.SWA_ERR_INVALID_ARGUMENT
+    assert call(dt=7) == swa.SWA_ERR_INVALID_ARGUMENT
+
+
 def test_product_path_does_not_import_the_oracle():
     """The CUDA binding never reaches the oracle (no CPU fallback)."""
     pkg = os.path.join(ROOT, "causal_attention_swa_b200")
