@@ -432,6 +432,43 @@ def other_configs(swa, inputs, torch, stream, device, pk, info, cpu):
                                  "sample": f"512 of {N} tokens per sequence; {dt:.2f} s"}
     res["qkv_proj_b2n16384c1024"] = entry
     del x, w, qo, ko, vo
+
+    # ring forward: the compute of each rank of an 8-rank ring over one
+    # 131072-token sequence, rank after rank on this GPU (each with the K/V
+    # chunks its ring steps receive); the K/V transport is not in it
+    from causal_attention_swa_b200 import ring
+    wl = inputs.WORKLOADS["attn_ring_b1h8n131072"]
+    W = 8
+    qb, kb, vb, _ = inputs.attn_bf16(**wl)
+    q, k, v = dev16(qb), dev16(kb), dev16(vb)
+    chunks = [[ring.zigzag_split(t, r, W) for t in (q, k, v)] for r in range(W)]
+    kvs = [torch.stack((kc[0], kc[1], vc[0], vc[1])) for _, kc, vc in chunks]
+    del q, k, v
+    per_rank = []
+    for r in range(W):
+        state = ring.RingForwardState(chunks[r][0], r, W)
+
+        def run(state=state, r=r):
+            for s_ in range(W):
+                state.step(s_, kvs[(r - s_) % W])
+        per_rank.append(timed_call(run, stream, device, reps=3, warm=1))
+    fl, _ = attn_flops(wl["B"], wl["H"], wl["N"])
+    ms = max(per_rank)
+    entry = {"workload": "ring causal attention forward, 8 ranks, B=1 H=8 N=131072 D=64 bf16, "
+                         "Q, K ~ N(0, 0.5^2): the compute of each rank (16 zigzag chunks of "
+                         "8192 tokens; 17 chunk calls and merges per rank), ranks timed one "
+                         "after another on this GPU; K/V transport not included",
+             "ms_per_rank_max": ms, "ms_per_rank_min": min(per_rank),
+             "tflops_per_rank": fl / W / (ms * 1e-3) / 1e12,
+             "frac": fl / W / (ms * 1e-3) / 1e12 / peak, "bound": "tensor",
+             "timing": "median of 2 runs of each rank's steps after 1 warm-up, CUDA events"}
+    if cpu:
+        rate, dt = oracle_attn_rate(qb, kb, vb, [0], 8192, False, threads)
+        entry["cpu_baseline"] = {"value": rate, "unit": "TFLOP/s", "cores": threads,
+                                 "kind": "oracle",
+                                 "sample": f"head 0, first 8192 tokens, forward; {dt:.1f} s"}
+    res["ring_fwd_b1h8n131072_w8"] = entry
+    del chunks, kvs
     if swa.get_device_error(device) != swa.SWA_OK:
         raise RuntimeError("device error word set during the other workloads")
     return res

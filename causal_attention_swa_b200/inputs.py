@@ -187,6 +187,8 @@ WORKLOADS = {
     # across GPUs by sequences
     "attn_fwdbwd_b2h16n16384": dict(B=2, H=16, N=16384, seed=4),
     "attn_fwdbwd_b1h8n65536": dict(B=1, H=8, N=65536, seed=5, qk_std=0.5),
+    # a sequence for an 8-rank ring (16 zigzag chunks of 8192 tokens)
+    "attn_ring_b1h8n131072": dict(B=1, H=8, N=131072, seed=6, qk_std=0.5),
 }
 
 # 0.01% of V's 1*8*65536*64 entries, rounded: 3355 entries set to +inf.
