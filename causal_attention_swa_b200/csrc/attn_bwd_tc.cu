@@ -178,7 +178,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ nlse2,
                      const float* __restrict__ delta, __nv_bfloat16* __restrict__ dk,
-                     __nv_bfloat16* __restrict__ dv, int N, int BH, int causal, float scale,
+                     __nv_bfloat16* __restrict__ dv, float* __restrict__ dk_acc,
+                     float* __restrict__ dv_acc, int N, int BH, int causal, float scale,
                      float scale_log2, const int* __restrict__ info, unsigned* __restrict__ err) {
   pdl_prologue();  // the next launch (independent outputs) overlaps this one's tail
   const int n_blocks = (N + BQ - 1) / BQ;
@@ -455,7 +456,25 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
           else if (ninf) av[e] = 0xFF800000u;
         }
       }
-      if (jg < N) {
+      if (jg < N && dv_acc != nullptr) {
+        // accumulate mode: add this call's dv, dk (float32) to the caller's sums
+        float4* va = reinterpret_cast<float4*>(dv_acc + ((size_t)head * N + jg) * HD + 16 * w);
+        float4* ka = reinterpret_cast<float4*>(dk_acc + ((size_t)head * N + jg) * HD + 16 * w);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float4 x = va[i], y = ka[i];
+          x.x += __uint_as_float(av[4 * i]);
+          x.y += __uint_as_float(av[4 * i + 1]);
+          x.z += __uint_as_float(av[4 * i + 2]);
+          x.w += __uint_as_float(av[4 * i + 3]);
+          y.x += __uint_as_float(ak[4 * i]) * scale;
+          y.y += __uint_as_float(ak[4 * i + 1]) * scale;
+          y.z += __uint_as_float(ak[4 * i + 2]) * scale;
+          y.w += __uint_as_float(ak[4 * i + 3]) * scale;
+          va[i] = x;
+          ka[i] = y;
+        }
+      } else if (jg < N) {
         uint4* dvd = reinterpret_cast<uint4*>(dv + ((size_t)head * N + jg) * HD + 16 * w);
         uint4* dkd = reinterpret_cast<uint4*>(dk + ((size_t)head * N + jg) * HD + 16 * w);
 #pragma unroll
@@ -513,9 +532,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const uint16_t* __restrict__ q,
                    const uint16_t* __restrict__ dout, const float* __restrict__ nlse2,
-                   const float* __restrict__ delta, __nv_bfloat16* __restrict__ dq, int N, int BH,
-                   int causal, float scale, float scale_log2, const int* __restrict__ info,
-                   unsigned* __restrict__ err) {
+                   const float* __restrict__ delta, __nv_bfloat16* __restrict__ dq,
+                   float* __restrict__ dq_acc, int N, int BH, int causal, float scale,
+                   float scale_log2, const int* __restrict__ info, unsigned* __restrict__ err) {
   pdl_prologue();  // the next launch (independent outputs) overlaps this one's tail
   const int n_blocks = (N + BQ - 1) / BQ;
   const int Npad = n_blocks * BQ;
@@ -752,7 +771,19 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
       uint32_t a[16];
       tmem_ld16(tmem + lane_off + kColDQ + 16 * w, a);
       tmem_wait_ld();
-      if (ig < N) {
+      if (ig < N && dq_acc != nullptr) {
+        // accumulate mode: add this call's dq (float32) to the caller's sums
+        float4* dqa = reinterpret_cast<float4*>(dq_acc + ((size_t)head * N + ig) * HD + 16 * w);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float4 x = dqa[i];
+          x.x += __uint_as_float(a[4 * i]) * scale;
+          x.y += __uint_as_float(a[4 * i + 1]) * scale;
+          x.z += __uint_as_float(a[4 * i + 2]) * scale;
+          x.w += __uint_as_float(a[4 * i + 3]) * scale;
+          dqa[i] = x;
+        }
+      } else if (ig < N) {
         uint4* dst = reinterpret_cast<uint4*>(dq + ((size_t)head * N + ig) * HD + 16 * w);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -778,9 +809,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
 template <bool kF16>
 cudaError_t launch_bwd_instance(const void* q, const void* k, const void* v, const void* dout,
                                 const float* nlse2, const float* delta, void* dq, void* dk,
-                                void* dv, int64_t BH, int64_t N, int causal, float scale,
-                                const int* info, unsigned* err, cudaStream_t s, bool after,
-                                int* launches) {
+                                void* dv, const BwdAcc& acc, int64_t BH, int64_t N, int causal,
+                                float scale, const int* info, unsigned* err, cudaStream_t s,
+                                bool after, int* launches) {
   CUtensorMap tq, tk, tv, tdo;
   cudaError_t e;
   if ((e = make_tmap_bf16_rows(&tq, q, BH, N, BQ)) != cudaSuccess) return e;
@@ -800,15 +831,15 @@ cudaError_t launch_bwd_instance(const void* q, const void* k, const void* v, con
   const dim3 grid((unsigned)(n_blocks * BH));
   e = launch_after(after, attn_bwd_dkdv_kernel<kF16>, grid, dim3(kThreads), kSmemKV, s, tq, tk,
                    tv, tdo, nlse2, delta, static_cast<__nv_bfloat16*>(dk),
-                   static_cast<__nv_bfloat16*>(dv), (int)N, (int)BH, causal, scale,
-                   scale * kLog2e, info, err);
+                   static_cast<__nv_bfloat16*>(dv), acc.dk, acc.dv, (int)N, (int)BH, causal,
+                   scale, scale * kLog2e, info, err);
   if (e != cudaSuccess) return e;
   *launches += 1;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   e = launch_after(true, attn_bwd_dq_kernel<kF16>, grid, dim3(kThreads), kSmemQ, s, tk, tv,
                    static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(dout), nlse2,
-                   delta, static_cast<__nv_bfloat16*>(dq), (int)N, (int)BH, causal, scale,
-                   scale * kLog2e, info, err);
+                   delta, static_cast<__nv_bfloat16*>(dq), acc.dq, (int)N, (int)BH, causal,
+                   scale, scale * kLog2e, info, err);
   if (e != cudaSuccess) return e;
   *launches += 1;
   return cudaGetLastError();
@@ -818,16 +849,16 @@ cudaError_t launch_bwd_instance(const void* q, const void* k, const void* v, con
 
 cudaError_t launch_attn_bwd_tc(const BwdOperands& f16, const BwdOperands& bf16,
                                const float* nlse2, const float* delta, void* dq, void* dk,
-                               void* dv, int64_t B, int64_t H, int64_t N, int causal,
-                               float scale, const int* info, unsigned* err, cudaStream_t s,
-                               int* launches) {
+                               void* dv, const BwdAcc& acc, int64_t B, int64_t H, int64_t N,
+                               int causal, float scale, const int* info, unsigned* err,
+                               cudaStream_t s, int* launches) {
   const int64_t BH = B * H;
   cudaError_t e = launch_bwd_instance<true>(f16.q, f16.k, f16.v, f16.dout, nlse2, delta, dq, dk,
-                                            dv, BH, N, causal, scale, info, err, s, false,
+                                            dv, acc, BH, N, causal, scale, info, err, s, false,
                                             launches);
   if (e != cudaSuccess) return e;
   return launch_bwd_instance<false>(bf16.q, bf16.k, bf16.v, bf16.dout, nlse2, delta, dq, dk, dv,
-                                    BH, N, causal, scale, info, err, s, true, launches);
+                                    acc, BH, N, causal, scale, info, err, s, true, launches);
 }
 
 }  // namespace swa

@@ -116,7 +116,32 @@ attn_merge_kernel(const void* __restrict__ out_part, const float* __restrict__ l
   if (out_final != nullptr) Vec8<T>::store(out_final, row, part, a);
 }
 
+// float32 -> bf16 (round to nearest even), eight values per thread.
+__global__ void __launch_bounds__(256)
+f32_to_bf16_kernel(const float4* __restrict__ src, uint4* __restrict__ dst, int64_t n8) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 a = src[2 * i], b = src[2 * i + 1];
+  const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t w[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * e], x[2 * e + 1]);
+    w[e] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 }  // namespace
+
+cudaError_t launch_f32_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t s,
+                               int* launches) {
+  const int64_t n8 = n / 8;
+  f32_to_bf16_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(
+      reinterpret_cast<const float4*>(src), static_cast<uint4*>(dst), n8);
+  *launches += 1;
+  return cudaGetLastError();
+}
 
 cudaError_t launch_attn_merge(swa_dtype dt, const void* out_part, const float* lse_part,
                               float* out_acc, float* lse_acc, void* out_final, int64_t rows,

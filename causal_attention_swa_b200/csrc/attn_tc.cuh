@@ -72,11 +72,19 @@ struct BwdOperands {
 // read `f16` (copies), the others `bf16`.  Four launches.  nlse2 = -lse *
 // log2 e and delta are [BH][Npad] float32; info holds four int32 per head
 // (non-finite flags of V and dout, largest exponents of V, Q/K and dout).
+// Accumulate mode of the backward (all null: write bf16 dq, dk, dv): float32
+// [BH][N][64] sums to which each call adds its dq, dk, dv instead.
+struct BwdAcc {
+  float* dq = nullptr;
+  float* dk = nullptr;
+  float* dv = nullptr;
+};
+
 cudaError_t launch_attn_bwd_tc(const BwdOperands& f16, const BwdOperands& bf16,
                                const float* nlse2, const float* delta, void* dq, void* dk,
-                               void* dv, int64_t B, int64_t H, int64_t N, int causal,
-                               float scale, const int* info, unsigned* err, cudaStream_t s,
-                               int* launches);
+                               void* dv, const BwdAcc& acc, int64_t B, int64_t H, int64_t N,
+                               int causal, float scale, const int* info, unsigned* err,
+                               cudaStream_t s, int* launches);
 
 }  // namespace swa
 

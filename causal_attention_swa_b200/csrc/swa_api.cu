@@ -241,18 +241,31 @@ size_t swa_attn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D, s
   return bwd_ws(B, H, N, D, dt).total;
 }
 
-swa_status swa_attn_bwd(const void* q, const void* k, const void* v, const void* out,
-                        const void* dout, const float* lse, void* dq, void* dk, void* dv,
-                        int64_t B, int64_t H, int64_t N, int64_t D, int causal, swa_dtype dt,
-                        void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The backward with bf16 (or float32) dq, dk, dv, or -- acc non-null, bf16
+// only -- with dq, dk, dv added to float32 sums.
+swa_status attn_bwd_impl(const void* q, const void* k, const void* v, const void* out,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                         const swa::BwdAcc& acc, int64_t B, int64_t H, int64_t N, int64_t D,
+                         int causal, swa_dtype dt, void* workspace, size_t workspace_bytes,
+                         void* stream) {
   t_msg[0] = 0;
   t_launches = 0;
   swa_status st = check_attn_shape(B, H, N, D, dt);
   if (st != SWA_OK) return st;
+  const bool accumulate = acc.dq != nullptr;
+  if (accumulate && dt != SWA_BF16)
+    return fail(SWA_ERR_UNSUPPORTED, "the accumulating backward takes bf16 inputs only");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
-      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+      !aligned16(lse))
     return fail(SWA_ERR_INVALID_ARGUMENT,
-                "q, k, v, out, dout, lse, dq, dk, dv must be non-null and 16-byte aligned");
+                "q, k, v, out, dout, lse must be non-null and 16-byte aligned");
+  if (accumulate ? (!aligned16(acc.dq) || !aligned16(acc.dk) || !aligned16(acc.dv))
+                 : (!aligned16(dq) || !aligned16(dk) || !aligned16(dv)))
+    return fail(SWA_ERR_INVALID_ARGUMENT, "dq, dk, dv must be non-null and 16-byte aligned");
   const BwdWs ws = bwd_ws(B, H, N, D, dt);
   if (!aligned16(workspace) || workspace_bytes < ws.total)
     return fail(SWA_ERR_INVALID_ARGUMENT, "workspace must be 16-byte aligned and >= %zu bytes",
@@ -287,12 +300,42 @@ swa_status swa_attn_bwd(const void* q, const void* k, const void* v, const void*
       ProfScope ps(SWA_KERNEL_ATTN_BWD, s);
       e = swa::launch_attn_bwd_tc(swa::BwdOperands{w.q16, w.k16, w.v16, w.do16},
                                   swa::BwdOperands{q, k, v, dout}, w.nlse2, w.delta, dq, dk, dv,
-                                  B, H, N, c, scale, w.info, err, s, &launches);
+                                  acc, B, H, N, c, scale, w.info, err, s, &launches);
     }
     if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_tc");
   }
   t_launches = launches;
   return SWA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+swa_status swa_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                        int64_t B, int64_t H, int64_t N, int64_t D, int causal, swa_dtype dt,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  return attn_bwd_impl(q, k, v, out, dout, lse, dq, dk, dv, swa::BwdAcc{}, B, H, N, D, causal,
+                       dt, workspace, workspace_bytes, stream);
+}
+
+swa_status swa_attn_bwd_acc(const void* q, const void* k, const void* v, const void* out,
+                            const void* dout, const float* lse, float* dq_acc, float* dk_acc,
+                            float* dv_acc, int64_t B, int64_t H, int64_t N, int64_t D,
+                            int causal, swa_dtype dt, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  if (dq_acc == nullptr || dk_acc == nullptr || dv_acc == nullptr) {
+    t_msg[0] = 0;
+    t_launches = 0;
+    return fail(SWA_ERR_INVALID_ARGUMENT, "dq_acc, dk_acc, dv_acc must be non-null");
+  }
+  swa::BwdAcc acc;
+  acc.dq = dq_acc;
+  acc.dk = dk_acc;
+  acc.dv = dv_acc;
+  return attn_bwd_impl(q, k, v, out, dout, lse, nullptr, nullptr, nullptr, acc, B, H, N, D,
+                       causal, dt, workspace, workspace_bytes, stream);
 }
 
 size_t swa_attn_grad_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D, swa_dtype dt) {
@@ -358,7 +401,7 @@ swa_status swa_attn_grad(const void* q, const void* k, const void* v, void* out,
       ProfScope ps(SWA_KERNEL_ATTN_BWD, s);
       e = swa::launch_attn_bwd_tc(swa::BwdOperands{w.q16, w.k16, w.v16, w.do16},
                                   swa::BwdOperands{q, k, v, out}, w.nlse2, w.delta, dq, dk, dv,
-                                  B, H, N, c, scale, w.info, err, s, &launches);
+                                  swa::BwdAcc{}, B, H, N, c, scale, w.info, err, s, &launches);
     }
     if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_tc");
   }
@@ -513,6 +556,22 @@ swa_status swa_attn_merge(const void* out_part, const float* lse_part, float* ou
                                          rows, first ? 1 : 0, static_cast<cudaStream_t>(stream),
                                          &launches);
   if (e != cudaSuccess) return cuda_fail(e, "attn_merge");
+  t_launches = launches;
+  return SWA_OK;
+}
+
+swa_status swa_f32_to_bf16(const float* src, void* dst, int64_t n, void* stream) {
+  t_msg[0] = 0;
+  t_launches = 0;
+  if (n < 8 || n % 8 != 0 || n > ((int64_t)1 << 40))
+    return fail(SWA_ERR_INVALID_ARGUMENT, "n must be a positive multiple of 8 (got %lld)",
+                (long long)n);
+  if (!aligned16(src) || !aligned16(dst))
+    return fail(SWA_ERR_INVALID_ARGUMENT, "src, dst must be non-null and 16-byte aligned");
+  int launches = 0;
+  cudaError_t e = swa::launch_f32_to_bf16(src, dst, n, static_cast<cudaStream_t>(stream),
+                                          &launches);
+  if (e != cudaSuccess) return cuda_fail(e, "f32_to_bf16");
   t_launches = launches;
   return SWA_OK;
 }

@@ -71,6 +71,10 @@ cudaError_t launch_attn_merge(swa_dtype dt, const void* out_part, const float* l
                               float* out_acc, float* lse_acc, void* out_final, int64_t rows,
                               int first, cudaStream_t s, int* launches);
 
+// float32 -> bf16 of n values (n a multiple of 8; 16-byte aligned buffers).
+cudaError_t launch_f32_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t s,
+                               int* launches);
+
 // The prep pass over [BH][N][64] bf16 tensors: f16 copies of v (and of q and
 // k if q is non-null, of dout if non-null) into v16 (q16, k16, do16); with
 // `out` non-null (dout then too) delta = dout . out and nlse2 = -lse log2 e

@@ -1,4 +1,4 @@
-"""Sequence-sharded causal attention forward over W ranks (ring).
+"""Sequence-sharded causal attention over W ranks (ring): forward and backward.
 
 For sequences too long for one GPU's share of a step, the N tokens of each
 (b, h) are split into 2W chunks of C = N / (2W) tokens, and rank r holds
@@ -17,9 +17,18 @@ view's weighted average over the union of disjoint key sets, computed
 exactly from the sets' own averages and normalisers) into a float32
 accumulator; the last partial of a query chunk also writes the bf16 result.
 
+The backward (the GRADIENT query over the sharded sequence) walks the same
+plan: each (query chunk, key chunk) pair adds its dq, dk, dv terms to
+float32 sums (swa_attn_bwd_acc, with the merged forward's out and lse, so P
+and delta are the whole row's); dq stays with its rank, while each key
+chunk's dk, dv sums travel around the ring with its K and V and reach their
+owner after the last step.  Float32 sums, not bf16 partials: sum_j dS_ij
+k_j cancels across key chunks.
+
 Every arithmetic step runs in libswa.so's kernels; this module only
-allocates, orders the calls and moves K/V with torch.distributed
-point-to-point operations (NCCL on GPUs), which overlap the compute.
+allocates, orders the calls and moves K/V (and the dk, dv sums) with
+torch.distributed point-to-point operations (NCCL on GPUs); K/V transfers
+overlap the compute.
 """
 from __future__ import annotations
 
@@ -147,3 +156,76 @@ def ring_attn_fwd(qa, qb, ka, kb, va, vb, group=None, step_fn=None):
         if s + 1 < world:
             kv, nxt = nxt, kv
     return None if state is None else state.result()
+
+
+@dataclass
+class RingBackwardState:
+    """One rank's backward: float32 dq sums per held query chunk, and the
+    plan of (query slot, key slot, mode) sub-calls per ring step."""
+    q: tuple[torch.Tensor, torch.Tensor]
+    out: tuple[torch.Tensor, torch.Tensor]
+    dout: tuple[torch.Tensor, torch.Tensor]
+    lse: tuple[torch.Tensor, torch.Tensor]
+    rank: int
+    world: int
+
+    def __post_init__(self):
+        self.dq_acc = [torch.zeros(t.shape, dtype=torch.float32, device=t.device) for t in self.q]
+        self.plan = plan(self.rank, self.world)
+
+    def step(self, s: int, kv: torch.Tensor, dkv: torch.Tensor) -> None:
+        """Ring step s: kv = stack(k0, k1, v0, v1) of rank (rank - s) mod world,
+        dkv = the float32 sums (dk0, dk1, dv0, dv1) travelling with them."""
+        for qs, ks, mode in self.plan[s]:
+            swa.attn_bwd_acc(self.q[qs], kv[ks], kv[2 + ks], self.out[qs], self.dout[qs],
+                             self.lse[qs], self.dq_acc[qs], dkv[ks], dkv[2 + ks],
+                             causal=(mode == "causal"))
+
+    def dq(self):
+        return tuple(swa.f32_to_bf16(a) for a in self.dq_acc)
+
+
+def ring_attn_bwd(qa, qb, ka, kb, va, vb, outs, douts, lses, group=None, step_fn=None):
+    """Backward of ring_attn_fwd for upstream gradients douts = (dout_a, dout_b)
+    (douts = outs for loss = 1/2 sum out^2), given the forward's merged
+    outs and lses of this rank's two chunks (bf16 inputs).
+
+    Returns ((dq_a, dq_b), (dk_a, dk_b), (dv_a, dv_b)) in bf16.  `step_fn(s,
+    src, kv, dkv)`, if given, replaces the compute (for transport tests)."""
+    if dist.is_available() and dist.is_initialized():
+        rank, world = dist.get_rank(group), dist.get_world_size(group)
+    else:
+        rank, world = 0, 1
+    kv = torch.stack((ka, kb, va, vb))
+    dkv = torch.zeros(kv.shape, dtype=torch.float32, device=kv.device)
+    nxt = torch.empty_like(kv) if world > 1 else None
+    nxt_d = torch.empty_like(dkv) if world > 1 else None
+    state = None if step_fn is not None else RingBackwardState(
+        (qa, qb), tuple(outs), tuple(douts), tuple(lses), rank, world)
+    for s in range(world):
+        src = (rank - s) % world
+        reqs = []
+        if s + 1 < world:  # K/V move on while this step computes with them
+            reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, kv, (rank + 1) % world, group),
+                                           dist.P2POp(dist.irecv, nxt, (rank - 1) % world, group)])
+        if step_fn is not None:
+            step_fn(s, src, kv, dkv)
+        else:
+            state.step(s, kv, dkv)
+        for r in reqs:
+            r.wait()
+        if world > 1:
+            # the updated sums follow their K/V; after the last step they reach
+            # their owner (rank src = rank + 1 - world = rank + 1 mod world)
+            for r in dist.batch_isend_irecv([
+                    dist.P2POp(dist.isend, dkv, (rank + 1) % world, group),
+                    dist.P2POp(dist.irecv, nxt_d, (rank - 1) % world, group)]):
+                r.wait()
+            dkv, nxt_d = nxt_d, dkv
+        if s + 1 < world:
+            kv, nxt = nxt, kv
+    if state is None:
+        return None, dkv
+    dk = (swa.f32_to_bf16(dkv[0]), swa.f32_to_bf16(dkv[1]))
+    dv = (swa.f32_to_bf16(dkv[2]), swa.f32_to_bf16(dkv[3]))
+    return state.dq(), dk, dv

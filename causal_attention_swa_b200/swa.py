@@ -29,7 +29,7 @@ EXPORTS = (
     "swa_profile_kernel", "swa_attn_fwd_noalloc", "swa_selftest_wait_timeout",
     "swa_attn_grad_workspace_size", "swa_attn_grad", "swa_nw_regrid_nd",
     "swa_nw_regrid_bwd_workspace_size", "swa_nw_regrid_bwd", "swa_qkv_proj",
-    "swa_attn_merge",
+    "swa_attn_merge", "swa_attn_bwd_acc", "swa_f32_to_bf16",
 )
 (SWA_KERNEL_NONE, SWA_KERNEL_ATTN_FWD, SWA_KERNEL_ATTN_BWD, SWA_KERNEL_NW, SWA_KERNEL_NW_BWD,
  SWA_KERNEL_QKV) = range(6)
@@ -87,6 +87,10 @@ def load_library():
     lib.swa_qkv_proj.restype = I
     lib.swa_attn_merge.argtypes = [P, P, P, P, P, I64, I64, I, I, P]
     lib.swa_attn_merge.restype = I
+    lib.swa_attn_bwd_acc.argtypes = [P, P, P, P, P, P, P, P, P, I64, I64, I64, I64, I, I, P, SZ, P]
+    lib.swa_attn_bwd_acc.restype = I
+    lib.swa_f32_to_bf16.argtypes = [P, P, I64, P]
+    lib.swa_f32_to_bf16.restype = I
     lib.swa_get_device_error.argtypes = [P]
     lib.swa_get_device_error.restype = I
     lib.swa_selftest_wait_timeout.argtypes = [P]
@@ -362,6 +366,44 @@ def attn_merge(out_part, lse_part, out_acc, lse_acc, first: bool, out_final=None
                             _dtype_code(out_part), _stream_ptr(out_part.device))
     _check(st, "swa_attn_merge")
     return out_acc, lse_acc
+
+
+def attn_bwd_acc(q, k, v, out, dout, lse, dq_acc, dk_acc, dv_acc, causal: bool = True,
+                 workspace=None):
+    """swa_attn_bwd_acc: like attn_bwd (bf16 q, k, v, out, dout [B,H,N,64], lse
+    [B,H,N]) but adds dq, dk, dv to the float32 sums dq_acc, dk_acc, dv_acc."""
+    if not isinstance(q, torch.Tensor) or q.dim() != 4:
+        raise ValueError("q must be a [B, H, N, D] tensor")
+    B, H, N, D = q.shape
+    dt = _dtype_code(q)
+    shapes = {"lse": ((B, H, N), torch.float32)}
+    for n in ("dq_acc", "dk_acc", "dv_acc"):
+        shapes[n] = (q.shape, torch.float32)
+    _require_like(q, {"k": k, "v": v, "out": out, "dout": dout, "lse": lse, "dq_acc": dq_acc,
+                      "dk_acc": dk_acc, "dv_acc": dv_acc},
+                  lambda n: shapes.get(n, (q.shape, q.dtype)))
+    lib = load_library()
+    _require_cuda(q, k, v, out, dout, lse, dq_acc, dk_acc, dv_acc)
+    nbytes = attn_bwd_workspace_size(B, H, N, D, dt)
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib.swa_attn_bwd_acc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                              _ptr(dq_acc), _ptr(dk_acc), _ptr(dv_acc), B, H, N, D,
+                              int(bool(causal)), dt, _ptr(ws), nbytes, _stream_ptr(q.device))
+    _check(st, "swa_attn_bwd_acc")
+    return dq_acc, dk_acc, dv_acc
+
+
+def f32_to_bf16(src, dst=None):
+    """swa_f32_to_bf16: a float32 CUDA tensor rounded into a bf16 one."""
+    if dst is None:
+        dst = torch.empty(src.shape, dtype=torch.bfloat16, device=src.device)
+    if src.dtype != torch.float32 or dst.dtype != torch.bfloat16 or src.shape != dst.shape:
+        raise ValueError("src must be float32 and dst bfloat16 of the same shape")
+    _require_cuda(src, dst)
+    st = load_library().swa_f32_to_bf16(_ptr(src), _ptr(dst), src.numel(),
+                                        _stream_ptr(src.device))
+    _check(st, "swa_f32_to_bf16")
+    return dst
 
 
 def selftest_wait_timeout(device=None) -> None:

@@ -127,6 +127,23 @@ swa_status swa_attn_bwd(const void* q, const void* k, const void* v, const void*
                         swa_dtype dtype, void* workspace, size_t workspace_bytes,
                         void* stream);
 
+/*
+ * swa_attn_bwd that ADDS dq, dk, dv to float32 sums instead of writing them
+ * (sequence sharding: a query chunk's dq, and a key chunk's dk and dv, are
+ * sums over the chunk pairs computed by several calls; a bf16 rounding of
+ * each partial dq would lose the cancellation in sum_j dS_ij k_j).
+ *   dq_acc, dk_acc, dv_acc  [B,H,N,D] float32   (in/out)  += this call's terms
+ * Other arguments, workspace (swa_attn_bwd_workspace_size) and errors as
+ * swa_attn_bwd; bf16 inputs only (else SWA_ERR_UNSUPPORTED).  Each row of
+ * the sums is read and written once per call, without atomics: calls that
+ * share a sum must run one after another (one stream).
+ */
+swa_status swa_attn_bwd_acc(const void* q, const void* k, const void* v, const void* out,
+                            const void* dout, const float* lse, float* dq_acc, float* dk_acc,
+                            float* dv_acc, int64_t B, int64_t H, int64_t N, int64_t D,
+                            int causal, swa_dtype dtype, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
 /* Bytes of workspace swa_attn_grad needs (as swa_attn_bwd_workspace_size). */
 size_t swa_attn_grad_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D,
                                     swa_dtype dtype);
@@ -258,6 +275,14 @@ swa_status swa_qkv_proj(const void* x, const void* w, void* q, void* k, void* v,
 swa_status swa_attn_merge(const void* out_part, const float* lse_part, float* out_acc,
                           float* lse_acc, void* out_final, int64_t rows, int64_t D, int first,
                           swa_dtype dtype, void* stream);
+
+/*
+ * dst[i] = bf16(src[i]) (round to nearest even) for i < n: float32 sums
+ * (swa_attn_merge's accumulator, swa_attn_bwd_acc's) to bf16 tensors.
+ * n a positive multiple of 8; src, dst 16-byte aligned (else
+ * SWA_ERR_INVALID_ARGUMENT).  One kernel on `stream`.
+ */
+swa_status swa_f32_to_bf16(const float* src, void* dst, int64_t n, void* stream);
 
 /*
  * Synchronises `stream`, then reads and clears this device's error word.

@@ -154,6 +154,24 @@ def test_merge_argument_errors(lib):
     assert call(dt=7) == swa.SWA_ERR_INVALID_ARGUMENT
 
 
+def test_accumulating_backward_and_cast_argument_errors(lib):
+    ws = 1 << 30
+    args = [FAKE] * 9 + [1, 2, 256, 64, 1, swa.SWA_BF16, FAKE, ws, None]
+    for i in (6, 7, 8):  # a missing float32 sum
+        bad = list(args)
+        bad[i] = None
+        assert lib.swa_attn_bwd_acc(*bad) == swa.SWA_ERR_INVALID_ARGUMENT
+    f32 = list(args)
+    f32[14] = swa.SWA_F32
+    assert lib.swa_attn_bwd_acc(*f32) == swa.SWA_ERR_UNSUPPORTED
+    small = list(args)
+    small[16] = 64
+    assert lib.swa_attn_bwd_acc(*small) == swa.SWA_ERR_INVALID_ARGUMENT
+    assert lib.swa_f32_to_bf16(FAKE, FAKE, 12, None) == swa.SWA_ERR_INVALID_ARGUMENT
+    assert lib.swa_f32_to_bf16(FAKE, FAKE, 0, None) == swa.SWA_ERR_INVALID_ARGUMENT
+    assert lib.swa_f32_to_bf16(None, FAKE, 64, None) == swa.SWA_ERR_INVALID_ARGUMENT
+
+
 def test_product_path_does_not_import_the_oracle():
     """The CUDA binding never reaches the oracle (no CPU fallback)."""
     pkg = os.path.join(ROOT, "causal_attention_swa_b200")

@@ -117,3 +117,83 @@ def test_merge_of_two_key_halves_is_the_whole_row():
     check_bf16(fin, w_out[:, :, : N // 2], "merged out")
     check_bf16(acc, w_out[:, :, : N // 2], "merged accumulator")
     check_lse(lacc, w_lse[:, :, : N // 2], "merged lse")
+
+
+def _emulate_bwd(q, k, v, out, lse, dout, world):
+    """The ring backward's ranks one after another: rank r at step s works on
+    the K/V chunks (and the travelling dk, dv sums) of rank (r - s) mod W."""
+    def split(t):
+        return [ring.zigzag_split(t, r, world) for r in range(world)]
+    qs, ks, vs, os_, ds = split(q), split(k), split(v), split(out), split(dout)
+    ls = split(lse.unsqueeze(-1))
+    sums = {r: torch.zeros((4,) + ks[r][0].shape, dtype=torch.float32, device="cuda")
+            for r in range(world)}
+    dqs = []
+    for r in range(world):
+        state = ring.RingBackwardState(qs[r], os_[r], ds[r],
+                                       (ls[r][0].squeeze(-1).contiguous(),
+                                        ls[r][1].squeeze(-1).contiguous()), r, world)
+        for s in range(world):
+            src = (r - s) % world
+            state.step(s, torch.stack((ks[src][0], ks[src][1], vs[src][0], vs[src][1])),
+                       sums[src])
+        dqs.append(state.dq())
+    dks = [(swa.f32_to_bf16(sums[r][0]), swa.f32_to_bf16(sums[r][1])) for r in range(world)]
+    dvs = [(swa.f32_to_bf16(sums[r][2]), swa.f32_to_bf16(sums[r][3])) for r in range(world)]
+    torch.cuda.synchronize()
+    assert swa.get_device_error() == swa.SWA_OK
+    return tuple(ring.zigzag_join(p, world) for p in (dqs, dks, dvs))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_ring_backward_emulated_ranks_match_the_oracle(world):
+    """dq, dk, dv of loss = 1/2 sum out^2 over the sharded sequence, with the
+    ring forward's stored output as dout, against the oracle's backward at
+    that same output (the comparison of the swa_attn_bwd unit test)."""
+    (qb, kb, vb), N = _bf16_case(world, 300, seed=50 + world)
+    q, k, v = _dev(qb), _dev(kb), _dev(vb)
+    out, lse = _emulate(q, k, v, world)
+    dq, dk, dv = _emulate_bwd(q, k, v, out, lse, out, world)
+    o64 = to_f64(out)
+    w_dq, w_dk, w_dv = oracle.attn_bwd(*(inputs.bf16_to_f64(b) for b in (qb, kb, vb)), o64,
+                                       out=o64)
+    check_bf16(dq, w_dq, f"ring dq (W={world})")
+    check_bf16(dk, w_dk, f"ring dk (W={world})")
+    check_bf16(dv, w_dv, f"ring dv (W={world})")
+
+
+def test_ring_backward_driver_on_one_rank_matches_swa_attn_bwd():
+    (qb, kb, vb), N = _bf16_case(1, 640, seed=55)
+    q, k, v = _dev(qb), _dev(kb), _dev(vb)
+    out, lse = swa.attn_fwd(q, k, v, causal=True)
+    parts = [ring.zigzag_split(t, 0, 1) for t in (q, k, v, out)]
+    la, lb = ring.zigzag_split(lse.unsqueeze(-1), 0, 1)
+    lses = (la.squeeze(-1).contiguous(), lb.squeeze(-1).contiguous())
+    (dqa, dqb), (dka, dkb), (dva, dvb) = ring.ring_attn_bwd(
+        *parts[0], *parts[1], *parts[2], parts[3], parts[3], lses)
+    torch.cuda.synchronize()
+    got = [ring.zigzag_join([p], 1) for p in ((dqa, dqb), (dka, dkb), (dva, dvb))]
+    want = swa.attn_bwd(q, k, v, out, out, lse, causal=True)
+    for g, w, name in zip(got, want, ("dq", "dk", "dv")):
+        check_bf16(g, to_f64(w), f"ring driver {name} vs one call", rel=4e-2)
+    o64 = to_f64(out)
+    w_dq, w_dk, w_dv = oracle.attn_bwd(*(inputs.bf16_to_f64(b) for b in (qb, kb, vb)), o64,
+                                       out=o64)
+    for g, w, name in zip(got, (w_dq, w_dk, w_dv), ("dq", "dk", "dv")):
+        check_bf16(g, w, f"ring driver {name}")
+
+
+def test_backward_accumulate_mode_adds_to_the_sums():
+    """swa_attn_bwd_acc twice into the same float32 sums equals twice the
+    bf16 backward (within its rounding), and starts from what is there."""
+    N = 384
+    qb, kb, vb = inputs.attn_bf16_batch(1, 2, N, seed=56)
+    q, k, v = _dev(qb), _dev(kb), _dev(vb)
+    out, lse = swa.attn_fwd(q, k, v, causal=True)
+    ref = [to_f64(t) for t in swa.attn_bwd(q, k, v, out, out, lse, causal=True)]
+    sums = [torch.full(q.shape, 0.5, dtype=torch.float32, device="cuda") for _ in range(3)]
+    for _ in range(2):
+        swa.attn_bwd_acc(q, k, v, out, out, lse, *sums, causal=True)
+    torch.cuda.synchronize()
+    for s_, r, name in zip(sums, ref, ("dq", "dk", "dv")):
+        check_bf16((s_.double().cpu().numpy() - 0.5) / 2.0, r, f"accumulated {name}")

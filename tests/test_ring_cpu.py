@@ -95,3 +95,45 @@ def test_ring_delivers_each_ranks_kv_in_order_over_gloo(world):
             assert src == (r - s) % world
             # k chunks 0, 1 and v chunks 0, 1 of rank src (tags 2..5)
             assert tags == [100.0 * src + j for j in range(2, 6)]
+
+
+def _bwd_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    shape = (1, 2, 3, 64)
+    t = [torch.full(shape, float(100 * rank + j)) for j in range(6)]
+    seen = []
+
+    def add(s, src, kv, dkv):
+        seen.append((s, src, float(kv[0].flatten()[0])))
+        dkv += 1000.0 * src + rank + 1  # tagged by the sums' owner and this rank
+
+    _, dkv = ring.ring_attn_bwd(t[0], t[1], t[2], t[3], t[4], t[5], None, None, None,
+                                step_fn=add)
+    q.put((rank, seen, [float(dkv[i].flatten()[0]) for i in range(4)]))
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_ring_backward_sums_visit_every_rank_and_return_home_over_gloo(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_bwd_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = {r: (seen, sums) for r, seen, sums in (q.get(timeout=120) for _ in procs)}
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for r in range(world):
+        seen, sums = results[r]
+        assert [(s, src) for s, src, _ in seen] == [(s, (r - s) % world) for s in range(world)]
+        assert [k0 for _, _, k0 in seen] == [100.0 * ((r - s) % world) + 2 for s in range(world)]
+        # rank r ends with its own chunks' sums: one term from every rank
+        want = world * 1000.0 * r + world * (world + 1) / 2
+        assert sums == [want] * 4
