@@ -94,7 +94,6 @@ constexpr int kThreads = 576;
 constexpr int kQStages = 4;             // dkdv's Q/dO ring depth
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDP = 256;
-constexpr int kHeadGroup = 4;           // heads scheduled together (their operands share L2)
 
 // Per-head information (four int32 per head, from the prep pass):
 //   [0] bit 0: V holds an infinity or NaN; bit 1: dout does
@@ -129,17 +128,18 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
-// Block -> (head, block index) in groups of kHeadGroup heads; inside a
+// Block -> (head, block index) in groups of `group_heads` heads (head_group()
+// on the host: the operands a head's blocks stream stay in L2); inside a
 // group the heaviest blocks first, heads interleaved.  heavy_low: block
 // index 0 is the heaviest (dkdv: key block 0 meets every query block);
 // else the last one is (dq: the last query block sees every key block).
-__device__ __forceinline__ void block_order(int n_blocks, int BH, bool heavy_low, int* head,
-                                            int* blk) {
-  const int group = blockIdx.x / (kHeadGroup * n_blocks);
-  const int g_heads = min(kHeadGroup, BH - group * kHeadGroup);
-  const int r = blockIdx.x - group * kHeadGroup * n_blocks;
+__device__ __forceinline__ void block_order(int n_blocks, int BH, int group_heads,
+                                            bool heavy_low, int* head, int* blk) {
+  const int group = blockIdx.x / (group_heads * n_blocks);
+  const int g_heads = min(group_heads, BH - group * group_heads);
+  const int r = blockIdx.x - group * group_heads * n_blocks;
   const int rank = r / g_heads;
-  *head = group * kHeadGroup + r % g_heads;
+  *head = group * group_heads + r % g_heads;
   *blk = heavy_low ? rank : n_blocks - 1 - rank;
 }
 
@@ -179,13 +179,14 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ nlse2,
                      const float* __restrict__ delta, __nv_bfloat16* __restrict__ dk,
                      __nv_bfloat16* __restrict__ dv, float* __restrict__ dk_acc,
-                     float* __restrict__ dv_acc, int N, int BH, int causal, float scale,
+                     float* __restrict__ dv_acc, int N, int BH, int group_heads, int causal,
+                     float scale,
                      float scale_log2, const int* __restrict__ info, unsigned* __restrict__ err) {
   pdl_prologue();  // the next launch (independent outputs) overlaps this one's tail
   const int n_blocks = (N + BQ - 1) / BQ;
   const int Npad = n_blocks * BQ;
   int head, jb;
-  block_order(n_blocks, BH, true, &head, &jb);
+  block_order(n_blocks, BH, group_heads, true, &head, &jb);
   if (head_is_f16(info, head) != kF16) return;  // the other instance's head
   // a head with a non-finite V or dout: dV of the diagonal block reads a
   // cleaned copy of its dO (non-causal: no masked pair meets dO at all)
@@ -533,13 +534,14 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const uint16_t* __restrict__ q,
                    const uint16_t* __restrict__ dout, const float* __restrict__ nlse2,
                    const float* __restrict__ delta, __nv_bfloat16* __restrict__ dq,
-                   float* __restrict__ dq_acc, int N, int BH, int causal, float scale,
+                   float* __restrict__ dq_acc, int N, int BH, int group_heads, int causal,
+                   float scale,
                    float scale_log2, const int* __restrict__ info, unsigned* __restrict__ err) {
   pdl_prologue();  // the next launch (independent outputs) overlaps this one's tail
   const int n_blocks = (N + BQ - 1) / BQ;
   const int Npad = n_blocks * BQ;
   int head, ib;
-  block_order(n_blocks, BH, false, &head, &ib);
+  block_order(n_blocks, BH, group_heads, false, &head, &ib);
   if (head_is_f16(info, head) != kF16) return;  // the other instance's head
   const bool nonfinite = info[kInfoInts * head] != 0;  // V or dout holds an infinity or NaN
 
@@ -831,15 +833,15 @@ cudaError_t launch_bwd_instance(const void* q, const void* k, const void* v, con
   const dim3 grid((unsigned)(n_blocks * BH));
   e = launch_after(after, attn_bwd_dkdv_kernel<kF16>, grid, dim3(kThreads), kSmemKV, s, tq, tk,
                    tv, tdo, nlse2, delta, static_cast<__nv_bfloat16*>(dk),
-                   static_cast<__nv_bfloat16*>(dv), acc.dk, acc.dv, (int)N, (int)BH, causal,
-                   scale, scale * kLog2e, info, err);
+                   static_cast<__nv_bfloat16*>(dv), acc.dk, acc.dv, (int)N, (int)BH,
+                   head_group(BH, N), causal, scale, scale * kLog2e, info, err);
   if (e != cudaSuccess) return e;
   *launches += 1;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   e = launch_after(true, attn_bwd_dq_kernel<kF16>, grid, dim3(kThreads), kSmemQ, s, tk, tv,
                    static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(dout), nlse2,
-                   delta, static_cast<__nv_bfloat16*>(dq), acc.dq, (int)N, (int)BH, causal,
-                   scale, scale * kLog2e, info, err);
+                   delta, static_cast<__nv_bfloat16*>(dq), acc.dq, (int)N, (int)BH,
+                   head_group(BH, N), causal, scale, scale * kLog2e, info, err);
   if (e != cudaSuccess) return e;
   *launches += 1;
   return cudaGetLastError();

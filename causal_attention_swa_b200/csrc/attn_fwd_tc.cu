@@ -119,7 +119,6 @@ static_assert(2 * kSoftmaxRegs + kOtherRegs <= 3 * kLaunchRegs, "register split 
 constexpr int kTmaWarp = kSoftmaxWarps;
 constexpr int kMmaWarp = kSoftmaxWarps + 1;  // issuer of tile 0; kMmaWarp + 1 issues tile 1
 constexpr uint32_t kTmemCols = 512;
-constexpr int kHeadGroup = 4;                // heads scheduled together (K, V share L2)
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int kCleanWarp = kSoftmaxWarps + 3;  // warp 11
 // Per-head information (kHeadInfoInts int32 per head): bit 0 of [0] is set if
@@ -222,19 +221,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
-                   float* __restrict__ lse, int N, int BH, int n_ctiles, int causal,
+                   float* __restrict__ lse, int N, int BH, int n_ctiles, int head_group,
+                   int causal,
                    float scale_log2, const int* __restrict__ vinfo,
                    const uint4* __restrict__ vrows, int all_bf16,
                    uint16_t* __restrict__ do16, float* __restrict__ delta,
                    float* __restrict__ nlse2, unsigned* __restrict__ err) {
   pdl_prologue();  // the other instance's launch overlaps this one's tail
-  // Heads in groups of kHeadGroup, whose K and V (4 MB per head at N = 16384)
+  // Heads in groups of head_group (head_group() on the host), whose K and V
   // stay in L2 while the group's blocks run; inside a group the heaviest
   // (latest) query tiles first, heads interleaved.
-  const int group = blockIdx.x / (kHeadGroup * n_ctiles);
-  const int g_heads = min(kHeadGroup, BH - group * kHeadGroup);
-  const int rr = blockIdx.x - group * kHeadGroup * n_ctiles;
-  const int head = group * kHeadGroup + rr % g_heads;
+  const int group = blockIdx.x / (head_group * n_ctiles);
+  const int g_heads = min(head_group, BH - group * head_group);
+  const int rr = blockIdx.x - group * head_group * n_ctiles;
+  const int head = group * head_group + rr % g_heads;
   const int c = n_ctiles - 1 - rr / g_heads;
   const bool nonfinite = (vinfo[kHeadInfoInts * head] & 1) != 0;
   const bool f16_head = !all_bf16 && vinfo[kHeadInfoInts * head + 1] < kF16ExpLimit;
@@ -642,7 +642,7 @@ cudaError_t launch_fwd_instance(const CUtensorMap& tq, const CUtensorMap& tk,
   const int64_t grid = (int64_t)n_ctiles * BH;
   e = launch_after(after, attn_fwd_tc_kernel<kF16>, dim3((unsigned)grid), dim3(kThreads),
                    kSmemBytes, s, tq, tk, tv, static_cast<__nv_bfloat16*>(out), lse, (int)N,
-                   (int)BH, n_ctiles, causal, scale * kLog2e, vinfo,
+                   (int)BH, n_ctiles, head_group(BH, N), causal, scale * kLog2e, vinfo,
                    reinterpret_cast<const uint4*>(vrows), all_bf16,
                    static_cast<uint16_t*>(saved.do16), saved.delta, saved.nlse2, err);
   if (e != cudaSuccess) return e;

@@ -37,6 +37,20 @@ cudaError_t launch_after(bool after, void (*kernel)(KArgs...), dim3 grid, dim3 b
 cudaError_t make_tmap_bf16_rows(CUtensorMap* map, const void* base, int64_t BH, int64_t N,
                                 int box_rows);
 
+// Heads whose blocks are scheduled together.  Every block of a head streams
+// 256 N bytes of its 16-bit rows (K and V in the forward and dq, Q and dO
+// in dK/dV).  When all heads' rows fit in 64 MB of the 126 MB L2, one group:
+// the whole grid runs heaviest blocks first (no late group whose heavy
+// blocks form a tail).  Else groups of four heads, whose rows stay in L2
+// while the group's blocks run (groups of 16 at 2x16x16384 left the time
+// unchanged and raised DRAM traffic 1.6x).  Inside a group blocks run
+// heaviest first, heads interleaved.
+inline int head_group(int64_t BH, int64_t N) {
+  const int64_t per_head = 256 * (N > 0 ? N : 1);
+  if (BH * per_head <= (int64_t(64) << 20)) return static_cast<int>(BH);
+  return static_cast<int>(BH < 4 ? BH : 4);
+}
+
 // What the forward saves for the backward of loss = 1/2 sum out^2 (all
 // null for a plain forward): do16 [BH][N][64] f16 copy of out; delta and
 // nlse2 [BH][Npad] float32 (sum_d out_d^2 and -lse log2 e; padding rows 0
