@@ -368,7 +368,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       const bool need_mask = (causal && ib == jb) || (i0 + BQ > N) || (j0 + BK > N);
       // dP^T_i done implies S^T_i (issued before it) is done and Q_i's
       // stage (with lse and delta) has landed
-      if (!mbar_wait_parked(&sm.dp_full, it & 1, abort, err, kDevTimeoutMma)) {
+      if (!mbar_wait_spin(&sm.dp_full, it & 1, abort, err, kDevTimeoutMma)) {
         ok = false;
         break;
       }
@@ -437,13 +437,13 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       warp_arrive(&sm.sm_done);
     }
     // ---- columns 16w..16w+15 of this key's dv and dk
-    if (ok && mbar_wait_parked(&sm.acc_full, 0, abort, err, kDevTimeoutMma)) {
+    if (ok && mbar_wait_spin(&sm.acc_full, 0, abort, err, kDevTimeoutMma)) {
       fence_after_sync();
       uint32_t av[16], ak[16];
       tmem_ld16(tmem + lane_off + kColDV + 16 * w, av);
       tmem_ld16(tmem + lane_off + kColDK + 16 * w, ak);
       tmem_wait_ld();
-      if (clean_diag && mbar_wait_parked(&sm.diag_clean, 0, abort, err, kDevTimeoutOther)) {
+      if (clean_diag && mbar_wait_spin(&sm.diag_clean, 0, abort, err, kDevTimeoutOther)) {
         // merge the IEEE class of the diagonal block's rows i >= jg into dv
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -505,6 +505,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
 
 // ======================================================================= dQ
 
+// Every role of this kernel polls its barriers (mbar_wait_spin): each of
+// its waits sits on the block's critical path.
 // Q_i and dO_i, the A operands of S and dP in every key block, sit in TMEM
 // (columns [448, 480) and [480, 512), written once by the compute warps from
 // their own rows), so those MMAs read only K_j and V_j from shared memory.
@@ -589,7 +591,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
       for (int jt = 0; jt < n_k; ++jt) {
         const int s = jt % kKVStagesQ;
         const int round = jt / kKVStagesQ;
-        if (round > 0 && !mbar_wait_parked(&sm.kv_empty[s], (round - 1) & 1, abort, err,
+        if (round > 0 && !mbar_wait_spin(&sm.kv_empty[s], (round - 1) & 1, abort, err,
                                            kDevTimeoutEmpty))
           break;
         mbar_arrive_expect_tx(&sm.kv_full[s], 2 * kTileBytes);
@@ -618,10 +620,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                      first ? 0u : 1u);
       };
       auto wait_kv = [&](int jt) {
-        return mbar_wait_parked(&sm.kv_full[jt % kKVStagesQ], (jt / kKVStagesQ) & 1, abort,
+        return mbar_wait_spin(&sm.kv_full[jt % kKVStagesQ], (jt / kKVStagesQ) & 1, abort,
                                 err, kDevTimeoutFull);
       };
-      bool ok = mbar_wait_parked(&sm.qt_ready, 0, abort, err, kDevTimeoutOther) && n_k > 0 &&
+      bool ok = mbar_wait_spin(&sm.qt_ready, 0, abort, err, kDevTimeoutOther) && n_k > 0 &&
                 wait_kv(0);
       if (ok) {
         fence_after_sync();
@@ -638,12 +640,12 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
           if (!wait_kv(jt + 1)) break;
           fence_after_sync();
           issue_kk(col_s(b ^ 1), kColQ, smem_u32(sm.k[sn]));
-          if (!mbar_wait_parked(&sm.dp_free, jt & 1, abort, err, kDevTimeoutOther)) break;
+          if (!mbar_wait_spin(&sm.dp_free, jt & 1, abort, err, kDevTimeoutOther)) break;
           fence_after_sync();
           issue_kk(kColDP, kColDO, smem_u32(sm.v[sn]));
           mma_commit_elect(&sm.dp_full);
         }
-        if (!mbar_wait_parked(&sm.sm_done, jt & 1, abort, err, kDevTimeoutOther)) break;
+        if (!mbar_wait_spin(&sm.sm_done, jt & 1, abort, err, kDevTimeoutOther)) break;
         fence_after_sync();
         const uint32_t k0 = smem_u32(sm.k[st]);
         issue_dq(col_s(b), k0, jt == 0);
@@ -695,7 +697,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
       const int j0 = jt * BK;
       const bool need_mask = (causal && jt == ib) || (j0 + BK > N) || (i0 + BQ > N);
       // dP_jt done implies S_jt (issued before it) is done
-      if (!mbar_wait_parked(&sm.dp_full, jt & 1, abort, err, kDevTimeoutMma)) {
+      if (!mbar_wait_spin(&sm.dp_full, jt & 1, abort, err, kDevTimeoutMma)) {
         ok = false;
         break;
       }
@@ -768,7 +770,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
       warp_arrive(&sm.sm_done);
     }
     // ---- columns 16w..16w+15 of this query's dq
-    if (ok && mbar_wait_parked(&sm.acc_full, 0, abort, err, kDevTimeoutMma)) {
+    if (ok && mbar_wait_spin(&sm.acc_full, 0, abort, err, kDevTimeoutMma)) {
       fence_after_sync();
       uint32_t a[16];
       tmem_ld16(tmem + lane_off + kColDQ + 16 * w, a);

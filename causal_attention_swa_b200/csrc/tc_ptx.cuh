@@ -112,6 +112,24 @@ __device__ __forceinline__ bool mbar_wait_parked(uint64_t* bar, uint32_t parity,
   }
 }
 
+// The same wait polling without the suspend hint, for warps whose wake-up
+// sits on the critical path (the backward's compute warps waiting for an MMA
+// result while the other warps of their scheduler wait on the same phase).
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort, unsigned* err,
+                                               unsigned code) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      atomicCAS(err, 0u, code);
+      *abort = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
 // ----------------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
