@@ -39,8 +39,9 @@
 // pv_done[t]; the softmax warps wait on pv_done before they rescale O_t or
 // overwrite P_t, and store P_t only after computing all of it, by which
 // time O_t += P_t,j-1 V_j-1 has long finished.
-// Every wait parks the waiting warp (try_wait with a suspend hint), so idle
-// roles take no issue slots from the softmax warps that share a scheduler.
+// Every wait polls its barrier (try_wait without a suspend hint): a parked
+// warp wakes late enough to cost the forward about 2%, and the polls of the
+// idle roles did not slow the softmax warps that share their schedulers.
 // At D = 64 the exponentials bound the kernel: a score costs one MUFU ex2
 // (16 per clock per SM) and 4 * 64 MMA flops (about 8000 per clock per SM),
 // so ex2 time is about twice the MMA time.  A warp whose ex2 loop runs over
@@ -309,7 +310,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         bool ok = true;
         for (int t = 0; t < 2 && ok && round > 0; ++t)
           if (j - kStages < n_t[t])
-            ok = mbar_wait_parked(&sm.kv_empty[t][s], (round - 1) & 1, abort, err,
+            ok = mbar_wait_spin(&sm.kv_empty[t][s], (round - 1) & 1, abort, err,
                                   kDevTimeoutEmpty);
         if (!ok) break;
         mbar_arrive_expect_tx(&sm.k_full[s], kTileBytes);
@@ -345,10 +346,10 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         mma_commit_elect(&sm.kv_empty[t][j % kStages]);
       };
       auto wait_k = [&](int j) {
-        return mbar_wait_parked(&sm.k_full[j % kStages], (j / kStages) & 1, abort, err,
+        return mbar_wait_spin(&sm.k_full[j % kStages], (j / kStages) & 1, abort, err,
                                 kDevTimeoutFull);
       };
-      bool ok = n_t[t] > 0 && mbar_wait_parked(&sm.q_full, 0, abort, err, kDevTimeoutFull) &&
+      bool ok = n_t[t] > 0 && mbar_wait_spin(&sm.q_full, 0, abort, err, kDevTimeoutFull) &&
                 wait_k(0);
       if (ok) {
         fence_after_sync();
@@ -357,15 +358,15 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       for (int j = 0; ok && j < n_t[t]; ++j) {
         // S_t,j+1 as soon as the softmax warps hold S_t,j in registers
         if (j + 1 < n_t[t]) {
-          if (!mbar_wait_parked(&sm.s_free[t], j & 1, abort, err, kDevTimeoutOther) ||
+          if (!mbar_wait_spin(&sm.s_free[t], j & 1, abort, err, kDevTimeoutOther) ||
               !wait_k(j + 1))
             break;
           fence_after_sync();
           issue_s(j + 1);
         }
-        if (!mbar_wait_parked(convert ? &sm.v_ready[j % kStages] : &sm.v_full[j % kStages],
+        if (!mbar_wait_spin(convert ? &sm.v_ready[j % kStages] : &sm.v_full[j % kStages],
                               (j / kStages) & 1, abort, err, kDevTimeoutFull) ||
-            !mbar_wait_parked(&sm.p_full[t], j & 1, abort, err, kDevTimeoutOther))
+            !mbar_wait_spin(&sm.p_full[t], j & 1, abort, err, kDevTimeoutOther))
           break;
         fence_after_sync();
         issue_pv(j);
@@ -380,7 +381,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (convert) {
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % kStages;
-        if (!mbar_wait_parked(&sm.v_full[s], (j / kStages) & 1, abort, err, kDevTimeoutFull))
+        if (!mbar_wait_spin(&sm.v_full[s], (j / kStages) & 1, abort, err, kDevTimeoutFull))
           break;
         const uint4* rowmask =
             vrows != nullptr ? vrows + (size_t)head * ((N + BN - 1) / BN) + j : nullptr;
@@ -411,7 +412,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     bool s_ready = false;  // S_t,j already seen complete by the probe of tile j-1
     const float2 sc2 = make_float2(scale_log2, scale_log2);
     for (int j = 0; j < n_t[t]; ++j) {
-      if (!s_ready && !mbar_wait_parked(&sm.s_full[t], j & 1, abort, err, kDevTimeoutMma)) {
+      if (!s_ready && !mbar_wait_spin(&sm.s_full[t], j & 1, abort, err, kDevTimeoutMma)) {
         ok = false;
         break;
       }
@@ -470,7 +471,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       if (j > 0) {
         if (!pv_ready &&
-            !mbar_wait_parked(&sm.pv_done[t], (j - 1) & 1, abort, err, kDevTimeoutMma)) {
+            !mbar_wait_spin(&sm.pv_done[t], (j - 1) & 1, abort, err, kDevTimeoutMma)) {
           ok = false;
           break;
         }
@@ -525,7 +526,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       l += (rsp[0].x + rsp[0].y) + (rsp[1].x + rsp[1].y);
     }
     if (ok && n_t[t] > 0 &&
-        mbar_wait_parked(&sm.pv_done[t], (n_t[t] - 1) & 1, abort, err, kDevTimeoutMma)) {
+        mbar_wait_spin(&sm.pv_done[t], (n_t[t] - 1) & 1, abort, err, kDevTimeoutMma)) {
       fence_after_sync();
       const float inv = 1.f / l;
       float o[HD];  // out_row, float32
@@ -537,7 +538,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
         for (int e = 0; e < 16; ++e) o[i * 16 + e] = __uint_as_float(u[e]) * inv;
       }
-      if (nonfinite && mbar_wait_parked(&sm.cls_done, 0, abort, err, kDevTimeoutOther)) {
+      if (nonfinite && mbar_wait_spin(&sm.cls_done, 0, abort, err, kDevTimeoutOther)) {
         // IEEE class of sum_{j in J(row)} P_ij v_jd with every P_ij > 0
         const int last = causal ? row : N - 1;
 #pragma unroll

@@ -113,8 +113,9 @@ __device__ __forceinline__ bool mbar_wait_parked(uint64_t* bar, uint32_t parity,
 }
 
 // The same wait polling without the suspend hint, for warps whose wake-up
-// sits on the critical path (the backward's compute warps waiting for an MMA
-// result while the other warps of their scheduler wait on the same phase).
+// sits on the critical path: in the attention kernels a parked warp's
+// wake-up after the phase completes delays the step that waits for it (the
+// forward's roles, the backward's compute warps, every dQ role).
 __device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity,
                                                volatile int* abort, unsigned* err,
                                                unsigned code) {
