@@ -5,15 +5,21 @@
 // x is [B*N, C] (rows = tokens), w is [3*H*64, C] (one row per output
 // feature: Wq's features h*64 + d, then Wk's, then Wv's -- the layout of a
 // linear layer's weight, so both operands are K-major).  Output tile =
-// 128 tokens x 128 features (two heads of one of q, k, v); the K loop walks
-// C in steps of 64 (one 128-byte swizzle row per operand row).
+// 128 tokens x 256 features (four heads of one of q, k, v); the K loop walks
+// C in steps of 64 (one 128-byte swizzle row per operand row).  N = 256
+// because shared memory carries both the MMA's operand reads and the TMA
+// writes that refill the stages, 128 bytes per clock in all: per tensor-pipe
+// cycle an N = 128 product needs 128 bytes of reads and 128 of writes, an
+// N = 256 one 96 and 96, which lifts that bound from one half of the tensor
+// peak to two thirds.
 //
-// Block = 6 warps: warp 0 TMA producer (x and w tiles into a 3-stage ring),
+// Block = 6 warps: warp 0 TMA producer (x and w tiles into a 2-stage ring),
 // warp 1 MMA issuer (one elected lane) and TMEM owner, warps 2-5 epilogue
 // (a warp reaches the TMEM lanes of its subpartition, 32 (w mod 4)..; lane =
-// token; each thread converts its token's 128 features to bf16 and stores
-// two 128-byte head rows).  Three stages of 32 KB keep two blocks per SM,
-// so one block's epilogue runs under the other's main loop.  Rows past B*N and features past 3*H*64 read as zeros
+// token; each thread converts its token's 256 features to bf16 and stores
+// four 128-byte head rows).  Two stages of 48 KB keep two blocks per SM
+// (and their 2 x 256 TMEM columns), so one block's epilogue runs under the
+// other's main loop.  Rows past B*N and features past 3*H*64 read as zeros
 // (TMA fill) and are not written.  Every wait is bounded (device error word).
 #include <cudaTypedefs.h>
 
@@ -26,16 +32,16 @@ namespace {
 using namespace tc;
 
 constexpr int TM = 128;                  // tokens per tile (MMA M)
-constexpr int TN = 128;                  // features per tile (MMA N)
+constexpr int TN = 256;                  // features per tile (MMA N)
 constexpr int TK = 64;                   // input channels per stage
 constexpr int HD = 64;
-constexpr int kStages = 3;
+constexpr int kStages = 2;
 constexpr int kTileBytes = TM * TK * 2;  // 16 KB
 constexpr int kThreads = 192;
 
 struct __align__(1024) SmemP {
   uint8_t x[kStages][kTileBytes];
-  uint8_t w[kStages][kTileBytes];
+  uint8_t w[kStages][2 * kTileBytes];  // 256 feature rows: two 128-row loads
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t acc_full;
@@ -84,9 +90,10 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         if (round > 0 &&
             !mbar_wait_parked(&sm.empty[s], (round - 1) & 1, abort, err, kDevTimeoutEmpty))
           break;
-        mbar_arrive_expect_tx(&sm.full[s], 2 * kTileBytes);
+        mbar_arrive_expect_tx(&sm.full[s], 3 * kTileBytes);
         tma_load_3d(sm.x[s], &tm_x, &sm.full[s], kt * TK, m0, 0);
         tma_load_3d(sm.w[s], &tm_w, &sm.full[s], kt * TK, f0, 0);
+        tma_load_3d(sm.w[s] + kTileBytes, &tm_w, &sm.full[s], kt * TK, f0 + 128, 0);
       }
     }
     __syncwarp();
@@ -122,7 +129,7 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       const int b = m / N, n = m - b * N;
       const int per = H * HD;  // features of each of q, k, v
 #pragma unroll
-      for (int g = 0; g < TN / HD; ++g) {  // two 64-feature groups: one head each
+      for (int g = 0; g < TN / HD; ++g) {  // four 64-feature groups: one head each
         uint32_t packed[HD / 2];
 #pragma unroll
         for (int i = 0; i < HD / 16; ++i) {
