@@ -1,8 +1,10 @@
 """GPU parity of the QKV projection in front of attention ("Wiki notes",
 page 5, mini_attention: Q = x Wq, K = x Wk, V = x Wv) through the C ABI,
 against the float64 oracle (x w^T and the head split), element by element:
-ragged token counts, an odd head count (a tile that straddles q and k), and
-the projection of the 2 x 16384-token, 16-head workload (C = 1024).
+ragged token counts, an odd head count (a tile that straddles q and k), a
+case with several tiles per block of the persistent grid and ragged edges
+in both directions, and the projection of the 2 x 16384-token, 16-head
+workload (C = 1024).
 Tolerance: the bf16 per-row bound of tests/_compare.py."""
 import numpy as np
 import pytest
@@ -38,6 +40,13 @@ def test_qkv_projection_small(B, N, C, H):
 
 def test_qkv_projection_b2_n16384_c1024_h16():
     check(2, 16384, 1024, 16, seed=6)
+
+
+def test_qkv_projection_many_tiles_per_block_with_ragged_edges():
+    # 20000 tokens (157 token tiles, the last 32 rows) x 960 features (4
+    # feature tiles, the last 192 wide): 628 tiles, so every block of the
+    # persistent grid takes several and both TMEM accumulators take turns
+    check(1, 20000, 128, 5, seed=7)
 
 
 def test_qkv_projection_rejects_unsupported_shapes():
