@@ -592,7 +592,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
         const int s = jt % kKVStagesQ;
         const int round = jt / kKVStagesQ;
         if (round > 0 && !mbar_wait_spin(&sm.kv_empty[s], (round - 1) & 1, abort, err,
-                                           kDevTimeoutEmpty))
+                                         kDevTimeoutEmpty))
           break;
         mbar_arrive_expect_tx(&sm.kv_full[s], 2 * kTileBytes);
         tma_load_3d(sm.k[s], &tm_k, &sm.kv_full[s], 0, jt * BK, head);
@@ -621,7 +621,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
       };
       auto wait_kv = [&](int jt) {
         return mbar_wait_spin(&sm.kv_full[jt % kKVStagesQ], (jt / kKVStagesQ) & 1, abort,
-                                err, kDevTimeoutFull);
+                              err, kDevTimeoutFull);
       };
       bool ok = mbar_wait_spin(&sm.qt_ready, 0, abort, err, kDevTimeoutOther) && n_k > 0 &&
                 wait_kv(0);

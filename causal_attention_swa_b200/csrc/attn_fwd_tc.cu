@@ -311,7 +311,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int t = 0; t < 2 && ok && round > 0; ++t)
           if (j - kStages < n_t[t])
             ok = mbar_wait_spin(&sm.kv_empty[t][s], (round - 1) & 1, abort, err,
-                                  kDevTimeoutEmpty);
+                                kDevTimeoutEmpty);
         if (!ok) break;
         mbar_arrive_expect_tx(&sm.k_full[s], kTileBytes);
         tma_load_3d(sm.k[s], &tm_k, &sm.k_full[s], 0, j * BN, head);
@@ -347,7 +347,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       };
       auto wait_k = [&](int j) {
         return mbar_wait_spin(&sm.k_full[j % kStages], (j / kStages) & 1, abort, err,
-                                kDevTimeoutFull);
+                              kDevTimeoutFull);
       };
       bool ok = n_t[t] > 0 && mbar_wait_spin(&sm.q_full, 0, abort, err, kDevTimeoutFull) &&
                 wait_k(0);
@@ -365,7 +365,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           issue_s(j + 1);
         }
         if (!mbar_wait_spin(convert ? &sm.v_ready[j % kStages] : &sm.v_full[j % kStages],
-                              (j / kStages) & 1, abort, err, kDevTimeoutFull) ||
+                            (j / kStages) & 1, abort, err, kDevTimeoutFull) ||
             !mbar_wait_spin(&sm.p_full[t], j & 1, abort, err, kDevTimeoutOther))
           break;
         fence_after_sync();
