@@ -293,8 +293,9 @@ swa_status swa_get_device_error(void* stream);
 
 /*
  * Diagnostic of the device-side failure path: enqueues on `stream` one small
- * kernel whose bounded waits (the same code every tensor-core kernel's
- * waits use) run out, since nothing arrives at the barriers they wait on.
+ * kernel whose bounded waits (both forms the tensor-core kernels use: parked
+ * with a suspend hint, and polling) run out, since nothing arrives at the
+ * barriers they wait on.
  * The kernel exits normally after about 2 s of SM clock; a following
  * swa_get_device_error() reports SWA_ERR_DEVICE_TIMEOUT and clears the
  * word, and the context stays usable.  Returns SWA_OK once enqueued, or

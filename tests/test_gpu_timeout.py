@@ -1,5 +1,6 @@
 """Failure detection on the GPU without a fault: a kernel whose bounded waits
-run out (nothing arrives at its barriers) leaves SWA_ERR_DEVICE_TIMEOUT in the
+(parked and polling, one block each) run out (nothing arrives at their
+barriers) leaves SWA_ERR_DEVICE_TIMEOUT in the
 device error word, the word is cleared once read, and the context stays
 usable: an attention call afterwards still matches the oracle."""
 import numpy as np
